@@ -1,0 +1,300 @@
+"""Pins for the fp64 oracle: it is checked against things other than itself.
+
+Each test ties one part of the oracle to something the pages or mathematics
+fix: brute-force deletion, closed forms of special cases, invariants, textbook
+routines.  See the oracle package docstring for which test pins which function.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import bruteforce
+from kv_cache_eviction_scores_b200 import workloads as W
+
+from conftest import GOLDEN
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _np(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---- the closed form against actual deletion (core formula; the write-up's
+#      independent delete-and-re-softmax check) -----------------------------
+
+@pytest.mark.parametrize("seed", [42, 43, 44])
+def test_closed_form_equals_deletion_on_protocol_shapes(seed):
+    proto = _load("writeup_protocol.json")
+    spec = W.config_spec(0)
+    assert (spec.B, spec.Hq, spec.Hkv, spec.d, spec.window) == (
+        proto["batch"], proto["query_heads"], proto["kv_heads"], proto["head_dim"],
+        proto["window"])
+    assert spec.lengths[0] == proto["history_slots"] + proto["window"]
+    assert spec.lengths[0] - spec.keep[0] == proto["evict"]
+    wl = W.generate(spec, seed)
+    raw, _, _, st, _ = oracle.raw_scores(wl.q, wl.k, wl.v, wl.lengths)
+    assert st == oracle.OK
+    bf = bruteforce.raw_scores(_np(wl.q.double()), _np(wl.k.double()), _np(wl.v.double()),
+                               wl.lengths)
+    m = np.isfinite(bf)
+    err = np.abs(raw[m] - bf[m])
+    # Same order as the page's 5.55e-16 largest error (its inputs differ).
+    assert err.max() <= 4 * proto["max_abs_err_closed_form_vs_deletion"]
+    assert np.all(err <= 1e-12 * np.abs(bf[m]) + 1e-15)
+
+
+def test_closed_form_equals_deletion_on_random_tiny_shapes():
+    rng = torch.Generator().manual_seed(7)
+    for i in range(30):
+        spec = W.random_spec(rng, max_n=30)
+        wl = W.generate(spec, 1000 + i)
+        raw, _, _, st, _ = oracle.raw_scores(wl.q, wl.k, wl.v, wl.lengths)
+        assert st == oracle.OK
+        bf = bruteforce.raw_scores(_np(wl.q.double()), _np(wl.k.double()),
+                                   _np(wl.v.double()), wl.lengths)
+        assert np.array_equal(np.isnan(raw), np.isnan(bf))
+        m = ~np.isnan(bf)
+        assert np.all(np.abs(raw[m] - bf[m]) <= 1e-11 * np.abs(bf[m]) + 1e-14), spec
+
+
+# ---- closed forms of special cases --------------------------------------
+
+def test_uniform_attention_closed_form():
+    """q = 0: p_j = 1/N_t over the N_t = P_t + 1 visible keys, a_t = their mean,
+    p/(1-p) = 1/(N_t - 1), so s_j = sum_{t: P_t >= j} ||mean_t - v_j||^2 / (N_t-1)^2."""
+    g = torch.Generator().manual_seed(3)
+    B, Hkv, G, w, d, L = 1, 2, 2, 4, 5, 17
+    q = torch.zeros(B, Hkv * G, w, d, dtype=torch.float64)
+    k = torch.randn(B, Hkv, L, d, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, L, d, generator=g, dtype=torch.float64)
+    raw, _, _, st, _ = oracle.raw_scores(q, k, v, [L])
+    assert st == oracle.OK
+    vv = v.numpy()
+    for hq in range(Hkv * G):
+        h = hq // G
+        expect = np.zeros(L)
+        for t in range(w):
+            P = L - w + t
+            N = P + 1
+            mean = vv[0, h, :N].mean(axis=0)
+            for j in range(N):
+                expect[j] += np.sum((mean - vv[0, h, j]) ** 2) / (N - 1) ** 2
+        np.testing.assert_allclose(raw[0, hq], expect, rtol=1e-12, atol=1e-15)
+
+
+def test_golden_uniform_three_tokens():
+    gd = _load("uniform_three_tokens.json")
+    q, k, v = _np(gd["q"]), _np(gd["k"]), _np(gd["v"])
+    raw, _, _, st, _ = oracle.raw_scores(q, k, v, gd["lengths"])
+    np.testing.assert_allclose(raw[0, 0], gd["raw"], rtol=1e-14, atol=1e-15)
+    for case in gd["cases"]:
+        s = oracle.scores(q, k, v, gd["lengths"], gd["window"], case["pool"])
+        want = np.array([float(x) for x in case["scores"]])
+        np.testing.assert_allclose(s[0, 0], want, rtol=1e-14, atol=1e-15)
+        keep, ev = oracle.select(s, gd["lengths"], [case["keep"]])
+        assert keep[0, 0].tolist() == case["keep_idx"]
+        assert ev[0, 0].tolist() == case["evict_idx"]
+
+
+def test_golden_two_token_closed_form():
+    gd = _load("two_token_closed_form.json")
+    q, k, v = _np(gd["q"]), _np(gd["k"]), _np(gd["v"])
+    raw, _, _, st, _ = oracle.raw_scores(q, k, v, gd["lengths"])
+    p0 = 1.0 / (1.0 + math.exp(gd["logit_gap"]))
+    p1 = 1.0 - p0
+    np.testing.assert_allclose(raw[0, 0], [p0 * p0 * gd["sq_dist"], p1 * p1 * gd["sq_dist"]],
+                               rtol=1e-13)
+
+
+# ---- invariants ----------------------------------------------------------
+
+def test_value_scaling_scales_scores_by_c_squared():
+    wl = W.generate(W.config_spec(0), 42)
+    raw, *_ = oracle.raw_scores(wl.q, wl.k, wl.v, wl.lengths)
+    raw3, *_ = oracle.raw_scores(wl.q, wl.k, wl.v.double() * 3.0, wl.lengths)
+    np.testing.assert_allclose(raw3, 9.0 * raw, rtol=1e-13)
+
+
+def test_history_permutation_permutes_scores():
+    """Every window query sees all history positions, so permuting history
+    tokens (keys and values together) permutes their raw scores."""
+    wl = W.generate(W.config_spec(0), 43)
+    L, w = wl.lengths[0], wl.spec.window
+    perm = torch.randperm(L - w, generator=torch.Generator().manual_seed(5))
+    full = torch.cat([perm, torch.arange(L - w, L)])
+    k2, v2 = wl.k.clone(), wl.v.clone()
+    k2[:, :, :L] = wl.k[:, :, full]
+    v2[:, :, :L] = wl.v[:, :, full]
+    raw, *_ = oracle.raw_scores(wl.q, wl.k, wl.v, wl.lengths)
+    raw2, *_ = oracle.raw_scores(wl.q, k2, v2, wl.lengths)
+    np.testing.assert_allclose(raw2[:, :, :L], raw[:, :, full.numpy()], rtol=1e-12)
+
+
+def test_gqa_merge_identity_for_one_query_head_per_kv_head():
+    spec = W.Spec("g1", B=2, Hq=3, Hkv=3, d=6, lengths=[20, 14], window=3, pool=1,
+                  keep=[10, 7], dtype="f32")
+    wl = W.generate(spec, 11)
+    s, merged, raw, st = oracle.scores(wl.q, wl.k, wl.v, wl.lengths, 3, 1, intermediates=True)
+    np.testing.assert_array_equal(np.isnan(merged), np.isnan(raw))
+    m = ~np.isnan(raw)
+    np.testing.assert_array_equal(merged[m], raw[m])
+
+
+def test_gqa_merge_of_duplicated_query_heads_equals_one_head():
+    spec = W.Spec("dup", B=1, Hq=6, Hkv=2, d=4, lengths=[25], window=4, pool=1, keep=[12],
+                  dtype="f32")
+    wl = W.generate(spec, 12)
+    q = wl.q.clone()
+    for h in range(2):
+        for g in range(3):
+            q[:, h * 3 + g] = wl.q[:, h * 3]
+    s, merged, raw, st = oracle.scores(q, wl.k, wl.v, wl.lengths, 4, 1, intermediates=True)
+    for h in range(2):
+        np.testing.assert_allclose(merged[0, h, :25], raw[0, h * 3, :25], rtol=1e-14)
+
+
+def test_gqa_merge_is_mean_of_group():
+    spec = W.Spec("mean", B=1, Hq=4, Hkv=2, d=4, lengths=[15], window=2, pool=1, keep=[8],
+                  dtype="f32")
+    wl = W.generate(spec, 13)
+    s, merged, raw, st = oracle.scores(wl.q, wl.k, wl.v, wl.lengths, 2, 1, intermediates=True)
+    np.testing.assert_allclose(merged[0, 0, :15], raw[0, 0:2, :15].mean(axis=0), rtol=1e-14)
+    np.testing.assert_allclose(merged[0, 1, :15], raw[0, 2:4, :15].mean(axis=0), rtol=1e-14)
+
+
+# ---- MaxPool1D and protection (Algorithm 1) ------------------------------
+
+@pytest.mark.parametrize("pool", [1, 3, 5, 7, 9])
+def test_pool_matches_sliding_max(pool):
+    rng = np.random.default_rng(pool)
+    B, Hkv, n_max, w = 2, 3, 40, 4
+    lengths = [40, 23]
+    merged = rng.integers(0, 6, size=(B, Hkv, n_max)).astype(np.float64)  # plateaus
+    out = oracle.pool_protect(merged, w, pool, lengths)
+    r = pool // 2
+    for b in range(B):
+        L = lengths[b]
+        for h in range(Hkv):
+            x = merged[b, h, :L]
+            # textbook sliding window maximum with -inf padding (numpy)
+            padded = np.concatenate([np.full(r, -np.inf), x, np.full(r, -np.inf)])
+            win = np.lib.stride_tricks.sliding_window_view(padded, pool).max(axis=1)
+            assert np.array_equal(out[b, h, : L - w], win[: L - w])
+            assert np.all(out[b, h, : L - w] >= x[: L - w])
+            assert np.all(np.isposinf(out[b, h, L - w: L]))
+            assert np.all(np.isnan(out[b, h, L:]))
+            if pool == 1:
+                assert np.array_equal(out[b, h, : L - w], x[: L - w])
+
+
+def test_window_is_protected_and_never_evicted():
+    wl = W.generate(W.config_spec(0), 44)
+    s = oracle.scores(wl.q, wl.k, wl.v, wl.lengths, 3, 3)
+    L, w = wl.lengths[0], 3
+    assert np.all(np.isposinf(s[0, :, L - w: L]))
+    keep, ev = oracle.select(s, wl.lengths, [w])  # keep only as many as the window
+    for h in range(s.shape[1]):
+        assert sorted(keep[0, h].tolist()) == list(range(L - w, L))
+        assert not set(ev[0, h].tolist()) & set(range(L - w, L))
+
+
+# ---- singular input (Algorithm 1 paragraph: rejected, no epsilon) --------
+
+def test_singular_input_is_rejected():
+    d, L, w = 8, 12, 2
+    q = torch.zeros(1, 1, w, d, dtype=torch.float64)
+    q[..., 0] = 1.0
+    k = torch.zeros(1, 1, L, d, dtype=torch.float64)
+    v = torch.randn(1, 1, L, d, generator=torch.Generator().manual_seed(1), dtype=torch.float64)
+    k[0, 0, 3, 0] = 100.0 * math.sqrt(d)  # logit 100 above every other one
+    with pytest.raises(oracle.SingularError):
+        oracle.scores(q, k, v, [L], w, 3)
+    raw, _, _, st, where = oracle.raw_scores(q, k, v, [L], raise_singular=False)
+    assert st == oracle.ERR_SINGULAR and where[3] == 3
+
+
+def test_peaked_but_nonsingular_input_is_accepted():
+    d, L, w = 8, 12, 2
+    q = torch.zeros(1, 1, w, d, dtype=torch.float64)
+    q[..., 0] = 1.0
+    k = torch.zeros(1, 1, L, d, dtype=torch.float64)
+    v = torch.randn(1, 1, L, d, generator=torch.Generator().manual_seed(1), dtype=torch.float64)
+    k[0, 0, 3, 0] = 5.0 * math.sqrt(d)  # p about 0.93, far from 1
+    s = oracle.scores(q, k, v, [L], w, 1)
+    assert np.all(np.isfinite(s[0, 0, : L - w]))
+
+
+def test_argument_errors():
+    wl = W.generate(W.config_spec(0), 42)
+    with pytest.raises(ValueError):
+        oracle.scores(wl.q, wl.k, wl.v, wl.lengths, 3, 2)      # even pool kernel
+    with pytest.raises(ValueError):
+        oracle.scores(wl.q, wl.k, wl.v, [3], 3, 3)             # L must exceed w
+    with pytest.raises(ValueError):
+        oracle.scores(wl.q, wl.k, wl.v, [23], 3, 3)            # L beyond n_max
+
+
+# ---- selection -----------------------------------------------------------
+
+def _brute_select(s, L, keep):
+    order = sorted(range(L), key=lambda j: (s[j], j))
+    E = L - keep
+    return sorted(order[E:]), sorted(order[:E])
+
+
+def test_select_matches_full_sort_with_ties():
+    rng = np.random.default_rng(0)
+    B, Hkv, n_max = 3, 2, 300
+    lengths = [300, 123, 7]
+    keep = [30, 100, 7]
+    s = rng.integers(0, 20, size=(B, Hkv, n_max)).astype(np.float64) / 7.0
+    for b, L in enumerate(lengths):
+        s[b, :, L - 3: L] = np.inf
+        s[b, :, L:] = np.nan
+    keep_idx, ev_idx = oracle.select(s, lengths, keep)
+    for b, L in enumerate(lengths):
+        for h in range(Hkv):
+            kk, ee = _brute_select(s[b, h].tolist(), L, keep[b])
+            got_k = [x for x in keep_idx[b, h].tolist() if x >= 0]
+            got_e = [x for x in ev_idx[b, h].tolist() if x >= 0]
+            assert got_k == kk and got_e == ee
+            assert all(x == -1 for x in keep_idx[b, h, len(kk):])
+
+
+def test_constant_values_give_zero_scores_and_all_ties():
+    """All v_j equal => a = v_j => every Delta is 0; eviction falls back to the
+    position order among the tied zeros.  (v = 0 keeps a = sum p_j v_j exactly
+    0 in floating point; any other constant leaves rounding residues ~1e-33.)"""
+    spec = W.Spec("constv", B=1, Hq=2, Hkv=1, d=4, lengths=[16], window=3, pool=3, keep=[6],
+                  dtype="f32")
+    wl = W.generate(spec, 21)
+    v = torch.zeros_like(wl.v)
+    s = oracle.scores(wl.q, wl.k, v, wl.lengths, 3, 3)
+    assert np.all(s[0, 0, :13] == 0.0)
+    keep, ev = oracle.select(s, wl.lengths, [6])
+    assert ev[0, 0].tolist() == list(range(10))
+    assert keep[0, 0].tolist() == [10, 11, 12, 13, 14, 15]
+
+
+# ---- sampled scoring equals the whole-problem oracle ---------------------
+
+def test_scores_at_equals_full_oracle():
+    spec = W.Spec("mid", B=1, Hq=4, Hkv=2, d=16, lengths=[90], window=5, pool=5, keep=[30],
+                  dtype="bf16")
+    wl = W.generate(spec, 31)
+    full = oracle.scores(wl.q, wl.k, wl.v, wl.lengths, 5, 5)
+    pos = [0, 1, 2, 40, 83, 84, 85, 86, 89]
+    for h in range(2):
+        got = oracle.scores_at(wl.q[0, 2 * h: 2 * h + 2], wl.k[0, h, :90], wl.v[0, h, :90],
+                               5, 5, pos)
+        np.testing.assert_allclose(got, full[0, h, pos], rtol=1e-13)
