@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of DropKV prefill-time eviction scoring on B200.
+
+One step = the whole scoring path on one input set: dropkv_scores (window
+attention statistics, exact single-removal perturbation scores summed over the
+window, GQA mean-merge, MaxPool1D, window protection) followed by dropkv_select
+(exact lowest-score eviction per KV head).
+
+Workload (N=1): the 128K-token Llama-3.1-8B-shaped case -- B=1, Hq=32, Hkv=8,
+d=128, n=131072, w=64, bf16 Gaussian Q/K/V with 4 outlier K channels x8 per KV
+head, pool 7, keep 5%.  K+V are 537 MB, larger than the 126 MB L2, so no L2
+flush is needed between steps.  With N GPUs (torchrun) every rank scores its
+own independent input set (seed 42 + rank): weak scaling, no data-path
+collective; the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (one query head of 32: its 64 window queries over all 131072 keys,
+scaled by 32) on the host cores.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from kv_cache_eviction_scores_b200 import workloads as W  # noqa: E402
+
+METRIC = "KV tokens scored/sec per GPU at n=128K; achieved HBM GB/s as % of roofline"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+CSRC = os.path.join(ROOT, "kv_cache_eviction_scores_b200", "csrc")
+
+# kernel order per scoring call (must match the library's launch sequence)
+KERNELS = {
+    "simt": ["k_simt_pass1", "k_simt_pass2", "k_epilogue"],
+    "tensor": ["k_tc_pass1", "k_tc_combine", "k_tc_pass2", "k_epilogue"],
+}
+KERNEL_SRC = {
+    "k_simt_pass1": "simt.cu", "k_simt_pass2": "simt.cu", "k_epilogue": "epilogue.cu",
+    "k_tc_pass1": "tc.cu", "k_tc_combine": "tc.cu", "k_tc_pass2": "tc.cu",
+}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", type=int, default=3, help="workload index (3 = 128K headline)")
+    p.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
+    p.add_argument("--e2e-steps", type=int, default=None)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("sm_max_mhz", 1965.0)), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1965.0, "fallback"
+
+
+def workload_desc(spec):
+    return (f"{spec.name}: B={spec.B} Hq={spec.Hq} Hkv={spec.Hkv} d={spec.d} "
+            f"n={spec.lengths} w={spec.window} pool={spec.pool} keep={spec.keep} {spec.dtype}")
+
+
+def visible_elements(spec):
+    """(token, window query) pairs with token visible to the query, all heads."""
+    w = spec.window
+    per_query_head = sum(w * (L - w) + w * (w + 1) // 2 for L in spec.lengths)
+    return per_query_head * spec.Hq
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index, enabled=True):
+        self.proc = None
+        self.path = None
+        self.dev = device_index
+        self.enabled = enabled
+
+    def start(self):
+        if not self.enabled:
+            return
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"]
+        except Exception:
+            sel = ["-i", str(self.dev)]
+        self.path = os.path.join("/tmp", f"dropkv_clocks_{os.getpid()}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ reference ----
+
+def oracle_sample(wl):
+    """fp64 oracle on one query head (its window queries over all keys) of
+    batch row 0, followed by merge/pool/protect/select of that head."""
+    import oracle
+    spec = wl.spec
+    L = wl.lengths[0]
+    t0 = time.perf_counter()
+    s = oracle.scores(wl.q[0:1, 0:1], wl.k[0:1, 0:1, :L], wl.v[0:1, 0:1, :L], [L], spec.window,
+                      spec.pool)
+    oracle.select(s, [L], [wl.keep[0]])
+    dt = time.perf_counter() - t0
+    frac = 1.0 / (spec.Hq * spec.B)  # this sample's share of the whole workload (row 0 = full L)
+    return dt, frac
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    spec = W.config_spec(args.config)
+    wl = W.generate(spec, 42)
+    tokens = sum(wl.lengths)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, frac = oracle_sample(wl)
+        if i >= args.warmup:
+            times.append(dt / frac)
+    t = statistics.mean(times)
+    cores = oracle.num_threads()
+    sample = (f"one query head of {spec.Hq} (its {spec.window} window queries over all "
+              f"{wl.lengths[0]} keys) of batch row 0 per step, fp64, scaled by {spec.Hq * spec.B}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tokens / t, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(spec), "global_batch": spec.B,
+                   "seq_len": max(spec.lengths), "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": tokens / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tokens / t, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ours ----
+
+def source_hash(fname):
+    with open(os.path.join(CSRC, fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def traffic_for(kernel):
+    """ncu DRAM bytes per launch of `kernel`, if captured on the current source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        e = d[kernel]
+        if e.get("csrc_sha256") != source_hash(KERNEL_SRC[kernel]):
+            return None
+        return float(e["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def roofline(kernel, spec, us, hbm_peak, tc_peak, sm_mhz):
+    """Roofline object for one kernel from its live CUDA-event duration."""
+    elems = visible_elements(spec)
+    d = spec.d
+    valid = sum(spec.lengths) * spec.Hkv
+    if kernel in ("k_simt_pass1", "k_simt_pass2"):
+        # two length-d contractions per visible (token, query) element on FP32 FMA units
+        flops = 2 * 2 * d * elems
+        peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # FP32 lanes x FMA x clock, TFLOP/s
+        ach = flops / (us * 1e-6) / 1e12
+        return {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": traffic_for(kernel),
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x max SM clock",
+                "work": f"{flops:.4g} flop (4*d per visible element)"}
+    if kernel in ("k_tc_pass1", "k_tc_pass2"):
+        flops = 2 * 2 * d * elems  # two algorithmic contractions per element
+        ach = flops / (us * 1e-6) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": ach / tc_peak, "traffic": traffic_for(kernel),
+                "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst) of measured",
+                "work": f"{flops:.4g} flop (4*d per visible element)"}
+    # HBM-bound helpers
+    nbytes = valid * 4 * 2
+    ach = nbytes / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+            "frac": ach / hbm_peak, "traffic": traffic_for(kernel),
+            "work": f"{nbytes} B"}
+
+
+def run_ours(args):
+    import kv_cache_eviction_scores_b200 as dk
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dk.lib()
+
+    spec = W.config_spec(args.config)
+    wl = W.generate(spec, 42 + rank)
+    q, k, v = wl.q.to(dev), wl.k.to(dev), wl.v.to(dev)
+    shape = dk.make_shape(q, k, spec.window, spec.pool)
+    path = {dk.PATH_SIMT: "simt", dk.PATH_TENSOR: "tensor"}[
+        dk.auto_path(shape) if args.path == "auto" else {"simt": 1, "tensor": 2}[args.path]]
+    ws = torch.empty(dk.scores_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    sel_ws = torch.empty(max(16, dk.select_workspace_bytes(spec.B, spec.Hkv, spec.n_max)),
+                         dtype=torch.uint8, device=dev)
+    scores = torch.empty(spec.B, spec.Hkv, spec.n_max, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    names = KERNELS[path]
+    nk = len(names)
+
+    def step(events=None):
+        dk.dropkv_scores(q, k, v, spec.window, spec.pool, wl.lengths, path=path, out=scores,
+                         workspace=ws, status=status, kernel_events=events)
+        return dk.dropkv_select(scores, wl.keep, wl.lengths, workspace=sel_ws)
+
+    K, Wm = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(K)]
+    for row in ev:
+        for e in row:
+            e.record()  # creates the handle
+    for _ in range(Wm):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != dk.OK:
+        raise dk.SingularError(int(status.item()), "bench inputs")
+    clocks = ClockSampler(local, enabled=not args.no_clocks)
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K):
+        step(ev[i])
+    t1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    if dist:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms = ms_total / K
+    kern_us = {}
+    for j, name in enumerate(names):
+        kern_us[name] = statistics.mean(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1])
+                                        for i in range(K)) * 1e3
+    if int(status.item()) != dk.OK:
+        raise dk.SingularError(int(status.item()), "bench inputs")
+
+    # ---- end to end through the public API, host buffers, copies inside ----
+    E = args.e2e_steps if args.e2e_steps is not None else max(3, min(K, 10))
+    qh, kh, vh = (t.pin_memory() for t in (wl.q, wl.k, wl.v))
+    sc_h = torch.empty(scores.shape, dtype=torch.float32).pin_memory()
+    keep_idx, ev_idx = step()
+    kp_h = torch.empty(keep_idx.shape, dtype=torch.int32).pin_memory()
+    ev_h = torch.empty(ev_idx.shape, dtype=torch.int32).pin_memory()
+    st_h = torch.empty(1, dtype=torch.int32).pin_memory()
+    torch.cuda.synchronize()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        kk, ee = step()
+        sc_h.copy_(scores, non_blocking=True)
+        kp_h.copy_(kk, non_blocking=True)
+        ev_h.copy_(ee, non_blocking=True)
+        st_h.copy_(status, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(E):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+    if dist:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+        dist.barrier()
+    e2e_ms /= E
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = sum(t.numel() * t.element_size() for t in (sc_h, kp_h, ev_h, st_h))
+
+    tokens = sum(wl.lengths)
+    value = world * tokens / (ms * 1e-3)
+    hbm_peak, tc_peak, sm_mhz, peak_src = peaks()
+    dominant = max(kern_us, key=kern_us.get)
+    roof = roofline(dominant, spec, kern_us[dominant], hbm_peak, tc_peak, sm_mhz)
+    roof["kernel"] = dominant
+    roof["peak_of"] = peak_src
+    kv_bytes = 2 * spec.Hkv * tokens * spec.d * 2
+    alg_bytes = kv_bytes + q.numel() * 2 + spec.B * spec.Hkv * spec.n_max * 4
+    launches = dk.scores_launches(shape, wl.lengths, path) + dk.select_launches(
+        spec.B, spec.Hkv, spec.n_max, wl.lengths)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if path == "tensor" else "f32",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(spec), "path": path, "global_batch": spec.B * world,
+                   "seq_len": max(spec.lengths),
+                   "parallelism": f"replicas x{world} (independent inputs per GPU)",
+                   "l2": f"inputs {kv_bytes / 1e6:.0f} MB > 126 MB L2; no flush"},
+        "hbm": {"alg_bytes_per_step": alg_bytes,
+                "achieved_gbs": alg_bytes / (ms * 1e-3) / 1e9 * 1.0,
+                "peak_gbs": hbm_peak, "frac": alg_bytes / (ms * 1e-3) / 1e9 / hbm_peak,
+                "of": peak_src},
+        "roofline": roof,
+        "kernels_us": kern_us,
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches * K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        dt, frac = oracle_sample(wl)
+        line["cpu_baseline"] = {
+            "value": tokens / (dt / frac), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"one query head of {spec.Hq} of batch row 0 (its {spec.window} window "
+                      f"queries over all {wl.lengths[0]} keys), fp64, {dt:.2f} s, scaled by "
+                      f"{int(round(1 / frac))}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,272 @@
+"""DropKV prefill-time KV-cache eviction scoring on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``libdropkv.so`` (C ABI: ``include/dropkv.h``).
+It only marshals arguments: PyTorch supplies device memory and the current
+stream, and every step of the scoring path runs in the library's CUDA kernels.
+There is no CPU fallback; without the built library every call raises.
+
+What is scored (write-up "DropKV：精确单项输出扰动评分组件", section 核心公式
+and the Algorithm 1 paragraph): for the last ``window`` prompt queries,
+p = softmax(K q / sqrt d), a = sum_j p_j v_j, Delta_j = p_j/(1-p_j) (a - v_j),
+s_j = sum_t ||Delta_j||^2; scores are averaged over the query heads of each KV
+head, max-pooled, the window is set to +inf, and the lowest scores are evicted.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = [
+    "DropKVError", "SingularError", "Shape", "Options", "lib", "lib_path",
+    "make_shape", "scores_workspace_bytes", "select_workspace_bytes", "dropkv_scores",
+    "dropkv_select", "evict", "auto_path", "scores_launches", "select_launches",
+    "OK", "ERR_ARG", "ERR_SINGULAR", "ERR_CUDA", "ERR_UNSUPPORTED", "ERR_WORKSPACE",
+    "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR",
+]
+
+OK, ERR_ARG, ERR_SINGULAR, ERR_CUDA, ERR_UNSUPPORTED, ERR_WORKSPACE = range(6)
+PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
+_PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tensor": PATH_TENSOR}
+BF16, F32 = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libdropkv.so")
+
+
+class DropKVError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = _status_string(status)
+        super().__init__(f"{what}: {msg} (status {status})" if what else msg)
+
+
+class SingularError(DropKVError):
+    """Some window probability rounds to 1: exact single removal is undefined."""
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "Hq", "Hkv", "n_max", "d", "window", "pool_kernel", "dtype")]
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("attn_out", ctypes.c_void_p), ("stats_out", ctypes.c_void_p),
+                ("events", ctypes.c_void_p), ("n_events", ctypes.c_int32),
+                ("reserved2", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libdropkv.so (built in-tree by ``python -m kv_cache_eviction_scores_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"libdropkv.so is not built ({path}); run "
+                           "`python -m kv_cache_eviction_scores_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+    ip = ctypes.POINTER(ctypes.c_int32)
+    sp = ctypes.POINTER(Shape)
+    L.dropkv_scores_workspace_bytes.argtypes = [sp]
+    L.dropkv_scores_workspace_bytes.restype = sz
+    L.dropkv_scores.argtypes = [sp, vp, vp, vp, ip, vp, vp, sz, vp]
+    L.dropkv_scores.restype = i32
+    L.dropkv_scores_async.argtypes = [sp, vp, vp, vp, ip, vp, vp, sz, vp, vp]
+    L.dropkv_scores_async.restype = i32
+    L.dropkv_scores_ex.argtypes = [sp, vp, vp, vp, ip, vp, vp, sz, vp, vp,
+                                   ctypes.POINTER(Options)]
+    L.dropkv_scores_ex.restype = i32
+    L.dropkv_select_workspace_bytes.argtypes = [i32, i32, i32]
+    L.dropkv_select_workspace_bytes.restype = sz
+    L.dropkv_select.argtypes = [i32, i32, i32, vp, ip, ip, vp, i32, vp, i32, vp, sz, vp]
+    L.dropkv_select.restype = i32
+    L.dropkv_auto_path.argtypes = [sp]
+    L.dropkv_auto_path.restype = i32
+    L.dropkv_scores_launches.argtypes = [sp, ip, i32]
+    L.dropkv_scores_launches.restype = i32
+    L.dropkv_select_launches.argtypes = [i32, i32, i32, ip]
+    L.dropkv_select_launches.restype = i32
+    L.dropkv_status_string.argtypes = [i32]
+    L.dropkv_status_string.restype = ctypes.c_char_p
+    L.dropkv_abi_version.argtypes = []
+    L.dropkv_abi_version.restype = i32
+    _lib = L
+    return L
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().dropkv_status_string(status).decode()
+    except Exception:
+        return f"status {status}"
+
+
+def _check(status: int, what: str):
+    if status == OK:
+        return
+    if status == ERR_SINGULAR:
+        raise SingularError(status, what)
+    raise DropKVError(status, what)
+
+
+def _i32_array(vals: Optional[Sequence[int]]):
+    if vals is None:
+        return None
+    arr = (ctypes.c_int32 * len(vals))(*[int(x) for x in vals])
+    return arr
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, window: int, pool_kernel: int) -> Shape:
+    B, Hq, w, d = q.shape
+    Bk, Hkv, n_max, dk = k.shape
+    if (B, d) != (Bk, dk) or w != window:
+        raise ValueError("q must be [B, Hq, window, d] and k, v [B, Hkv, n_max, d]")
+    if q.dtype == torch.bfloat16:
+        dt = BF16
+    elif q.dtype == torch.float32:
+        dt = F32
+    else:
+        raise TypeError("q, k, v must be bfloat16 or float32")
+    return Shape(B, Hq, Hkv, n_max, d, window, pool_kernel, dt)
+
+
+def scores_workspace_bytes(shape: Shape) -> int:
+    return int(lib().dropkv_scores_workspace_bytes(ctypes.byref(shape)))
+
+
+def select_workspace_bytes(B: int, Hkv: int, n_max: int) -> int:
+    return int(lib().dropkv_select_workspace_bytes(B, Hkv, n_max))
+
+
+def auto_path(shape: Shape) -> int:
+    return int(lib().dropkv_auto_path(ctypes.byref(shape)))
+
+
+def scores_launches(shape: Shape, lengths=None, path: str = "auto") -> int:
+    return int(lib().dropkv_scores_launches(ctypes.byref(shape), _i32_array(lengths),
+                                            _PATHS[path]))
+
+
+def select_launches(B: int, Hkv: int, n_max: int, lengths=None) -> int:
+    return int(lib().dropkv_select_launches(B, Hkv, n_max, _i32_array(lengths)))
+
+
+def _check_inputs(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share one dtype")
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k and v must be on one device")
+
+
+def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int,
+                  pool_kernel: int, lengths: Optional[Sequence[int]] = None, *,
+                  path: str = "auto", out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, return_attn: bool = False,
+                  status: Optional[torch.Tensor] = None, kernel_events=None):
+    """fp32 scores [B, Hkv, n_max] (pooled, window = +inf, padding = NaN).
+
+    q: [B, Hq, window, d] window queries; k, v: [B, Hkv, n_max, d]; lengths:
+    per-row lengths (host ints) or None for n_max.  With ``status`` (a CUDA
+    int32 tensor of one element) the call is asynchronous and the singular flag
+    lands there; otherwise it synchronises and raises SingularError.
+    With ``return_attn`` also returns the window attention outputs
+    [B, Hq, window, d] and (max logit, normaliser) stats [B, Hq, window, 2].
+    ``kernel_events``: torch.cuda.Event objects (each recorded once already so
+    that its handle exists); events 2i / 2i+1 bracket the i-th kernel launch.
+    """
+    _check_inputs(q, k, v)
+    shape = make_shape(q, k, window, pool_kernel)
+    dev = q.device
+    if out is None:
+        out = torch.empty(shape.B, shape.Hkv, shape.n_max, dtype=torch.float32, device=dev)
+    need = scores_workspace_bytes(shape)
+    if need == 0:
+        raise DropKVError(ERR_ARG, "dropkv_scores_workspace_bytes")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    opts = Options(_PATHS[path], 0, None, None, None, 0, 0)
+    ev_arr = None
+    if kernel_events:
+        # raw cudaEvent_t handles of (already recorded once) torch.cuda.Event objects
+        ev_arr = (ctypes.c_void_p * len(kernel_events))(*[e.cuda_event for e in kernel_events])
+        opts.events = ctypes.cast(ev_arr, ctypes.c_void_p)
+        opts.n_events = len(kernel_events)
+    attn = stats = None
+    if return_attn:
+        attn = torch.empty(shape.B, shape.Hq, window, shape.d, dtype=torch.float32, device=dev)
+        stats = torch.empty(shape.B, shape.Hq, window, 2, dtype=torch.float32, device=dev)
+        opts.attn_out = attn.data_ptr()
+        opts.stats_out = stats.data_ptr()
+    st = lib().dropkv_scores_ex(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                _i32_array(lengths), _ptr(out), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(dev),
+                                _ptr(status), ctypes.byref(opts))
+    _check(st, "dropkv_scores")
+    if return_attn:
+        return out, attn, stats
+    return out
+
+
+def dropkv_select(scores: torch.Tensor, keep_counts: Sequence[int],
+                  lengths: Optional[Sequence[int]] = None, *, max_keep: Optional[int] = None,
+                  max_evict: Optional[int] = None,
+                  workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Keep / evict positions per (b, h), ascending, padded with -1 (int32)."""
+    if not scores.is_cuda or scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise TypeError("scores must be a contiguous CUDA float32 tensor")
+    B, Hkv, n_max = scores.shape
+    lens = list(lengths) if lengths is not None else [n_max] * B
+    keep = [int(x) for x in keep_counts]
+    if len(keep) != B or len(lens) != B:
+        raise ValueError("keep_counts and lengths need one entry per batch row")
+    if max_keep is None:
+        max_keep = max(keep)
+    if max_evict is None:
+        max_evict = max(L - kc for L, kc in zip(lens, keep))
+    dev = scores.device
+    keep_idx = torch.empty(B, Hkv, max_keep, dtype=torch.int32, device=dev)
+    evict_idx = torch.empty(B, Hkv, max_evict, dtype=torch.int32, device=dev)
+    need = select_workspace_bytes(B, Hkv, n_max)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = lib().dropkv_select(B, Hkv, n_max, _ptr(scores), _i32_array(lengths),
+                             _i32_array(keep), _ptr(keep_idx), max_keep, _ptr(evict_idx),
+                             max_evict, _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(st, "dropkv_select")
+    return keep_idx, evict_idx
+
+
+def evict(q, k, v, window: int, pool_kernel: int, keep_counts: Sequence[int],
+          lengths: Optional[Sequence[int]] = None, *, path: str = "auto"):
+    """Scores and the keep / evict lists in one call: (scores, keep_idx, evict_idx)."""
+    s = dropkv_scores(q, k, v, window, pool_kernel, lengths, path=path)
+    keep_idx, evict_idx = dropkv_select(s, keep_counts, lengths)
+    return s, keep_idx, evict_idx

@@ -1,0 +1,93 @@
+// internal.h -- host-side declarations shared by the libdropkv.so sources.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "dropkv.h"
+
+namespace dropkv {
+
+// Batch rows handled per launch; larger batches are processed in slices.
+constexpr int kMaxB = 64;
+
+// Bits of the device status word (the value equals DROPKV_ERR_SINGULAR).
+constexpr int kStatusSingular = DROPKV_ERR_SINGULAR;
+
+// Per-slice sequence lengths, passed by value as a kernel parameter.
+struct Lens {
+  int32_t B;
+  int32_t L[kMaxB];
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Optional caller-owned CUDA events recorded around each kernel launch.
+struct KernelEvents {
+  void* const* ev = nullptr;
+  int n = 0;
+  int i = 0;
+  void begin(cudaStream_t st) {
+    if (ev && 2 * i + 1 < n) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[2 * i]), st);
+  }
+  void end(cudaStream_t st) {
+    if (ev && 2 * i + 1 < n) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[2 * i + 1]), st);
+    ++i;
+  }
+};
+
+// ---- scoring: workspace carve-up ------------------------------------------
+struct ScoresLayout {
+  size_t status;     // int32 status word (sync variant)
+  size_t stats;      // fp32 [B, Hq, w, 2]  (max logit, normaliser)
+  size_t attn;       // fp32 [B, Hq, w, d]  window attention output a
+  size_t parts;      // fp32 [nparts][B, Hkv, n_max] partial merged scores
+  size_t tc_partial; // fp32 pass-1 split partials (tensor path)
+  size_t tc_ahi;     // bf16 [B, Hq, w, d] high part of a (tensor path)
+  size_t tc_alo;     // bf16 [B, Hq, w, d] low part of a (tensor path)
+  size_t tc_qstat;   // fp32 [B, Hq, w, 4] per-query pass-2 constants (tensor path)
+  size_t total;
+  int nparts;
+};
+
+// Tensor-path plan for one batch slice.
+struct TcPlan {
+  int chunks;        // query chunks per KV head (G*w split into chunks of nqc rows)
+  int nqc;           // rows per chunk (multiple of 16, <= 128)
+  int max_ctas;      // upper bound of pass-1 CTAs (sizes the partial buffer)
+};
+
+bool tc_shape_ok(const dropkv_shape& s);
+TcPlan tc_plan(const dropkv_shape& s);
+ScoresLayout scores_layout(const dropkv_shape& s, int B_slice);
+
+// ---- launchers (each returns the CUDA error of its launch) ----------------
+cudaError_t launch_simt_pass1(const dropkv_shape& s, const void* q, const void* k,
+                              const void* v, const Lens& lens, float* stats, float* attn,
+                              cudaStream_t st);
+cudaError_t launch_simt_pass2(const dropkv_shape& s, const void* q, const void* k,
+                              const void* v, const Lens& lens, const float* stats,
+                              const float* attn, float* part, int32_t* status,
+                              cudaStream_t st);
+cudaError_t launch_epilogue(const dropkv_shape& s, const Lens& lens, const float* parts,
+                            int nparts, size_t part_stride, float* scores, cudaStream_t st);
+
+// Tensor-core path (tcgen05 + TMA); returns cudaErrorNotSupported when the
+// tensor maps cannot be encoded.
+cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k,
+                             const void* v, const Lens& lens, const ScoresLayout& lay,
+                             char* ws, float* attn_out, float* stats_out, int32_t* status,
+                             cudaStream_t st, KernelEvents& kev);
+int tc_launch_count();
+int tc_split_target();
+bool tc_available();
+
+// ---- selection --------------------------------------------------------------
+size_t select_workspace_bytes(int B, int Hkv, int n_max);
+int select_launch_count();
+cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const int32_t* L,
+                          const int32_t* keep, int32_t* keep_idx, int32_t max_keep,
+                          int32_t* evict_idx, int32_t max_evict, void* ws, cudaStream_t st);
+
+}  // namespace dropkv
