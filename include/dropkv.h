@@ -58,8 +58,9 @@ typedef enum dropkv_status {
 } dropkv_status;
 
 typedef enum dropkv_dtype {
-  DROPKV_BF16 = 0,  /* q, k, v stored as bfloat16; arithmetic in fp32 */
-  DROPKV_F32 = 1    /* q, k, v stored as float32; arithmetic in fp32  */
+  DROPKV_BF16 = 0,  /* q, k, v stored as bfloat16; arithmetic in fp32 (tensor-core
+                       operands bf16 with fp32 accumulation)                          */
+  DROPKV_F32 = 1    /* q, k, v stored as float32; arithmetic in fp64 (CUDA cores)      */
 } dropkv_dtype;
 
 /* Which kernels compute the scores (dropkv_options.path). */
@@ -152,6 +153,7 @@ DROPKV_API size_t dropkv_select_workspace_bytes(int32_t B, int32_t Hkv, int32_t 
  *                then -1;  max_keep >= every keep_counts[b].
  *   evict_idx    device int32 [B, Hkv, max_evict]: evicted positions ascending,
  *                then -1;  max_evict >= every lengths[b] - keep_counts[b].
+ *                (keep_idx / evict_idx may be NULL when max_keep / max_evict is 0.)
  * Asynchronous on `stream`; integer results are exact.
  */
 DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,

@@ -91,9 +91,9 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   l.status = o;
   o += kAlign;
   l.stats = o;
-  o = align_up(o + rows * 2 * sizeof(float), kAlign);
+  o = align_up(o + rows * 2 * sizeof(double), kAlign);
   l.attn = o;
-  o = align_up(o + rows * s.d * sizeof(float), kAlign);
+  o = align_up(o + rows * s.d * sizeof(double), kAlign);
   l.parts = o;
   o = align_up(o + (size_t)l.nparts * Bs * s.Hkv * (size_t)s.n_max * sizeof(float), kAlign);
   l.tc_partial = l.tc_ahi = l.tc_alo = l.tc_qstat = o;
@@ -160,20 +160,21 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
     const char* ks = reinterpret_cast<const char*>(k) + kvoff * esz;
     const char* vs = reinterpret_cast<const char*>(v) + kvoff * esz;
     float* sc = scores + (size_t)b0 * s.Hkv * s.n_max;
-    float* attn = (opt && opt->attn_out) ? opt->attn_out + qoff
-                                        : reinterpret_cast<float*>(ws + lay.attn);
-    float* stats = (opt && opt->stats_out) ? opt->stats_out + (size_t)b0 * s.Hq * s.window * 2
-                                          : reinterpret_cast<float*>(ws + lay.stats);
+    float* attn_user = (opt && opt->attn_out) ? opt->attn_out + qoff : nullptr;
+    float* stats_user =
+        (opt && opt->stats_out) ? opt->stats_out + (size_t)b0 * s.Hq * s.window * 2 : nullptr;
+    double* stats_ws = reinterpret_cast<double*>(ws + lay.stats);
+    void* attn_ws = ws + lay.attn;
     float* parts = reinterpret_cast<float*>(ws + lay.parts);
     const size_t part_stride = (size_t)Bs * s.Hkv * s.n_max;
     cudaError_t e;
     if (path == DROPKV_PATH_SIMT) {
       kev.begin(st);
-      e = launch_simt_pass1(s, qs, ks, vs, lens, stats, attn, st);
+      e = launch_simt_pass1(s, qs, ks, vs, lens, stats_ws, attn_ws, stats_user, attn_user, st);
       kev.end(st);
       if (e == cudaSuccess) {
         kev.begin(st);
-        e = launch_simt_pass2(s, qs, ks, vs, lens, stats, attn, parts, status_word, st);
+        e = launch_simt_pass2(s, qs, ks, vs, lens, stats_ws, attn_ws, parts, status_word, st);
         kev.end(st);
       }
       if (e == cudaSuccess) {
@@ -182,9 +183,8 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
         kev.end(st);
       }
     } else {
-      e = launch_tc_scores(s, qs, ks, vs, lens, lay, ws,
-                           (opt && opt->attn_out) ? attn : nullptr,
-                           (opt && opt->stats_out) ? stats : nullptr, status_word, st, kev);
+      e = launch_tc_scores(s, qs, ks, vs, lens, lay, ws, attn_user, stats_user, status_word, st,
+                           kev);
       if (e == cudaSuccess) {
         kev.begin(st);
         e = launch_epilogue(s, lens, parts, lay.nparts, part_stride, sc, st);
@@ -251,8 +251,8 @@ dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* 
                             int32_t* keep_idx, int32_t max_keep, int32_t* evict_idx,
                             int32_t max_evict, void* workspace, size_t workspace_bytes,
                             void* stream) {
-  if (B < 1 || Hkv < 1 || n_max < 1 || !scores || !keep_counts || !keep_idx || !evict_idx)
-    return DROPKV_ERR_ARG;
+  if (B < 1 || Hkv < 1 || n_max < 1 || !scores || !keep_counts) return DROPKV_ERR_ARG;
+  if ((!keep_idx && max_keep > 0) || (!evict_idx && max_evict > 0)) return DROPKV_ERR_ARG;
   if (max_keep < 0 || max_evict < 0) return DROPKV_ERR_ARG;
   if (!aligned16(scores) || ((uintptr_t)keep_idx & 3u) || ((uintptr_t)evict_idx & 3u))
     return DROPKV_ERR_ARG;

@@ -40,8 +40,8 @@ struct KernelEvents {
 // ---- scoring: workspace carve-up ------------------------------------------
 struct ScoresLayout {
   size_t status;     // int32 status word (sync variant)
-  size_t stats;      // fp32 [B, Hq, w, 2]  (max logit, normaliser)
-  size_t attn;       // fp32 [B, Hq, w, d]  window attention output a
+  size_t stats;      // fp64 [B, Hq, w, 2]  (max logit, normaliser), SIMT path
+  size_t attn;       // [B, Hq, w, d] window attention output a (8 bytes per element)
   size_t parts;      // fp32 [nparts][B, Hkv, n_max] partial merged scores
   size_t tc_partial; // fp32 pass-1 split partials (tensor path)
   size_t tc_ahi;     // bf16 [B, Hq, w, d] high part of a (tensor path)
@@ -63,12 +63,15 @@ TcPlan tc_plan(const dropkv_shape& s);
 ScoresLayout scores_layout(const dropkv_shape& s, int B_slice);
 
 // ---- launchers (each returns the CUDA error of its launch) ----------------
+// SIMT path.  stats_ws: fp64 [rows][2]; attn_ws: [rows][d] in the path's
+// arithmetic type (fp32 for bf16 inputs, fp64 for fp32 inputs); the *_user
+// pointers (optional) receive fp32 copies.
 cudaError_t launch_simt_pass1(const dropkv_shape& s, const void* q, const void* k,
-                              const void* v, const Lens& lens, float* stats, float* attn,
-                              cudaStream_t st);
+                              const void* v, const Lens& lens, double* stats_ws, void* attn_ws,
+                              float* stats_user, float* attn_user, cudaStream_t st);
 cudaError_t launch_simt_pass2(const dropkv_shape& s, const void* q, const void* k,
-                              const void* v, const Lens& lens, const float* stats,
-                              const float* attn, float* part, int32_t* status,
+                              const void* v, const Lens& lens, const double* stats_ws,
+                              const void* attn_ws, float* part, int32_t* status,
                               cudaStream_t st);
 cudaError_t launch_epilogue(const dropkv_shape& s, const Lens& lens, const float* parts,
                             int nparts, size_t part_stride, float* scores, cudaStream_t st);
