@@ -148,18 +148,27 @@ class ClockSampler:
 # ------------------------------------------------------------ reference ----
 
 def oracle_sample(wl):
-    """fp64 oracle on one query head (its window queries over all keys) of
-    batch row 0, followed by merge/pool/protect/select of that head."""
+    """fp64 oracle on the first KV heads of batch row 0 (all their query heads,
+    window queries over every key), then merge/pool/protect/select of them.
+    The oracle runs one OpenMP thread per query head, so the sample takes as
+    many KV heads as keep the host cores busy.  Returns (seconds, share of the
+    whole workload, threads used, description)."""
     import oracle
     spec = wl.spec
     L = wl.lengths[0]
+    G = spec.G
+    nkv = max(1, min(spec.Hkv, oracle.num_threads() // G))
     t0 = time.perf_counter()
-    s = oracle.scores(wl.q[0:1, 0:1], wl.k[0:1, 0:1, :L], wl.v[0:1, 0:1, :L], [L], spec.window,
-                      spec.pool)
+    s = oracle.scores(wl.q[0:1, 0:nkv * G], wl.k[0:1, 0:nkv, :L], wl.v[0:1, 0:nkv, :L], [L],
+                      spec.window, spec.pool)
     oracle.select(s, [L], [wl.keep[0]])
     dt = time.perf_counter() - t0
-    frac = 1.0 / (spec.Hq * spec.B)  # this sample's share of the whole workload (row 0 = full L)
-    return dt, frac
+    frac = (nkv * G * L) / (spec.Hq * sum(wl.lengths))
+    threads = min(oracle.num_threads(), nkv * G)
+    desc = (f"{nkv} of {spec.Hkv} KV heads of batch row 0 ({nkv * G} query heads x "
+            f"{spec.window} window queries over all {L} keys), fp64, {dt:.2f} s, "
+            f"scaled by {1 / frac:.3g}")
+    return dt, frac, threads, desc
 
 
 def run_reference(args):
@@ -172,13 +181,11 @@ def run_reference(args):
     tokens = sum(wl.lengths)
     times = []
     for i in range(args.warmup + args.steps):
-        dt, frac = oracle_sample(wl)
+        dt, frac, cores, sample = oracle_sample(wl)
         if i >= args.warmup:
             times.append(dt / frac)
     t = statistics.mean(times)
-    cores = oracle.num_threads()
-    sample = (f"one query head of {spec.Hq} (its {spec.window} window queries over all "
-              f"{wl.lengths[0]} keys) of batch row 0 per step, fp64, scaled by {spec.Hq * spec.B}")
+    sample = "per step: " + sample
     line = {
         "impl": "reference", "metric": METRIC, "value": tokens / t, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -242,6 +249,53 @@ def roofline(kernel, spec, us, hbm_peak, tc_peak, sm_mhz):
     return {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
             "frac": ach / hbm_peak, "traffic": traffic_for(kernel),
             "work": f"{nbytes} B"}
+
+
+def run_e2e(dk, wl, q, k, v, scores, status, step, E, dist, dev, world):
+    """Same metric through the public API with host buffers: every step copies
+    the inputs host->device (pinned) and the scores / index lists / status back."""
+    qh, kh, vh = (t.pin_memory() for t in (wl.q, wl.k, wl.v))
+    sc_h = torch.empty(scores.shape, dtype=torch.float32).pin_memory()
+    keep_idx, ev_idx = step()
+    kp_h = torch.empty(keep_idx.shape, dtype=torch.int32).pin_memory()
+    ev_h = torch.empty(ev_idx.shape, dtype=torch.int32).pin_memory()
+    st_h = torch.empty(1, dtype=torch.int32).pin_memory()
+    torch.cuda.synchronize()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        kk, ee = step()
+        sc_h.copy_(scores, non_blocking=True)
+        kp_h.copy_(kk, non_blocking=True)
+        ev_h.copy_(ee, non_blocking=True)
+        st_h.copy_(status, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(E):
+        e2e_step()
+    a1.record()
+    torch.cuda.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+    if dist:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+        dist.barrier()
+    e2e_ms /= E
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = sum(t.numel() * t.element_size() for t in (sc_h, kp_h, ev_h, st_h))
+
+    tokens = sum(wl.lengths)
+    return {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
 def run_ours(args):
@@ -320,45 +374,9 @@ def run_ours(args):
 
     # ---- end to end through the public API, host buffers, copies inside ----
     E = args.e2e_steps if args.e2e_steps is not None else max(3, min(K, 10))
-    qh, kh, vh = (t.pin_memory() for t in (wl.q, wl.k, wl.v))
-    sc_h = torch.empty(scores.shape, dtype=torch.float32).pin_memory()
-    keep_idx, ev_idx = step()
-    kp_h = torch.empty(keep_idx.shape, dtype=torch.int32).pin_memory()
-    ev_h = torch.empty(ev_idx.shape, dtype=torch.int32).pin_memory()
-    st_h = torch.empty(1, dtype=torch.int32).pin_memory()
-    torch.cuda.synchronize()
-
-    def e2e_step():
-        q.copy_(qh, non_blocking=True)
-        k.copy_(kh, non_blocking=True)
-        v.copy_(vh, non_blocking=True)
-        kk, ee = step()
-        sc_h.copy_(scores, non_blocking=True)
-        kp_h.copy_(kk, non_blocking=True)
-        ev_h.copy_(ee, non_blocking=True)
-        st_h.copy_(status, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    a0 = torch.cuda.Event(enable_timing=True)
-    a1 = torch.cuda.Event(enable_timing=True)
-    a0.record()
-    for _ in range(E):
-        e2e_step()
-    a1.record()
-    torch.cuda.synchronize()
-    e2e_ms = a0.elapsed_time(a1)
-    if dist:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-        dist.barrier()
-    e2e_ms /= E
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-    d2h = sum(t.numel() * t.element_size() for t in (sc_h, kp_h, ev_h, st_h))
-
+    e2e = None
+    if E > 0:
+        e2e = run_e2e(dk, wl, q, k, v, scores, status, step, E, dist, dev, world)
     tokens = sum(wl.lengths)
     value = world * tokens / (ms * 1e-3)
     hbm_peak, tc_peak, sm_mhz, peak_src = peaks()
@@ -386,20 +404,14 @@ def run_ours(args):
                 "of": peak_src},
         "roofline": roof,
         "kernels_us": kern_us,
-        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "e2e": e2e,
         "gpu_launches": launches * K,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        dt, frac = oracle_sample(wl)
-        line["cpu_baseline"] = {
-            "value": tokens / (dt / frac), "unit": UNIT, "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"one query head of {spec.Hq} of batch row 0 (its {spec.window} window "
-                      f"queries over all {wl.lengths[0]} keys), fp64, {dt:.2f} s, scaled by "
-                      f"{int(round(1 / frac))}"}
+        dt, frac, cores, desc = oracle_sample(wl)
+        line["cpu_baseline"] = {"value": tokens / (dt / frac), "unit": UNIT, "cores": cores,
+                                "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -54,7 +54,8 @@ typedef enum dropkv_status {
   DROPKV_ERR_SINGULAR = 2,     /* some p_j rounds to 1 in fp32 (1 - p_j is not > 0)      */
   DROPKV_ERR_CUDA = 3,         /* a CUDA runtime or driver call failed                   */
   DROPKV_ERR_UNSUPPORTED = 4,  /* no sm_100 device, or a path forced on a shape it lacks */
-  DROPKV_ERR_WORKSPACE = 5     /* workspace NULL or smaller than the query returned      */
+  DROPKV_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than the query returned      */
+  DROPKV_ERR_TIMEOUT = 6       /* a device-side wait gave up (bounded waits, no hang)    */
 } dropkv_status;
 
 typedef enum dropkv_dtype {
@@ -124,9 +125,10 @@ DROPKV_API dropkv_status dropkv_scores(const dropkv_shape* shape, const void* q,
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /* As dropkv_scores, without the synchronisation: returns once the work is
- * enqueued.  status_dev (device int32, caller-owned) receives DROPKV_OK or
- * DROPKV_ERR_SINGULAR when the work completes.  Host-side errors are returned
- * directly and nothing is enqueued. */
+ * enqueued.  status_dev (device int32, caller-owned) receives DROPKV_OK, or
+ * the largest error code the kernels raised (DROPKV_ERR_SINGULAR, or
+ * DROPKV_ERR_TIMEOUT if a bounded device-side wait gave up), when the work
+ * completes.  Host-side errors are returned directly and nothing is enqueued. */
 DROPKV_API dropkv_status dropkv_scores_async(const dropkv_shape* shape, const void* q, const void* k,
                                   const void* v, const int32_t* lengths, float* scores,
                                   void* workspace, size_t workspace_bytes, void* stream,

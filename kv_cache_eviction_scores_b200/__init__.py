@@ -24,11 +24,11 @@ __all__ = [
     "DropKVError", "SingularError", "Shape", "Options", "lib", "lib_path",
     "make_shape", "scores_workspace_bytes", "select_workspace_bytes", "dropkv_scores",
     "dropkv_select", "evict", "auto_path", "scores_launches", "select_launches",
-    "OK", "ERR_ARG", "ERR_SINGULAR", "ERR_CUDA", "ERR_UNSUPPORTED", "ERR_WORKSPACE",
+    "OK", "ERR_ARG", "ERR_SINGULAR", "ERR_CUDA", "ERR_UNSUPPORTED", "ERR_WORKSPACE", "ERR_TIMEOUT",
     "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR",
 ]
 
-OK, ERR_ARG, ERR_SINGULAR, ERR_CUDA, ERR_UNSUPPORTED, ERR_WORKSPACE = range(6)
+OK, ERR_ARG, ERR_SINGULAR, ERR_CUDA, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TIMEOUT = range(7)
 PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
 _PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tensor": PATH_TENSOR}
 BF16, F32 = 0, 1

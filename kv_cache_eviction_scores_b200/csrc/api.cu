@@ -66,7 +66,7 @@ int resolve_path(const dropkv_shape& s, int requested) {
 // the token-major pass-2 MMA).
 bool tc_shape_ok(const dropkv_shape& s) {
   if (!tc_available()) return false;
-  if (s.dtype != DROPKV_BF16 || s.d != 128) return false;
+  if (s.dtype != DROPKV_BF16 || s.d != 128 || s.n_max < 128) return false;
   const int nq = (s.Hq / s.Hkv) * s.window;
   const int chunks = (nq + 127) / 128;
   if (nq % (16 * chunks) != 0) return false;
@@ -100,10 +100,10 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   if (tc) {
     const TcPlan p = tc_plan(s);
     // pass-1 partials: at most (split target + one per (b, h, chunk)) CTAs,
-    // each 128 rows of (max, normaliser, a[d]).
+    // two warpgroups each, 128 rows of (a[128], max, normaliser, pad).
     const size_t ctas = (size_t)tc_split_target() + (size_t)Bs * s.Hkv * p.chunks;
     l.tc_partial = o;
-    o = align_up(o + ctas * 128 * (s.d + 2) * sizeof(float), kAlign);
+    o = align_up(o + ctas * 2 * 128 * 132 * sizeof(float), kAlign);
     l.tc_ahi = o;
     o = align_up(o + rows * s.d * 2, kAlign);
     l.tc_alo = o;
@@ -200,7 +200,7 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
           cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return DROPKV_ERR_CUDA;
-  if (host_status & kStatusSingular) return DROPKV_ERR_SINGULAR;
+  if (host_status != 0) return static_cast<dropkv_status>(host_status);
   return DROPKV_OK;
 }
 
@@ -312,6 +312,7 @@ const char* dropkv_status_string(dropkv_status status) {
     case DROPKV_ERR_CUDA: return "CUDA error";
     case DROPKV_ERR_UNSUPPORTED: return "unsupported device or shape";
     case DROPKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case DROPKV_ERR_TIMEOUT: return "a device-side wait timed out";
   }
   return "unknown status";
 }

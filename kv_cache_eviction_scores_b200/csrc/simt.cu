@@ -196,7 +196,7 @@ k_simt_pass2(const T* __restrict__ q, const T* __restrict__ k, const T* __restri
         const A e = exp_acc(x - m);
         const A den = l - e;  // (1 - p_j) * l
         if (!(den > A(0))) {  // p_j rounds to 1: removal is singular
-          atomicOr(status, kStatusSingular);
+          atomicMax(status, kStatusSingular);
           continue;
         }
         const A ratio = e / den;  // p_j / (1 - p_j)

@@ -1,16 +1,835 @@
-// tc.cu -- tensor-core (tcgen05 + TMA) scoring path.
+// tc.cu -- tensor-core scoring path for bf16 inputs with head dim 128:
+// tcgen05 MMAs with accumulators in TMEM, operands staged by TMA.
+//
+// What is computed (write-up "DropKV：精确单项输出扰动评分组件", section 核心公式):
+// for every window query t of a KV head's query group, p = softmax(K q / sqrt d)
+// over the causally visible keys, a = sum_j p_j v_j, and for every token j the
+// perturbation weight p_j / (1 - p_j) with
+//     s_j = sum_t (p_j / (1 - p_j))^2 * (||a||^2 - 2 a.v_j + ||v_j||^2)
+// summed over all G*w window queries of the group (the GQA sum; the epilogue
+// divides by G).  No n x w matrix is stored: two streaming passes over K/V.
+//
+// Work split.  The G*w query rows of a KV head are cut into `chunks` chunks of
+// nqc <= 128 rows; the tokens of each (b, h, chunk) into `splits` contiguous
+// tile ranges so that about one CTA runs per SM.  Tiles are 128 tokens.
+//
+// k_tc_pass1 (query-major, one CTA per (b, h, chunk, split)):
+//   S = Q_chunk K_tile^T      tcgen05 M=128 (queries) N=128 (tokens) K=128
+//   online softmax per query row in registers (log2 domain; the reference max
+//   only moves up by more than 8, so exp2 stays <= 256 and O rarely rescales)
+//   P = exp2(S*c - m) written back over S in TMEM as two bf16 planes,
+//   P_hi = P truncated to bf16 and P_lo = bf16(P - P_hi), so P_hi + P_lo holds
+//   P to 2^-16 relative;  O += P_hi V + P_lo V   (A from TMEM, V MN-major).
+//   Two softmax warpgroups take alternate tiles, each with its own S/P buffer,
+//   O accumulator and (m, l): each writes one partial (m, l, O) per row.
+// k_tc_combine: merges the partials of a row into the final max M, normaliser
+//   L and output A = O / L; writes A as bf16 hi/lo planes (same 2^-16 split)
+//   plus the per-query constants (M, 1/L, L, ||A||^2) for pass 2.
+// k_tc_pass2 (token-major, one CTA per (b, h, chunk, split)):
+//   S^T = K_tile Q^T and D = V_tile A_hi^T + V_tile A_lo^T, tcgen05 M=128
+//   (tokens) N=nqc (queries) K=128; each thread owns one token and sums over
+//   the chunk's queries:  e = exp2(S*c - M), p = e / L,
+//   ratio = p + p^2 + p^3 when p < 2^-8 (exact to fp32 rounding), otherwise
+//   e / (L - e) with the singular check (L - e not > 0 => rejected),
+//   s += ratio^2 * (||A||^2 + ||v_j||^2 - 2 D); where that expansion cancels by
+//   more than 32x (A close to v_j: a dominant token) the squared distance is
+//   recomputed directly from fp32 A and v_j.
+//   Two warpgroups take alternate tiles.
+//
+// Warp roles (320 threads): warps 0-3 and 4-7 are the two warpgroups, warp 8
+// issues TMA loads, warp 9 allocates TMEM and issues MMAs (lane 0).  Every
+// wait on an mbarrier is bounded (2 s of %globaltimer); on expiry the kernel
+// records DROPKV_ERR_TIMEOUT, every role leaves its loop and TMEM is freed.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
 #include "internal.h"
+#include "tc_ptx.cuh"
 
 namespace dropkv {
 
-bool tc_available() { return false; }
-int tc_split_target() { return 296; }
+namespace {
+
+using namespace tc;
+
+constexpr int kTok = 128;          // tokens per tile
+constexpr int kHd = 128;           // head dim
+constexpr int kBox = 128 * 128;    // bytes of a 128-row x 64-col bf16 box (SW128)
+constexpr int kTileBytes = 2 * kBox;
+constexpr int kThreads = 320;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kPartStride = 132;   // floats per partial row: O[128], m, l, pad
+constexpr int kMaxCtas = 160;      // split target ceiling (one CTA per SM)
+
+struct TcArgs {
+  int32_t B, Hq, Hkv, n_max, w, G, nqc, chunks;
+  int32_t qbox_rows;     // rows of the pass-1 Q box: min(128, all query rows)
+  int32_t L[kMaxB];
+  int32_t splits[kMaxB];
+  int32_t cta_base[kMaxB + 1];
+  float c_log2;          // log2(e) / sqrt(d)
+  float* partial;        // [ctas][2][128][kPartStride]
+  int32_t* status;
+  __nv_bfloat16* ahi;    // [rows][128]
+  __nv_bfloat16* alo;    // [rows][128]
+  float4* qstat;         // [rows]: (M, 1/L, L, ||A||^2)
+  float* attn_user;      // optional [rows][128]
+  float* stats_user;     // optional [rows][2]
+  float* parts;          // [chunks][B*Hkv*n_max]
+  size_t part_stride;
+  float* attn_f32;       // [rows][128] fp32 window outputs a (read back by pass 2)
+  const __nv_bfloat16* v;  // [B*Hkv][n_max][128] values (rare direct-distance path)
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
+__device__ __forceinline__ uint32_t u32(float f) { return __float_as_uint(f); }
+__device__ __forceinline__ uint32_t pack_bf16_rn(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void decode_cta(const TcArgs& a, int cta, int& b, int& h, int& chunk,
+                                           int& t0, int& t1) {
+  b = 0;
+  while (b + 1 < a.B && cta >= a.cta_base[b + 1]) ++b;
+  const int local = cta - a.cta_base[b];
+  const int sp = local % a.splits[b];
+  const int hc = local / a.splits[b];
+  h = hc / a.chunks;
+  chunk = hc % a.chunks;
+  const int nt = (a.L[b] + kTok - 1) / kTok;
+  t0 = (int)((long long)sp * nt / a.splits[b]);
+  t1 = (int)((long long)(sp + 1) * nt / a.splits[b]);
+}
+
+// Records a timeout once and raises the CTA-wide abort flag.
+__device__ __forceinline__ void fail(const TcArgs& a, volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicMax(a.status, (int)DROPKV_ERR_TIMEOUT);
+}
+// Bounded wait whose outcome is the same for every lane of the warp, so the
+// warp stays converged for the .sync.aligned tcgen05 instructions after it.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  const bool ok = mbar_wait(bar, parity, kWaitNs);
+  return __all_sync(0xffffffffu, ok);
+}
+__device__ __forceinline__ bool warp_aborted(volatile int* f) {
+  return __any_sync(0xffffffffu, *f != 0);
+}
+
+// K-major SW128 operand of `rows` rows, head dim 128 in two 64-wide boxes:
+// descriptor of the 16-wide K slice kk (0..7).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int rows, int kk) {
+  return sdesc_sw128(base + (uint32_t)((kk >> 2) * rows * 128 + (kk & 3) * 32), 16, 1024);
+}
+// V tile as the MN-major B operand of P V: N = head dim (two 64-wide boxes,
+// 16 KB apart), K = tokens (128-byte rows); slice kk covers tokens 16kk..16kk+15.
+__device__ __forceinline__ uint64_t vmn_desc(uint32_t base, int kk) {
+  return sdesc_sw128(base + (uint32_t)(kk * 16 * 128), kBox, 1024);
+}
+
+// =========================== pass 1 =========================================
+__global__ void __launch_bounds__(kThreads, 1)
+k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + kTileBytes;        // 2 stages
+  uint8_t* sV = smem + 3 * kTileBytes;    // 2 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * kTileBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1 KB alignment
+    if (threadIdx.x == 0) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
+    return;
+  }
+  int b, h, chunk, t0, t1;
+  decode_cta(a, blockIdx.x, b, h, chunk, t0, t1);
+  const int T = t1 - t0;
+  const int L = a.L[b];
+  const uint32_t BQ = smem_u32(&bars[0]);
+  auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto KE = [&](int s) { return smem_u32(&bars[3 + s]); };
+  auto VF = [&](int s) { return smem_u32(&bars[5 + s]); };
+  auto VE = [&](int s) { return smem_u32(&bars[7 + s]); };
+  auto SF = [&](int s) { return smem_u32(&bars[9 + s]); };
+  auto PF = [&](int s) { return smem_u32(&bars[11 + s]); };
+  auto OD = [&](int s) { return smem_u32(&bars[13 + s]); };
+  if (threadIdx.x == 0) {
+    mbar_init(BQ, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1); mbar_init(VE(s), 1);
+      mbar_init(SF(s), 1); mbar_init(PF(s), 128); mbar_init(OD(s), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const int z = b * a.Hkv + h;
+  const int qrow0 = (b * a.Hkv + h) * a.G * a.w + chunk * a.nqc;
+
+  if (warp == 8) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+      mbar_expect_tx(BQ, 2u * 128u * (uint32_t)a.qbox_rows);
+      tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
+      tma_load_2d(smem_u32(sQ) + kBox, &tmQ, BQ, 64, qrow0);
+      auto load = [&](uint8_t* buf, uint32_t full, uint32_t empty, const CUtensorMap* m, int i) {
+        const int s = i & 1, ph = (i >> 1) & 1;
+        if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); return false; }
+        mbar_expect_tx(full, kTileBytes);
+        const uint32_t dst = smem_u32(buf + s * kTileBytes);
+        tma_load_3d(dst, m, full, 0, (t0 + i) * kTok, z);
+        tma_load_3d(dst + kBox, m, full, 64, (t0 + i) * kTok, z);
+        return true;
+      };
+      bool ok = T > 0 ? load(sK, KF(0), KE(0), &tmK, 0) : true;
+      for (int j = 0; j < T && ok && !*abort_flag; ++j) {
+        if (j + 1 < T) ok = load(sK, KF((j + 1) & 1), KE((j + 1) & 1), &tmK, j + 1);
+        if (ok) ok = load(sV, VF(j & 1), VE(j & 1), &tmV, j);
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T
+    constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);    // O += P V (V MN-major)
+    bool ok = warp_wait(BQ, 0);
+    if (!ok) fail(a, abort_flag);
+    const uint32_t qbase = smem_u32(sQ);
+    auto issue_S = [&](int i) {
+      const int s = i & 1, ph = (i >> 1) & 1;
+      if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t kb = smem_u32(sK + s * kTileBytes);
+        const uint32_t dS = tbase + (uint32_t)(s * 128);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(dS, kmajor_desc(qbase, 128, kk), kmajor_desc(kb, 128, kk), IDS, kk > 0);
+        mma_commit(KE(s));
+        mma_commit(SF(s));
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_PV = [&](int i) {
+      const int s = i & 1, ph = (i >> 1) & 1;
+      if (!warp_wait(PF(s), ph)) { fail(a, abort_flag); return false; }
+      if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
+      uint8_t* vb = sV + s * kTileBytes;
+      const int tile0 = (t0 + i) * kTok;
+      if (tile0 + kTok > L) {
+        // rows at or beyond L hold no data (possibly NaN): zero them so that the
+        // P = 0 weights of those rows contribute exactly 0 to O
+        const int r0 = L - tile0;
+        for (int idx = r0 * 8 + lane; idx < kTok * 8; idx += 32) {
+          const int r = idx >> 3, c16 = idx & 7;
+          *reinterpret_cast<uint4*>(vb + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vb + kBox + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t vbase = smem_u32(vb);
+        const uint32_t dO = tbase + 256u + (uint32_t)(s * 128);
+        const uint32_t pS = tbase + (uint32_t)(s * 128);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(dO, pS + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), vmn_desc(vbase, kk), IDP,
+                 (i >= 2 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(dO, pS + (uint32_t)(32 * (kk >> 1) + 16 + 8 * (kk & 1)), vmn_desc(vbase, kk), IDP,
+                 1u);
+        mma_commit(VE(s));
+        mma_commit(OD(s));
+      }
+      __syncwarp();
+      return true;
+    };
+    if (ok && T > 0) ok = issue_S(0);
+    for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
+      if (j + 1 < T) ok = issue_S(j + 1);
+      if (ok) ok = issue_PV(j);
+    }
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int wg = warp >> 2, wl = warp & 3;
+    const int row = wl * 32 + lane;  // query row within the chunk
+    const bool valid_row = row < a.nqc;
+    const int Prow = valid_row ? L - a.w + (chunk * a.nqc + row) % a.w : L - 1;
+    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+    const uint32_t tS = tbase + (uint32_t)(wg * 128) + lane_off;
+    const uint32_t tO = tbase + 256u + (uint32_t)(wg * 128) + lane_off;
+    const float c = a.c_log2;
+    float m_ref = -INFINITY, l = 0.f;
+    int n = 0;
+    for (int j = wg; j < T; j += 2, ++n) {
+      if (!warp_wait(SF(wg), n & 1)) { fail(a, abort_flag); break; }
+      if (warp_aborted(abort_flag)) break;
+      tc_fence_after();
+      const int tile0 = (t0 + j) * kTok;
+      const bool masked = tile0 + kTok - 1 > L - a.w;
+      // sweep 1: row max of this tile
+      float mx = -INFINITY;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[64];
+        tmem_ld32x2(tS + half * 64, tS + half * 64 + 32, r);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) {
+          const float x = (!masked || tile0 + half * 64 + u <= Prow) ? f32(r[u]) : -INFINITY;
+          mx = fmaxf(mx, x);
+        }
+      }
+      const float mt = mx * c;
+      float fac = 1.f;
+      bool resc = false;
+      if (mt > m_ref + 8.f) {
+        if (m_ref != -INFINITY) {
+          fac = ex2(m_ref - mt);
+          resc = (n > 0);
+        }
+        m_ref = mt;
+        l *= fac;
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        // O of this warpgroup must not be in flight: wait for its previous P V
+        if (!warp_wait(OD(wg), (n - 1) & 1)) { fail(a, abort_flag); break; }
+        tc_fence_after();
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
+          tmem_st32(tO + cc * 32, o);
+        }
+        tmem_st_wait();
+      }
+      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // sweep 2: P = exp2(S c - mu) as hi/lo bf16 planes over the S columns
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tS + cc * 32, r);
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int u2 = 0; u2 < 16; ++u2) {
+          const int u = 2 * u2;
+          const int tok = tile0 + cc * 32 + u;
+          const float x0 = (!masked || tok <= Prow) ? f32(r[u]) : -INFINITY;
+          const float x1 = (!masked || tok + 1 <= Prow) ? f32(r[u + 1]) : -INFINITY;
+          const float e0 = ex2(fmaf(x0, c, -mu));
+          const float e1 = ex2(fmaf(x1, c, -mu));
+          l += e0 + e1;
+          const uint32_t h0 = u32(e0) & 0xFFFF0000u, h1 = u32(e1) & 0xFFFF0000u;
+          hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);
+          lo[u2] = pack_bf16_rn(e0 - f32(h0), e1 - f32(h1));
+        }
+        tmem_st16(tS + cc * 32, hi);
+        tmem_st16(tS + cc * 32 + 16, lo);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(PF(wg));
+    }
+    // partial (m, l, O) of this warpgroup for its row
+    float* out = a.partial + (((size_t)blockIdx.x * 2 + wg) * 128 + row) * kPartStride;
+    bool have = n > 0 && !warp_aborted(abort_flag);
+    if (have) {
+      if (!warp_wait(OD(wg), (n - 1) & 1)) {
+        fail(a, abort_flag);
+        have = false;
+      }
+      tc_fence_after();
+    }
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t o[32];
+      if (have) tmem_ld32(tO + cc * 32, o);
+      if (valid_row) {
+#pragma unroll
+        for (int u = 0; u < 32; u += 4)
+          *reinterpret_cast<float4*>(out + cc * 32 + u) =
+              have ? make_float4(f32(o[u]), f32(o[u + 1]), f32(o[u + 2]), f32(o[u + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    if (valid_row) {
+      out[128] = have ? m_ref : -INFINITY;
+      out[129] = have ? l : 0.f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// =========================== combine ========================================
+// One warp per query row: merge the 2 * splits partials of its (b, h, chunk).
+__global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows = a.B * a.Hq * a.w;
+  const int r = blockIdx.x * 4 + warp;
+  if (r >= rows) return;
+  const int b = r / (a.Hq * a.w);
+  const int hq = (r / a.w) % a.Hq;
+  const int t = r % a.w;
+  const int h = hq / a.G;
+  const int gr = (hq % a.G) * a.w + t;
+  const int chunk = gr / a.nqc, rr = gr % a.nqc;
+  const int cta0 = a.cta_base[b] + (h * a.chunks + chunk) * a.splits[b];
+  const int np = 2 * a.splits[b];
+  auto P = [&](int i) {
+    return a.partial + (((size_t)cta0 * 2 + i) * 128 + rr) * kPartStride;
+  };
+  float M = -INFINITY;
+  for (int i = lane; i < np; i += 32) M = fmaxf(M, P(i)[128]);
+  M = warp_max(M);
+  float Lsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < np; ++i) {
+    const float* p = P(i);
+    const float mi = p[128];
+    const float wgt = (mi == -INFINITY) ? 0.f : ex2(mi - M);
+    Lsum += wgt * p[129];
+    const float4 o = *reinterpret_cast<const float4*>(p + lane * 4);
+    acc.x = fmaf(wgt, o.x, acc.x);
+    acc.y = fmaf(wgt, o.y, acc.y);
+    acc.z = fmaf(wgt, o.z, acc.z);
+    acc.w = fmaf(wgt, o.w, acc.w);
+  }
+  const float inv = 1.f / Lsum;
+  const float A[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  const float nA = warp_sum(A[0] * A[0] + A[1] * A[1] + A[2] * A[2] + A[3] * A[3]);
+  uint32_t hw[2], lw[2];
+  for (int i = 0; i < 2; ++i) {
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(A[2 * i], A[2 * i + 1]);
+    const float h0 = __bfloat162float(hv.x), h1 = __bfloat162float(hv.y);
+    const __nv_bfloat162 lv = __floats2bfloat162_rn(A[2 * i] - h0, A[2 * i + 1] - h1);
+    hw[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    lw[i] = *reinterpret_cast<const uint32_t*>(&lv);
+  }
+  *reinterpret_cast<uint2*>(a.ahi + (size_t)r * kHd + lane * 4) = make_uint2(hw[0], hw[1]);
+  *reinterpret_cast<uint2*>(a.alo + (size_t)r * kHd + lane * 4) = make_uint2(lw[0], lw[1]);
+  *reinterpret_cast<float4*>(a.attn_f32 + (size_t)r * kHd + lane * 4) =
+      make_float4(A[0], A[1], A[2], A[3]);
+  if (a.attn_user)
+    *reinterpret_cast<float4*>(a.attn_user + (size_t)r * kHd + lane * 4) =
+        make_float4(A[0], A[1], A[2], A[3]);
+  if (lane == 0) {
+    a.qstat[r] = make_float4(M, inv, Lsum, nA);
+    if (a.stats_user) {
+      a.stats_user[2 * (size_t)r] = M * 0.69314718055994531f;  // log2 units -> natural
+      a.stats_user[2 * (size_t)r + 1] = Lsum;
+    }
+  }
+}
+
+// =========================== pass 2 =========================================
+// ||a - v||^2 taken directly (fp32 a, bf16 v, both from global memory).  Used
+// only where the expansion ||a||^2 + ||v||^2 - 2 a.v cancels by more than 32x,
+// i.e. a is close to v (a dominant token, p_j near 1).
+__device__ __noinline__ float direct_sqdist(const float* A, const __nv_bfloat16* v) {
+  float s = 0.f;
+  for (int c = 0; c < kHd; c += 4) {
+    const float4 a4 = *reinterpret_cast<const float4*>(A + c);
+    const uint2 v4 = *reinterpret_cast<const uint2*>(v + c);
+    const float d0 = a4.x - __uint_as_float(v4.x << 16);
+    const float d1 = a4.y - __uint_as_float(v4.x & 0xFFFF0000u);
+    const float d2 = a4.z - __uint_as_float(v4.y << 16);
+    const float d3 = a4.w - __uint_as_float(v4.y & 0xFFFF0000u);
+    s = fmaf(d0, d0, s);
+    s = fmaf(d1, d1, s);
+    s = fmaf(d2, d2, s);
+    s = fmaf(d3, d3, s);
+  }
+  return s;
+}
+
+template <bool kMasked>
+__device__ __forceinline__ void score_cols(const uint32_t* xs, const uint32_t* ds, int ncol,
+                                           int col0, const float4* qc, const int* pcol, int tok,
+                                           float c, float nv, float& acc, int& sing,
+                                           const float* arows, const __nv_bfloat16* vrow) {
+#pragma unroll
+  for (int u = 0; u < ncol; ++u) {
+    const int col = col0 + u;
+    const float4 k = qc[col];  // (M, 1/L, L, ||A||^2), broadcast
+    const float e = ex2(fmaf(f32(xs[u]), c, -k.x));
+    const float p = e * k.y;
+    float ratio = fmaf(p, fmaf(p, p, p), p);  // p + p^2 + p^3 = p / (1 - p) for p < 2^-8
+    const bool vis = !kMasked || tok <= pcol[col];
+    const float base = k.w + nv;
+    float zt = fmaf(-2.f, f32(ds[u]), base);  // ||A||^2 + ||v||^2 - 2 A.v
+    const bool big = p >= 0.00390625f;
+    const bool cancel = zt < 0.03125f * base;
+    if (vis && (big || cancel)) {  // rare: dominant tokens only
+      if (big) {
+        const float den = k.z - e;  // (1 - p) L
+        if (!(den > 0.f)) sing = 1;
+        ratio = __fdiv_rn(e, den);
+      }
+      if (cancel) zt = direct_sqdist(arows + (size_t)col * kHd, vrow);
+    }
+    const float contrib = ratio * ratio * zt;
+    if (vis) acc += contrib;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmAhi,
+           const __grid_constant__ CUtensorMap tmAlo, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int nqc = a.nqc;
+  uint8_t* sK = smem;                        // 2 stages
+  uint8_t* sV = smem + 2 * kTileBytes;       // 2 stages
+  uint8_t* sQ = smem + 4 * kTileBytes;       // nqc rows x 2 boxes
+  uint8_t* sAh = sQ + nqc * 256;
+  uint8_t* sAl = sAh + nqc * 256;
+  float4* qc = reinterpret_cast<float4*>(sAl + nqc * 256);
+  int* pcol = reinterpret_cast<int*>(qc + nqc);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(pcol + nqc);  // 13 barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
+    return;
+  }
+  int b, h, chunk, t0, t1;
+  decode_cta(a, blockIdx.x, b, h, chunk, t0, t1);
+  const int T = t1 - t0;
+  const int L = a.L[b];
+  const uint32_t BQ = smem_u32(&bars[0]);
+  auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto KE = [&](int s) { return smem_u32(&bars[3 + s]); };
+  auto VF = [&](int s) { return smem_u32(&bars[5 + s]); };
+  auto VE = [&](int s) { return smem_u32(&bars[7 + s]); };
+  auto MD = [&](int s) { return smem_u32(&bars[9 + s]); };   // MMAs of a tile done
+  auto TF = [&](int s) { return smem_u32(&bars[11 + s]); };  // TMEM buffer read out
+  const int qrow0 = (b * a.Hkv + h) * a.G * a.w + chunk * nqc;
+  if (threadIdx.x == 0) {
+    mbar_init(BQ, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1);
+      mbar_init(VE(s), 1 + 4);  // MMA commit + the 4 warps that read ||v||^2
+      mbar_init(MD(s), 1); mbar_init(TF(s), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < nqc) {
+    const int i = threadIdx.x;
+    qc[i] = a.qstat[qrow0 + i];
+    pcol[i] = L - a.w + (chunk * nqc + i) % a.w;
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const int z = b * a.Hkv + h;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmAhi); prefetch_tmap(&tmAlo);
+      prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+      mbar_expect_tx(BQ, 3 * nqc * 256);
+      tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
+      tma_load_2d(smem_u32(sQ) + nqc * 128, &tmQ, BQ, 64, qrow0);
+      tma_load_2d(smem_u32(sAh), &tmAhi, BQ, 0, qrow0);
+      tma_load_2d(smem_u32(sAh) + nqc * 128, &tmAhi, BQ, 64, qrow0);
+      tma_load_2d(smem_u32(sAl), &tmAlo, BQ, 0, qrow0);
+      tma_load_2d(smem_u32(sAl) + nqc * 128, &tmAlo, BQ, 64, qrow0);
+      for (int j = 0; j < T && !*abort_flag; ++j) {  // single thread: no warp vote needed
+        const int s = j & 1, ph = (j >> 1) & 1;
+        const uint32_t dk = smem_u32(sK + s * kTileBytes), dv = smem_u32(sV + s * kTileBytes);
+        if (!mbar_wait(KE(s), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
+        mbar_expect_tx(KF(s), kTileBytes);
+        tma_load_3d(dk, &tmK, KF(s), 0, (t0 + j) * kTok, z);
+        tma_load_3d(dk + kBox, &tmK, KF(s), 64, (t0 + j) * kTok, z);
+        if (!mbar_wait(VE(s), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
+        mbar_expect_tx(VF(s), kTileBytes);
+        tma_load_3d(dv, &tmV, VF(s), 0, (t0 + j) * kTok, z);
+        tma_load_3d(dv + kBox, &tmV, VF(s), 64, (t0 + j) * kTok, z);
+      }
+    }
+  } else if (warp == 9) {
+    const uint32_t IDT = idesc_bf16(128, nqc, false, false);
+    bool ok = warp_wait(BQ, 0);
+    if (!ok) fail(a, abort_flag);
+    const uint32_t qb = smem_u32(sQ), hb = smem_u32(sAh), lb = smem_u32(sAl);
+    for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
+      const int s = j & 1, ph = (j >> 1) & 1;
+      const uint32_t dS = tbase + (uint32_t)(s * 256), dD = dS + 128u;
+      if (!warp_wait(TF(s), ph ^ 1) || !warp_wait(KF(s), ph)) {
+        fail(a, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t kb = smem_u32(sK + s * kTileBytes), vb = smem_u32(sV + s * kTileBytes);
+      if (lane == 0) {
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(dS, kmajor_desc(kb, 128, kk), kmajor_desc(qb, nqc, kk), IDT, kk > 0);
+        mma_commit(KE(s));
+      }
+      __syncwarp();
+      if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); break; }
+      tc_fence_after();
+      if (lane == 0) {
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(dD, kmajor_desc(vb, 128, kk), kmajor_desc(hb, nqc, kk), IDT, kk > 0);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(dD, kmajor_desc(vb, 128, kk), kmajor_desc(lb, nqc, kk), IDT, 1u);
+        mma_commit(VE(s));
+        mma_commit(MD(s));
+      }
+      __syncwarp();
+    }
+  } else {
+    const int wg = warp >> 2, wl = warp & 3;
+    const int row = wl * 32 + lane;  // token within the tile
+    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+    const uint32_t tS = tbase + (uint32_t)(wg * 256) + lane_off, tD = tS + 128u;
+    const float c = a.c_log2;
+    int sing = 0;
+    int n = 0;
+    for (int j = wg; j < T; j += 2, ++n) {
+      const int ph = n & 1;
+      const int tile0 = (t0 + j) * kTok;
+      const int tok = tile0 + row;
+      // ||v_j||^2 from the staged V tile (the order of the squares does not
+      // matter, so the 128-byte swizzle only chooses a conflict-free order)
+      if (!warp_wait(VF(wg), ph)) { fail(a, abort_flag); break; }
+      const uint8_t* vrow = sV + wg * kTileBytes + row * 128;
+      float nv = 0.f;
+#pragma unroll
+      for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(vrow + bx * kBox + ((i ^ (row & 7)) * 16));
+          const uint32_t wv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float lo = __uint_as_float(wv[k] << 16), hi = __uint_as_float(wv[k] & 0xFFFF0000u);
+            nv = fmaf(lo, lo, nv);
+            nv = fmaf(hi, hi, nv);
+          }
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(VE(wg));
+      if (!warp_wait(MD(wg), ph)) { fail(a, abort_flag); break; }
+      if (warp_aborted(abort_flag)) break;
+      tc_fence_after();
+      const bool masked = tile0 + kTok - 1 > L - a.w;
+      const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
+      const __nv_bfloat16* vrow_g = a.v + ((size_t)z * a.n_max + (tok < L ? tok : 0)) * kHd;
+      float acc = 0.f;
+      int col = 0;
+      for (; col + 32 <= nqc; col += 32) {
+        uint32_t xs[32], ds[32];
+        tmem_ld32(tS + col, xs);
+        tmem_ld32(tD + col, ds);
+        if (masked)
+          score_cols<true>(xs, ds, 32, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
+        else
+          score_cols<false>(xs, ds, 32, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
+      }
+      if (col < nqc) {  // nqc % 32 == 16
+        uint32_t xs[16], ds[16];
+        tmem_ld16(tS + col, xs);
+        tmem_ld16(tD + col, ds);
+        if (masked)
+          score_cols<true>(xs, ds, 16, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
+        else
+          score_cols<false>(xs, ds, 16, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(TF(wg));
+      if (tok < L) a.parts[(size_t)chunk * a.part_stride + (size_t)z * a.n_max + tok] = acc;
+    }
+    if (sing) atomicMax(a.status, (int)DROPKV_ERR_SINGULAR);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// =========================== host side ======================================
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows][128] row-major, box = 64 columns x box_rows rows, 128B swizzle.
+bool map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kHd, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kHd * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [heads][n_max][128], box = 64 columns x 128 tokens x 1 head.
+bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kHd, (cuuint64_t)n_max, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)kHd * 2, (cuuint64_t)n_max * kHd * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kTok, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t pass1_smem() { return 5 * (size_t)kTileBytes + 16 * 8 + 64; }
+size_t pass2_smem(int nqc) {
+  return 4 * (size_t)kTileBytes + 3 * (size_t)nqc * 256 + (size_t)nqc * 16 + (size_t)nqc * 4 +
+         13 * 8 + 8;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+}  // namespace
+
+bool tc_available() { return true; }
+int tc_split_target() { return kMaxCtas; }
 int tc_launch_count() { return 3; }
 
-cudaError_t launch_tc_scores(const dropkv_shape&, const void*, const void*, const void*,
-                             const Lens&, const ScoresLayout&, char*, float*, float*, int32_t*,
-                             cudaStream_t, KernelEvents&) {
-  return cudaErrorNotSupported;
+// Splits per batch row so that the CTAs (one per SM) carry balanced tile
+// counts: greedily give another split to the row whose CTAs are longest.
+void tc_splits(const Lens& lens, int units_per_row, int budget, int32_t* splits) {
+  int total = 0;
+  for (int b = 0; b < lens.B; ++b) {
+    splits[b] = 1;
+    total += units_per_row;
+  }
+  for (;;) {
+    int best = -1;
+    double worst = 0;
+    for (int b = 0; b < lens.B; ++b) {
+      const int nt = (lens.L[b] + kTok - 1) / kTok;
+      const double per = (double)nt / splits[b];
+      if (splits[b] < nt && per > worst) {
+        worst = per;
+        best = b;
+      }
+    }
+    if (best < 0 || total + units_per_row > budget) break;
+    splits[best] += 1;
+    total += units_per_row;
+  }
+}
+
+cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k, const void* v,
+                             const Lens& lens, const ScoresLayout& lay, char* ws, float* attn_out,
+                             float* stats_out, int32_t* status, cudaStream_t st,
+                             KernelEvents& kev) {
+  const TcPlan plan = tc_plan(s);
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = lens.B;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.n_max = s.n_max;
+  a.w = s.window;
+  a.G = s.Hq / s.Hkv;
+  a.nqc = plan.nqc;
+  a.chunks = plan.chunks;
+  for (int i = 0; i < lens.B; ++i) a.L[i] = lens.L[i];
+  const int units = s.Hkv * plan.chunks;
+  const int budget = std::min(num_sms(), kMaxCtas);
+  tc_splits(lens, units, std::max(budget, units * lens.B), a.splits);
+  a.cta_base[0] = 0;
+  for (int i = 0; i < lens.B; ++i) a.cta_base[i + 1] = a.cta_base[i] + units * a.splits[i];
+  const int ctas = a.cta_base[lens.B];
+  a.c_log2 = (float)(1.4426950408889634 / sqrt((double)s.d));
+  a.partial = reinterpret_cast<float*>(ws + lay.tc_partial);
+  a.status = status;
+  a.ahi = reinterpret_cast<__nv_bfloat16*>(ws + lay.tc_ahi);
+  a.alo = reinterpret_cast<__nv_bfloat16*>(ws + lay.tc_alo);
+  a.qstat = reinterpret_cast<float4*>(ws + lay.tc_qstat);
+  a.attn_user = attn_out;
+  a.stats_user = stats_out;
+  a.parts = reinterpret_cast<float*>(ws + lay.parts);
+  a.part_stride = (size_t)lens.B * s.Hkv * s.n_max;
+  a.attn_f32 = reinterpret_cast<float*>(ws + lay.attn);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+
+  const uint64_t rows = (uint64_t)lens.B * s.Hq * s.window;
+  a.qbox_rows = (int32_t)std::min<uint64_t>(128, rows);
+  CUtensorMap mQ1, mQ2, mK, mV, mAh, mAl;
+  if (!map_2d(&mQ1, q, rows, (uint32_t)a.qbox_rows) || !map_2d(&mQ2, q, rows, (uint32_t)plan.nqc) ||
+      !map_3d(&mK, k, (uint64_t)lens.B * s.Hkv, (uint64_t)s.n_max) ||
+      !map_3d(&mV, v, (uint64_t)lens.B * s.Hkv, (uint64_t)s.n_max) ||
+      !map_2d(&mAh, a.ahi, rows, (uint32_t)plan.nqc) ||
+      !map_2d(&mAl, a.alo, rows, (uint32_t)plan.nqc))
+    return cudaErrorNotSupported;
+
+  const size_t sm1 = pass1_smem(), sm2 = pass2_smem(plan.nqc);
+  cudaError_t e = cudaFuncSetAttribute(k_tc_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sm1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_tc_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+  if (e != cudaSuccess) return e;
+
+  kev.begin(st);
+  k_tc_pass1<<<ctas, kThreads, sm1, st>>>(mQ1, mK, mV, a);
+  kev.end(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  kev.begin(st);
+  k_tc_combine<<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(a);
+  kev.end(st);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  kev.begin(st);
+  k_tc_pass2<<<ctas, kThreads, sm2, st>>>(mQ2, mAh, mAl, mK, mV, a);
+  kev.end(st);
+  return cudaGetLastError();
 }
 
 }  // namespace dropkv
