@@ -164,6 +164,30 @@ DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, co
                             int32_t max_evict, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/*
+ * dropkv_select without a workspace, for callers that cannot allocate device
+ * memory (for example code inside a serving engine that owns all device memory
+ * through its own pool, or a path that cannot afford cudaMalloc's implicit
+ * device synchronisation).  The paper has no counterpart: this is an interface
+ * variant of the eviction step above, with the same arguments minus the
+ * workspace and the same results.
+ *   Scratch: a 1 MiB array of static device memory inside the library, held by
+ *   every GPU that loads the library until the process exits.  Sizes whose
+ *   dropkv_select_workspace_bytes(min(B, 64), Hkv, n_max) exceeds 1 MiB are
+ *   rejected with DROPKV_ERR_WORKSPACE before anything is enqueued.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  No call allocates or frees memory.
+ *   All calls share the array and it keeps the last call's contents (every
+ *   call resets what must start at zero): calls whose work overlaps on the GPU,
+ *   e.g. on two streams at once, race and must be serialised by the caller.
+ */
+DROPKV_API dropkv_status dropkv_select_noalloc(int32_t B, int32_t Hkv, int32_t n_max,
+                                               const float* scores, const int32_t* lengths,
+                                               const int32_t* keep_counts, int32_t* keep_idx,
+                                               int32_t max_keep, int32_t* evict_idx,
+                                               int32_t max_evict, void* stream);
+
 /* Which path DROPKV_PATH_AUTO picks for this shape (DROPKV_PATH_SIMT or
  * DROPKV_PATH_TENSOR); no device needed.  Returns -1 for an invalid shape. */
 DROPKV_API int32_t dropkv_auto_path(const dropkv_shape* shape);

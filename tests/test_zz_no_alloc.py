@@ -1,0 +1,83 @@
+"""dropkv_select_noalloc: the eviction step for callers that cannot allocate.
+
+Callers such as a serving engine that owns every byte of device memory through
+its own pool (or a path that cannot afford cudaMalloc's implicit device
+synchronisation) cannot hand dropkv_select a workspace.  dropkv_select_noalloc
+takes none and uses a 1 MiB scratch array compiled into the library.  This
+test calls it through the C ABI twice in a row and checks that both calls give
+exactly the keep / evict lists of dropkv_select (integer outputs: exact), and
+that sizes beyond the scratch are refused before anything runs.
+
+The file is named so that pytest collects it last.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_eviction_scores_b200 as dk
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _bind():
+    L = dk.lib()
+    i32, vp = ctypes.c_int32, ctypes.c_void_p
+    ip = ctypes.POINTER(ctypes.c_int32)
+    L.dropkv_select_noalloc.argtypes = [i32, i32, i32, vp, ip, ip, vp, i32, vp, i32, vp]
+    L.dropkv_select_noalloc.restype = i32
+    return L
+
+
+def _arr(vals):
+    return (ctypes.c_int32 * len(vals))(*[int(x) for x in vals])
+
+
+def _scores(B, Hkv, n_max, lengths, seed):
+    rng = np.random.default_rng(seed)
+    s = rng.integers(0, 64, size=(B, Hkv, n_max)).astype(np.float32) / 16.0  # many ties
+    for b, L in enumerate(lengths):
+        s[b, :, max(0, L - 4): L] = np.inf
+        s[b, :, L:] = np.nan
+    return torch.from_numpy(s).to(DEV)
+
+
+def test_noalloc_select_matches_select_on_two_calls_in_a_row():
+    L = _bind()
+    B, Hkv, n_max = 3, 4, 20000
+    lengths = [20000, 9000, 4097]
+    keep = [1000, 4500, 4097]
+    scores = _scores(B, Hkv, n_max, lengths, 11)
+    ref_keep, ref_ev = dk.dropkv_select(scores, keep, lengths)
+    torch.cuda.synchronize()
+    max_keep, max_evict = ref_keep.shape[2], ref_ev.shape[2]
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for call in range(2):
+        keep_idx = torch.full((B, Hkv, max_keep), 7, dtype=torch.int32, device=DEV)
+        ev_idx = torch.full((B, Hkv, max_evict), 7, dtype=torch.int32, device=DEV)
+        st = L.dropkv_select_noalloc(B, Hkv, n_max, ctypes.c_void_p(scores.data_ptr()),
+                                     _arr(lengths), _arr(keep), ctypes.c_void_p(keep_idx.data_ptr()),
+                                     max_keep, ctypes.c_void_p(ev_idx.data_ptr()), max_evict, stream)
+        assert st == dk.OK, f"call {call}: status {st}"
+        torch.cuda.synchronize()
+        assert torch.equal(keep_idx, ref_keep), f"call {call}: keep lists differ"
+        assert torch.equal(ev_idx, ref_ev), f"call {call}: evict lists differ"
+
+
+def test_noalloc_select_refuses_sizes_beyond_its_scratch():
+    L = _bind()
+    B, Hkv, n_max = 64, 4, 64  # 256 segments: the histograms alone need 2 MiB
+    assert dk.select_workspace_bytes(B, Hkv, n_max) > (1 << 20)
+    lengths = [n_max] * B
+    keep = [n_max // 2] * B
+    scores = _scores(B, Hkv, n_max, lengths, 3)  # real buffers of the declared sizes
+    keep_idx = torch.empty(B, Hkv, n_max // 2, dtype=torch.int32, device=DEV)
+    ev_idx = torch.empty(B, Hkv, n_max // 2, dtype=torch.int32, device=DEV)
+    st = L.dropkv_select_noalloc(B, Hkv, n_max, ctypes.c_void_p(scores.data_ptr()), _arr(lengths),
+                                 _arr(keep), ctypes.c_void_p(keep_idx.data_ptr()), n_max // 2,
+                                 ctypes.c_void_p(ev_idx.data_ptr()), n_max // 2, None)
+    assert st == dk.ERR_WORKSPACE
