@@ -89,6 +89,27 @@ def visible_elements(spec):
     return per_query_head * spec.Hq
 
 
+# ----------------------------------------------------------- multi-rank ----
+
+def rank_seed(rank):
+    """Each rank scores its own independent input set (weak scaling)."""
+    return 42 + rank
+
+
+def max_over_ranks(ms, dist, device):
+    """The slowest rank's time: the job is done when every rank is."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world, tokens_per_rank, ms):
+    """Tokens scored per second by all ranks together."""
+    return world * tokens_per_rank / (ms * 1e-3)
+
+
 # ---------------------------------------------------------------- clocks ----
 
 class ClockSampler:
@@ -283,18 +304,14 @@ def run_e2e(dk, wl, q, k, v, scores, status, step, E, dist, dev, world):
         e2e_step()
     a1.record()
     torch.cuda.synchronize()
-    e2e_ms = a0.elapsed_time(a1)
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev) / E
     if dist:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
         dist.barrier()
-    e2e_ms /= E
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = sum(t.numel() * t.element_size() for t in (sc_h, kp_h, ev_h, st_h))
 
     tokens = sum(wl.lengths)
-    return {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT,
+    return {"value": whole_job_value(world, tokens, e2e_ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
@@ -316,7 +333,7 @@ def run_ours(args):
     dk.lib()
 
     spec = W.config_spec(args.config)
-    wl = W.generate(spec, 42 + rank)
+    wl = W.generate(spec, rank_seed(rank))
     q, k, v = wl.q.to(dev), wl.k.to(dev), wl.v.to(dev)
     shape = dk.make_shape(q, k, spec.window, spec.pool)
     path = {dk.PATH_SIMT: "simt", dk.PATH_TENSOR: "tensor"}[
@@ -359,12 +376,7 @@ def run_ours(args):
     if dist:
         dist.barrier()
     clk = clocks.stop()
-    ms_total = t0.elapsed_time(t1)
-    if dist:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
-    ms = ms_total / K
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, dev) / K
     kern_us = {}
     for j, name in enumerate(names):
         kern_us[name] = statistics.mean(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1])
@@ -378,7 +390,7 @@ def run_ours(args):
     if E > 0:
         e2e = run_e2e(dk, wl, q, k, v, scores, status, step, E, dist, dev, world)
     tokens = sum(wl.lengths)
-    value = world * tokens / (ms * 1e-3)
+    value = whole_job_value(world, tokens, ms)
     hbm_peak, tc_peak, sm_mhz, peak_src = peaks()
     dominant = max(kern_us, key=kern_us.get)
     roof = roofline(dominant, spec, kern_us[dominant], hbm_peak, tc_peak, sm_mhz)
