@@ -96,7 +96,7 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   o = align_up(o + rows * s.d * sizeof(double), kAlign);
   l.parts = o;
   o = align_up(o + (size_t)l.nparts * Bs * s.Hkv * (size_t)s.n_max * sizeof(float), kAlign);
-  l.tc_partial = l.tc_ahi = l.tc_alo = l.tc_qstat = o;
+  l.tc_partial = l.tc_ahi = l.tc_alo = l.tc_qstat = l.tc_nv = o;
   if (tc) {
     const TcPlan p = tc_plan(s);
     // pass-1 partials: at most (split target + one per (b, h, chunk)) CTAs,
@@ -110,6 +110,8 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
     o = align_up(o + rows * s.d * 2, kAlign);
     l.tc_qstat = o;
     o = align_up(o + rows * 4 * sizeof(float), kAlign);
+    l.tc_nv = o;
+    o = align_up(o + (size_t)Bs * s.Hkv * (size_t)s.n_max * sizeof(float), kAlign);
   }
   l.total = o;
   return l;

@@ -84,6 +84,7 @@ struct TcArgs {
   size_t part_stride;
   float* attn_f32;       // [rows][128] fp32 window outputs a (read back by pass 2)
   const __nv_bfloat16* v;  // [B*Hkv][n_max][128] values (rare direct-distance path)
+  float* nvbuf;          // [B*Hkv][n_max] ||v_j||^2, written by pass 1, read by pass 2
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -169,7 +170,8 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1); mbar_init(VE(s), 1);
+      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1);
+      mbar_init(VE(s), 1 + 4);  // P V commit + the 4 warps that read ||v||^2 from the tile
       mbar_init(SF(s), 1); mbar_init(PF(s), 128); mbar_init(OD(s), 1);
     }
     *abort_flag = 0;
@@ -273,13 +275,17 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   } else {
     // ---------------- softmax warpgroups ----------------
     const int wg = warp >> 2, wl = warp & 3;
-    const int row = wl * 32 + lane;  // query row within the chunk
+    const int row = wl * 32 + lane;  // query row within the chunk; token row for ||v||^2
     const bool valid_row = row < a.nqc;
     const int Prow = valid_row ? L - a.w + (chunk * a.nqc + row) % a.w : L - 1;
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
     const uint32_t tS = tbase + (uint32_t)(wg * 128) + lane_off;
     const uint32_t tO = tbase + 256u + (uint32_t)(wg * 128) + lane_off;
     const float c = a.c_log2;
+    const uint64_t c2 = pk2(c, c);
+    // this CTA writes ||v_j||^2 for its share of the tile rows (the query
+    // chunks of a KV head cover the same tokens and split the rows)
+    const bool nv_share = (row * a.chunks) / 128 == chunk;
     float m_ref = -INFINITY, l = 0.f;
     int n = 0;
     for (int j = wg; j < T; j += 2, ++n) {
@@ -288,18 +294,22 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       const int tile0 = (t0 + j) * kTok;
       const bool masked = tile0 + kTok - 1 > L - a.w;
-      // sweep 1: row max of this tile
-      float mx = -INFINITY;
-      for (int half = 0; half < 2; ++half) {
-        uint32_t r[64];
-        tmem_ld32x2(tS + half * 64, tS + half * 64 + 32, r);
+      float m0 = -INFINITY, m1 = -INFINITY;
+      {
+        uint32_t sr[128];
+        tmem_ld128(tS, sr);
+        if (masked) {  // only the last tiles of a sequence: hide keys past P_t
 #pragma unroll
-        for (int u = 0; u < 64; ++u) {
-          const float x = (!masked || tile0 + half * 64 + u <= Prow) ? f32(r[u]) : -INFINITY;
-          mx = fmaxf(mx, x);
+          for (int u = 0; u < 128; ++u)
+            if (tile0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
+        }
+#pragma unroll
+        for (int u = 0; u < 128; u += 4) {
+          m0 = fmax3(m0, f32(sr[u]), f32(sr[u + 1]));
+          m1 = fmax3(m1, f32(sr[u + 2]), f32(sr[u + 3]));
         }
       }
-      const float mt = mx * c;
+      const float mt = fmaxf(m0, m1) * c;
       float fac = 1.f;
       bool resc = false;
       if (mt > m_ref + 8.f) {
@@ -310,8 +320,45 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         m_ref = mt;
         l *= fac;
       }
+      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const uint64_t nmu2 = pk2(-mu, -mu);
+      uint64_t l2 = pk2(0.f, 0.f);
+      // P = exp2(S c - mu) as hi/lo bf16 planes written over the S columns
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32], hi[16], lo[16];
+        tmem_ld32(tS + cc * 32, sr);  // second read of S: keeps 32 live registers, not 128
+        if (masked) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            if (tile0 + cc * 32 + u > Prow) sr[u] = 0xFF800000u;
+        }
+#pragma unroll
+        for (int u2 = 0; u2 < 16; ++u2) {
+          const int u = 2 * u2;
+          float y0, y1;
+          upk2(ffma2(pk2(f32(sr[u]), f32(sr[u + 1])), c2, nmu2), y0, y1);
+          const float e0 = ex2(y0), e1 = ex2(y1);
+          const uint64_t E = pk2(e0, e1);
+          l2 = fadd2(l2, E);
+          hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
+          const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
+          const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
+          float r0, r1;
+          upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
+          lo[u2] = pack_bf16_rn(r0, r1);
+        }
+        tmem_st16(tS + cc * 32, hi);
+        tmem_st16(tS + cc * 32 + 16, lo);
+      }
+      {
+        float la, lb;
+        upk2(l2, la, lb);
+        l += la + lb;
+      }
       if (__any_sync(0xffffffffu, resc)) {
-        // O of this warpgroup must not be in flight: wait for its previous P V
+        // the reference max moved: rescale O, once its previous P V has landed
+        // (done after writing P so that the S registers are dead here)
         if (!warp_wait(OD(wg), (n - 1) & 1)) { fail(a, abort_flag); break; }
         tc_fence_after();
         for (int cc = 0; cc < 4; ++cc) {
@@ -321,33 +368,35 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
           tmem_st32(tO + cc * 32, o);
         }
-        tmem_st_wait();
-      }
-      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // sweep 2: P = exp2(S c - mu) as hi/lo bf16 planes over the S columns
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tS + cc * 32, r);
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int u2 = 0; u2 < 16; ++u2) {
-          const int u = 2 * u2;
-          const int tok = tile0 + cc * 32 + u;
-          const float x0 = (!masked || tok <= Prow) ? f32(r[u]) : -INFINITY;
-          const float x1 = (!masked || tok + 1 <= Prow) ? f32(r[u + 1]) : -INFINITY;
-          const float e0 = ex2(fmaf(x0, c, -mu));
-          const float e1 = ex2(fmaf(x1, c, -mu));
-          l += e0 + e1;
-          const uint32_t h0 = u32(e0) & 0xFFFF0000u, h1 = u32(e1) & 0xFFFF0000u;
-          hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);
-          lo[u2] = pack_bf16_rn(e0 - f32(h0), e1 - f32(h1));
-        }
-        tmem_st16(tS + cc * 32, hi);
-        tmem_st16(tS + cc * 32 + 16, lo);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(PF(wg));
+      // side job while the tensor core runs P V: ||v||^2 of this tile's rows
+      if (!warp_wait(VF(wg), n & 1)) { fail(a, abort_flag); break; }
+      if (nv_share) {
+        const uint8_t* vrow = sV + wg * kTileBytes + row * 128;
+        uint64_t acc2 = pk2(0.f, 0.f);
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 q4 =
+                *reinterpret_cast<const uint4*>(vrow + bx * kBox + ((i ^ (row & 7)) * 16));
+            const uint32_t wv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t pr = pk2(f32(wv[k] << 16), f32(wv[k] & 0xFFFF0000u));
+              acc2 = ffma2(pr, pr, acc2);
+            }
+          }
+        float na, nb;
+        upk2(acc2, na, nb);
+        const int tok = tile0 + row;
+        if (tok < L) a.nvbuf[(size_t)z * a.n_max + tok] = na + nb;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(VE(wg));
     }
     // partial (m, l, O) of this warpgroup for its row
     float* out = a.partial + (((size_t)blockIdx.x * 2 + wg) * 128 + row) * kPartStride;
@@ -420,11 +469,13 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
   const float inv = 1.f / Lsum;
   const float A[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
   const float nA = warp_sum(A[0] * A[0] + A[1] * A[1] + A[2] * A[2] + A[3] * A[3]);
+  // pass 2 multiplies V by -2A (exact scaling) so that D = -2 A.v directly
   uint32_t hw[2], lw[2];
   for (int i = 0; i < 2; ++i) {
-    const __nv_bfloat162 hv = __floats2bfloat162_rn(A[2 * i], A[2 * i + 1]);
+    const float x0 = -2.f * A[2 * i], x1 = -2.f * A[2 * i + 1];
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(x0, x1);
     const float h0 = __bfloat162float(hv.x), h1 = __bfloat162float(hv.y);
-    const __nv_bfloat162 lv = __floats2bfloat162_rn(A[2 * i] - h0, A[2 * i + 1] - h1);
+    const __nv_bfloat162 lv = __floats2bfloat162_rn(x0 - h0, x1 - h1);
     hw[i] = *reinterpret_cast<const uint32_t*>(&hv);
     lw[i] = *reinterpret_cast<const uint32_t*>(&lv);
   }
@@ -465,34 +516,58 @@ __device__ __noinline__ float direct_sqdist(const float* A, const __nv_bfloat16*
   return s;
 }
 
-template <bool kMasked>
-__device__ __forceinline__ void score_cols(const uint32_t* xs, const uint32_t* ds, int ncol,
-                                           int col0, const float4* qc, const int* pcol, int tok,
-                                           float c, float nv, float& acc, int& sing,
-                                           const float* arows, const __nv_bfloat16* vrow) {
+// Fast path for 16 query columns of one token (no dominant token, no
+// possible cancellation, every key visible): packed fp32 pairs,
+//   p = 2^(x c - M'),  M' = M + log2 L,   ratio = p + p^2 + p^3,
+//   s += ratio^2 (D' + ||A||^2 + ||v||^2)   with D' = -2 A.v from the MMA.
+// kf holds (-M'_t, -M'_t+1, ||A_t||^2, ||A_t+1||^2) per column pair.
+__device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf, uint64_t c2,
+                                       uint64_t nv2, uint64_t& acc2, float& pmax) {
 #pragma unroll
-  for (int u = 0; u < ncol; ++u) {
-    const int col = col0 + u;
-    const float4 k = qc[col];  // (M, 1/L, L, ||A||^2), broadcast
-    const float e = ex2(fmaf(f32(xs[u]), c, -k.x));
-    const float p = e * k.y;
-    float ratio = fmaf(p, fmaf(p, p, p), p);  // p + p^2 + p^3 = p / (1 - p) for p < 2^-8
-    const bool vis = !kMasked || tok <= pcol[col];
-    const float base = k.w + nv;
-    float zt = fmaf(-2.f, f32(ds[u]), base);  // ||A||^2 + ||v||^2 - 2 A.v
-    const bool big = p >= 0.00390625f;
-    const bool cancel = zt < 0.03125f * base;
-    if (vis && (big || cancel)) {  // rare: dominant tokens only
-      if (big) {
-        const float den = k.z - e;  // (1 - p) L
-        if (!(den > 0.f)) sing = 1;
-        ratio = __fdiv_rn(e, den);
-      }
-      if (cancel) zt = direct_sqdist(arows + (size_t)col * kHd, vrow);
-    }
-    const float contrib = ratio * ratio * zt;
-    if (vis) acc += contrib;
+  for (int i = 0; i < 8; ++i) {
+    const float4 k = kf[i];
+    float y0, y1;
+    upk2(ffma2(pk2(f32(r[2 * i]), f32(r[2 * i + 1])), c2, pk2(k.x, k.y)), y0, y1);
+    const float p0 = ex2(y0), p1 = ex2(y1);
+    pmax = fmax3(pmax, p0, p1);
+    const uint64_t P = pk2(p0, p1);
+    const uint64_t ratio = ffma2(P, ffma2(P, P, P), P);
+    const uint64_t zt = fadd2(fadd2(pk2(f32(r[16 + 2 * i]), f32(r[16 + 2 * i + 1])),
+                                    pk2(k.z, k.w)), nv2);
+    acc2 = ffma2(fmul2(ratio, ratio), zt, acc2);
   }
+}
+
+// Careful path for 16 query columns of one token, re-read from TMEM: the
+// causal mask, ratio = e / (L - e) with the singular check when p >= 2^-8, and
+// the direct squared distance where the expansion cancels by more than 32x.
+// Warp-uniform call (the TMEM loads are warp-collective).
+__device__ __noinline__ float careful16(uint32_t tS, uint32_t tD, int col0, int tok, bool masked,
+                                        int L, int w, int crow0, const float4* qstat_rows,
+                                        float c, float nv, const float* arows,
+                                        const __nv_bfloat16* vrow, int* sing) {
+  uint32_t r[32];
+  tmem_ld16x2(tS + col0, tD + col0, r);
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int col = col0 + u;
+    const float4 k = qstat_rows[col];  // (M, 1/L, L, ||A||^2)
+    const bool vis = !masked || tok <= L - w + (crow0 + col) % w;
+    const float e = ex2(fmaf(f32(r[u]), c, -k.x));
+    const float p = e * k.y;
+    float ratio = fmaf(p, fmaf(p, p, p), p);
+    const float base = k.w + nv;
+    float zt = base + f32(r[16 + u]);
+    if (vis && p >= 0.00390625f) {
+      const float den = k.z - e;  // (1 - p) L
+      if (!(den > 0.f)) *sing = 1;
+      ratio = __fdiv_rn(e, den);
+    }
+    if (vis && zt < 0.03125f * base) zt = direct_sqdist(arows + (size_t)col * kHd, vrow);
+    if (vis) acc += ratio * ratio * zt;
+  }
+  return acc;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -506,9 +581,9 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   uint8_t* sQ = smem + 4 * kTileBytes;       // nqc rows x 2 boxes
   uint8_t* sAh = sQ + nqc * 256;
   uint8_t* sAl = sAh + nqc * 256;
-  float4* qc = reinterpret_cast<float4*>(sAl + nqc * 256);
-  int* pcol = reinterpret_cast<int*>(qc + nqc);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(pcol + nqc);  // 13 barriers
+  float4* kf = reinterpret_cast<float4*>(sAl + nqc * 256);   // [nqc/2] fast-path constants
+  float* nAmax = reinterpret_cast<float*>(kf + nqc / 2);      // [nqc/16] max ||A||^2 per chunk
+  uint64_t* bars = reinterpret_cast<uint64_t*>(nAmax + 8);    // 13 barriers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -531,8 +606,7 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1);
-      mbar_init(VE(s), 1 + 4);  // MMA commit + the 4 warps that read ||v||^2
+      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1); mbar_init(VE(s), 1);
       mbar_init(MD(s), 1); mbar_init(TF(s), 4);
     }
     *abort_flag = 0;
@@ -540,14 +614,21 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   }
   if (threadIdx.x < nqc) {
     const int i = threadIdx.x;
-    qc[i] = a.qstat[qrow0 + i];
-    pcol[i] = L - a.w + (chunk * nqc + i) % a.w;
+    const float4 q = a.qstat[qrow0 + i];  // (M, 1/L, L, ||A||^2)
+    float* kff = reinterpret_cast<float*>(kf);
+    kff[(i >> 1) * 4 + (i & 1)] = -(q.x + log2f(q.z));  // -M' folds 1/L into the exponent
+    kff[(i >> 1) * 4 + 2 + (i & 1)] = q.w;
   }
+  if (threadIdx.x < 8) nAmax[threadIdx.x] = 0.f;
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
     tc_fence_before();
   }
+  __syncthreads();
+  if (threadIdx.x < nqc)  // ||A||^2 >= 0, so the float bits order like ints
+    atomicMax(reinterpret_cast<int*>(nAmax) + threadIdx.x / 16,
+              __float_as_int(a.qstat[qrow0 + threadIdx.x].w));
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
@@ -615,62 +696,52 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
     const uint32_t tS = tbase + (uint32_t)(wg * 256) + lane_off, tD = tS + 128u;
     const float c = a.c_log2;
+    const uint64_t c2 = pk2(c, c);
+    const int nch = nqc / 16;
+    const float4* qrows = a.qstat + qrow0;
+    const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
     int sing = 0;
     int n = 0;
     for (int j = wg; j < T; j += 2, ++n) {
       const int ph = n & 1;
       const int tile0 = (t0 + j) * kTok;
       const int tok = tile0 + row;
-      // ||v_j||^2 from the staged V tile (the order of the squares does not
-      // matter, so the 128-byte swizzle only chooses a conflict-free order)
-      if (!warp_wait(VF(wg), ph)) { fail(a, abort_flag); break; }
-      const uint8_t* vrow = sV + wg * kTileBytes + row * 128;
-      float nv = 0.f;
-#pragma unroll
-      for (int bx = 0; bx < 2; ++bx)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 q4 = *reinterpret_cast<const uint4*>(vrow + bx * kBox + ((i ^ (row & 7)) * 16));
-          const uint32_t wv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float lo = __uint_as_float(wv[k] << 16), hi = __uint_as_float(wv[k] & 0xFFFF0000u);
-            nv = fmaf(lo, lo, nv);
-            nv = fmaf(hi, hi, nv);
-          }
-        }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(VE(wg));
+      const bool valid = tok < L;
+      const float nv = valid ? a.nvbuf[(size_t)z * a.n_max + tok] : 0.f;  // from pass 1
+      const __nv_bfloat16* vrow_g = a.v + ((size_t)z * a.n_max + (valid ? tok : 0)) * kHd;
       if (!warp_wait(MD(wg), ph)) { fail(a, abort_flag); break; }
       if (warp_aborted(abort_flag)) break;
       tc_fence_after();
       const bool masked = tile0 + kTok - 1 > L - a.w;
-      const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
-      const __nv_bfloat16* vrow_g = a.v + ((size_t)z * a.n_max + (tok < L ? tok : 0)) * kHd;
       float acc = 0.f;
-      int col = 0;
-      for (; col + 32 <= nqc; col += 32) {
-        uint32_t xs[32], ds[32];
-        tmem_ld32(tS + col, xs);
-        tmem_ld32(tD + col, ds);
-        if (masked)
-          score_cols<true>(xs, ds, 32, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
-        else
-          score_cols<false>(xs, ds, 32, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
-      }
-      if (col < nqc) {  // nqc % 32 == 16
-        uint32_t xs[16], ds[16];
-        tmem_ld16(tS + col, xs);
-        tmem_ld16(tD + col, ds);
-        if (masked)
-          score_cols<true>(xs, ds, 16, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
-        else
-          score_cols<false>(xs, ds, 16, col, qc, pcol, tok, c, nv, acc, sing, arows, vrow_g);
+      if (masked) {
+        for (int ch = 0; ch < nch; ++ch)
+          acc += careful16(tS, tD, ch * 16, tok, true, L, a.w, chunk * nqc, qrows, c, nv, arows,
+                           vrow_g, &sing);
+      } else {
+        const uint64_t nv2 = pk2(nv, nv);
+        for (int ch = 0; ch < nch; ++ch) {
+          uint32_t r[32];
+          tmem_ld16x2(tS + ch * 16, tD + ch * 16, r);
+          uint64_t a2 = pk2(0.f, 0.f);
+          float pmax = 0.f;
+          fast16(r, kf + ch * 8, c2, nv2, a2, pmax);
+          // dominant token (p >= 2^-8) or possible cancellation (||A||^2 >= 0.6 ||v||^2)
+          const bool redo = pmax >= 0.00390625f || nAmax[ch] >= 0.6f * nv;
+          if (__any_sync(0xffffffffu, redo)) {
+            acc += careful16(tS, tD, ch * 16, tok, false, L, a.w, chunk * nqc, qrows, c, nv,
+                             arows, vrow_g, &sing);
+          } else {
+            float x0, x1;
+            upk2(a2, x0, x1);
+            acc += x0 + x1;
+          }
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(TF(wg));
-      if (tok < L) a.parts[(size_t)chunk * a.part_stride + (size_t)z * a.n_max + tok] = acc;
+      if (valid) a.parts[(size_t)chunk * a.part_stride + (size_t)z * a.n_max + tok] = acc;
     }
     if (sing) atomicMax(a.status, (int)DROPKV_ERR_SINGULAR);
   }
@@ -724,8 +795,7 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
 
 size_t pass1_smem() { return 5 * (size_t)kTileBytes + 16 * 8 + 64; }
 size_t pass2_smem(int nqc) {
-  return 4 * (size_t)kTileBytes + 3 * (size_t)nqc * 256 + (size_t)nqc * 16 + (size_t)nqc * 4 +
-         13 * 8 + 8;
+  return 4 * (size_t)kTileBytes + 3 * (size_t)nqc * 256 + (size_t)nqc / 2 * 16 + 8 * 4 + 13 * 8 + 8;
 }
 
 int num_sms() {
@@ -800,6 +870,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   a.part_stride = (size_t)lens.B * s.Hkv * s.n_max;
   a.attn_f32 = reinterpret_cast<float*>(ws + lay.attn);
   a.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  a.nvbuf = reinterpret_cast<float*>(ws + lay.tc_nv);
 
   const uint64_t rows = (uint64_t)lens.B * s.Hq * s.window;
   a.qbox_rows = (int32_t)std::min<uint64_t>(128, rows);
