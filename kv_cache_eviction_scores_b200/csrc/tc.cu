@@ -140,6 +140,87 @@ __device__ __forceinline__ uint64_t vmn_desc(uint32_t base, int kk) {
 }
 
 // =========================== pass 1 =========================================
+// Read-only sweep over a query row of S (pass 1): the row's max of S c over
+// the visible keys.  Warp-collective.
+__device__ __forceinline__ float p1_tile_max(uint32_t tS, int tile0, bool masked, int Prow,
+                                             float c) {
+  uint32_t sr[128];
+  tmem_ld128(tS, sr);  // one 128-column load: fewer, larger TMEM transfers are faster
+  if (masked) {        // only the last tiles of a sequence: hide keys past P_t
+#pragma unroll
+    for (int u = 0; u < 128; ++u)
+      if (tile0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
+  }
+  float ya = -INFINITY, yb = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < 128; u += 4) {
+    ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
+    yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
+  }
+  return fmaxf(ya, yb) * c;  // c > 0, so the max commutes with the scaling
+}
+
+// Writing sweep over a query row of S (pass 1): P = exp2(S c - mu) as hi/lo
+// bf16 planes written over the S columns (tokens 16k..16k+15 keep hi in columns
+// [16k, 16k+8) and lo in [16k+8, 16k+16), inside the columns already read);
+// returns the row's sum of P.  Warp-collective.
+__device__ __forceinline__ float p1_tile_pass(uint32_t tS, int tile0, bool masked, int Prow,
+                                              uint64_t c2, float mu) {
+  const uint64_t nmu2 = pk2(-mu, -mu);
+  uint64_t l2 = pk2(0.f, 0.f);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {  // 32 tokens per load
+    uint32_t sr[32];
+    tmem_ld32(tS + cc * 32, sr);
+    if (masked) {
+#pragma unroll
+      for (int u = 0; u < 32; ++u)
+        if (tile0 + cc * 32 + u > Prow) sr[u] = 0xFF800000u;
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {  // 16 tokens -> 8 hi + 8 lo columns
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int u2 = 0; u2 < 8; ++u2) {
+        const int u = half * 16 + 2 * u2;
+        float d0, d1;
+        upk2(ffma2(pk2(f32(sr[u]), f32(sr[u + 1])), c2, nmu2), d0, d1);
+        const float e0 = ex2(d0), e1 = ex2(d1);
+        const uint64_t E = pk2(e0, e1);
+        l2 = fadd2(l2, E);
+        hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
+        const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
+        const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
+        float r0, r1;
+        upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
+        lo[u2] = pack_bf16_rn(r0, r1);
+      }
+      tmem_st8(tS + cc * 32 + half * 16, hi);
+      tmem_st8(tS + cc * 32 + half * 16 + 8, lo);
+    }
+  }
+  float la, lb;
+  upk2(l2, la, lb);
+  return la + lb;
+}
+
+// Rare path of pass 1, out of line: the reference max moved for some lanes
+// (factor fac <= 1 for them, 1 for the others), so this warpgroup's O is
+// rescaled once its previous P V has landed.  Warp-collective; nothing is in
+// flight on entry.  Returns false on a timeout.
+__device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, int n, uint32_t od_bar) {
+  if (!warp_wait(od_bar, (n - 1) & 1)) return false;
+  tc_fence_after();
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t o[32];
+    tmem_ld32(tO + cc * 32, o);
+#pragma unroll
+    for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
+    tmem_st32(tO + cc * 32, o);
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
@@ -255,12 +336,12 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t vbase = smem_u32(vb);
         const uint32_t dO = tbase + 256u + (uint32_t)(s * 128);
         const uint32_t pS = tbase + (uint32_t)(s * 128);
+        // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16)
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dO, pS + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)), vmn_desc(vbase, kk), IDP,
+          mma_ts(dO, pS + (uint32_t)(16 * kk), vmn_desc(vbase, kk), IDP,
                  (i >= 2 || kk > 0) ? 1u : 0u);
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dO, pS + (uint32_t)(32 * (kk >> 1) + 16 + 8 * (kk & 1)), vmn_desc(vbase, kk), IDP,
-                 1u);
+          mma_ts(dO, pS + (uint32_t)(16 * kk + 8), vmn_desc(vbase, kk), IDP, 1u);
         mma_commit(VE(s));
         mma_commit(OD(s));
       }
@@ -294,81 +375,23 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       const int tile0 = (t0 + j) * kTok;
       const bool masked = tile0 + kTok - 1 > L - a.w;
-      float m0 = -INFINITY, m1 = -INFINITY;
-      {
-        uint32_t sr[128];
-        tmem_ld128(tS, sr);
-        if (masked) {  // only the last tiles of a sequence: hide keys past P_t
-#pragma unroll
-          for (int u = 0; u < 128; ++u)
-            if (tile0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
-        }
-#pragma unroll
-        for (int u = 0; u < 128; u += 4) {
-          m0 = fmax3(m0, f32(sr[u]), f32(sr[u + 1]));
-          m1 = fmax3(m1, f32(sr[u + 2]), f32(sr[u + 3]));
-        }
-      }
-      const float mt = fmaxf(m0, m1) * c;
+      // the reference max moves only when a tile exceeds it by more than 8
+      // (so 2^(S c - m) <= 256); then l and this warpgroup's O are rescaled
+      const float mt = p1_tile_max(tS, tile0, masked, Prow, c);
       float fac = 1.f;
       bool resc = false;
       if (mt > m_ref + 8.f) {
-        if (m_ref != -INFINITY) {
-          fac = ex2(m_ref - mt);
-          resc = (n > 0);
-        }
+        if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
+        resc = m_ref != -INFINITY && n > 0;
         m_ref = mt;
         l *= fac;
       }
-      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const uint64_t nmu2 = pk2(-mu, -mu);
-      uint64_t l2 = pk2(0.f, 0.f);
-      // P = exp2(S c - mu) as hi/lo bf16 planes written over the S columns
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32], hi[16], lo[16];
-        tmem_ld32(tS + cc * 32, sr);  // second read of S: keeps 32 live registers, not 128
-        if (masked) {
-#pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (tile0 + cc * 32 + u > Prow) sr[u] = 0xFF800000u;
-        }
-#pragma unroll
-        for (int u2 = 0; u2 < 16; ++u2) {
-          const int u = 2 * u2;
-          float y0, y1;
-          upk2(ffma2(pk2(f32(sr[u]), f32(sr[u + 1])), c2, nmu2), y0, y1);
-          const float e0 = ex2(y0), e1 = ex2(y1);
-          const uint64_t E = pk2(e0, e1);
-          l2 = fadd2(l2, E);
-          hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
-          const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
-          const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
-          float r0, r1;
-          upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
-          lo[u2] = pack_bf16_rn(r0, r1);
-        }
-        tmem_st16(tS + cc * 32, hi);
-        tmem_st16(tS + cc * 32 + 16, lo);
+      // warp-uniform: every lane votes, and all or none call the rescale
+      if (__any_sync(0xffffffffu, resc) && !p1_rescale_o(tO, fac, n, OD(wg))) {
+        fail(a, abort_flag);
+        break;
       }
-      {
-        float la, lb;
-        upk2(l2, la, lb);
-        l += la + lb;
-      }
-      if (__any_sync(0xffffffffu, resc)) {
-        // the reference max moved: rescale O, once its previous P V has landed
-        // (done after writing P so that the S registers are dead here)
-        if (!warp_wait(OD(wg), (n - 1) & 1)) { fail(a, abort_flag); break; }
-        tc_fence_after();
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
-          tmem_st32(tO + cc * 32, o);
-        }
-      }
+      l += p1_tile_pass(tS, tile0, masked, Prow, c2, m_ref == -INFINITY ? 0.f : m_ref);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(PF(wg));
@@ -720,21 +743,40 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                            vrow_g, &sing);
       } else {
         const uint64_t nv2 = pk2(nv, nv);
-        for (int ch = 0; ch < nch; ++ch) {
-          uint32_t r[32];
-          tmem_ld16x2(tS + ch * 16, tD + ch * 16, r);
-          uint64_t a2 = pk2(0.f, 0.f);
-          float pmax = 0.f;
-          fast16(r, kf + ch * 8, c2, nv2, a2, pmax);
-          // dominant token (p >= 2^-8) or possible cancellation (||A||^2 >= 0.6 ||v||^2)
-          const bool redo = pmax >= 0.00390625f || nAmax[ch] >= 0.6f * nv;
-          if (__any_sync(0xffffffffu, redo)) {
-            acc += careful16(tS, tD, ch * 16, tok, false, L, a.w, chunk * nqc, qrows, c, nv,
-                             arows, vrow_g, &sing);
+        for (int ch = 0; ch < nch; ch += 2) {
+          // 32 columns of S^T and D in one TMEM round trip when available
+          const bool two = ch + 1 < nch;
+          uint32_t r0[32], r1[32];
+          if (two) {
+            uint32_t rr[64];
+            tmem_ld32x2(tS + ch * 16, tD + ch * 16, rr);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              r0[u] = rr[u];            // S^T columns ch*16 .. +15
+              r0[16 + u] = rr[32 + u];  // D columns ch*16 .. +15
+              r1[u] = rr[16 + u];
+              r1[16 + u] = rr[48 + u];
+            }
           } else {
-            float x0, x1;
-            upk2(a2, x0, x1);
-            acc += x0 + x1;
+            tmem_ld16x2(tS + ch * 16, tD + ch * 16, r0);
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            if (k == 1 && !two) break;
+            const int cw = ch + k;
+            uint64_t a2 = pk2(0.f, 0.f);
+            float pmax = 0.f;
+            fast16(k ? r1 : r0, kf + cw * 8, c2, nv2, a2, pmax);
+            // dominant token (p >= 2^-8) or possible cancellation (||A||^2 >= 0.6 ||v||^2)
+            const bool redo = pmax >= 0.00390625f || nAmax[cw] >= 0.6f * nv;
+            if (__any_sync(0xffffffffu, redo)) {
+              acc += careful16(tS, tD, cw * 16, tok, false, L, a.w, chunk * nqc, qrows, c, nv,
+                               arows, vrow_g, &sing);
+            } else {
+              float x0, x1;
+              upk2(a2, x0, x1);
+              acc += x0 + x1;
+            }
           }
         }
       }
