@@ -86,7 +86,7 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   ScoresLayout l;
   const size_t rows = (size_t)Bs * s.Hq * s.window;
   const bool tc = tc_shape_ok(s);
-  l.nparts = tc ? tc_plan(s).chunks : 1;
+  l.nparts = tc ? 2 * tc_plan(s).chunks : 1;  // tensor path: two column halves per chunk
   size_t o = 0;
   l.status = o;
   o += kAlign;
@@ -96,14 +96,14 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   o = align_up(o + rows * s.d * sizeof(double), kAlign);
   l.parts = o;
   o = align_up(o + (size_t)l.nparts * Bs * s.Hkv * (size_t)s.n_max * sizeof(float), kAlign);
-  l.tc_partial = l.tc_ahi = l.tc_alo = l.tc_qstat = l.tc_nv = o;
+  l.tc_partial = l.tc_ahi = l.tc_alo = l.tc_qstat = l.tc_nv = l.tc_tmin = o;
   if (tc) {
     const TcPlan p = tc_plan(s);
     // pass-1 partials: at most (split target + one per (b, h, chunk)) CTAs,
     // two warpgroups each, 128 rows of (a[128], max, normaliser, pad).
     const size_t ctas = (size_t)tc_split_target() + (size_t)Bs * s.Hkv * p.chunks;
     l.tc_partial = o;
-    o = align_up(o + ctas * 2 * 128 * 132 * sizeof(float), kAlign);
+    o = align_up(o + ctas * 128 * 132 * sizeof(float), kAlign);
     l.tc_ahi = o;
     o = align_up(o + rows * s.d * 2, kAlign);
     l.tc_alo = o;
@@ -112,6 +112,9 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
     o = align_up(o + rows * 4 * sizeof(float), kAlign);
     l.tc_nv = o;
     o = align_up(o + (size_t)Bs * s.Hkv * (size_t)s.n_max * sizeof(float), kAlign);
+    l.tc_tmin = o;
+    o = align_up(o + (size_t)Bs * s.Hkv * (size_t)((s.n_max + 127) / 128) * p.chunks * sizeof(float),
+                 kAlign);
   }
   l.total = o;
   return l;

@@ -61,10 +61,14 @@ constexpr int kTok = 128;          // tokens per tile
 constexpr int kHd = 128;           // head dim
 constexpr int kBox = 128 * 128;    // bytes of a 128-row x 64-col bf16 box (SW128)
 constexpr int kTileBytes = 2 * kBox;
-constexpr int kThreads = 320;
+constexpr int kThreads = 320;      // pass 2: 8 softmax/score warps, TMA warp, MMA warp
+constexpr int kThreads1 = 352;     // pass 1: the same plus the ||v||^2 warp
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr int kPartStride = 132;   // floats per partial row: O[128], m, l, pad
+constexpr int kPartStride = 132;   // floats per partial row: O[128], m, l (2 halves), pad
 constexpr int kMaxCtas = 160;      // split target ceiling (one CTA per SM)
+constexpr int kSt1 = 3;            // pass-1 K and V stages (HBM latency needs > 1 tile in flight)
+constexpr int kRing2 = 5;          // pass-2 ring of 32 KB K/V slots (the last one doubles as A_lo)
+constexpr float kLoSkip = 8e-4f;   // pass 2 drops A_lo when ||A||^2 <= kLoSkip ||v||^2 throughout
 
 struct TcArgs {
   int32_t B, Hq, Hkv, n_max, w, G, nqc, chunks;
@@ -73,7 +77,7 @@ struct TcArgs {
   int32_t splits[kMaxB];
   int32_t cta_base[kMaxB + 1];
   float c_log2;          // log2(e) / sqrt(d)
-  float* partial;        // [ctas][2][128][kPartStride]
+  float* partial;        // [ctas][128][kPartStride]
   int32_t* status;
   __nv_bfloat16* ahi;    // [rows][128]
   __nv_bfloat16* alo;    // [rows][128]
@@ -84,7 +88,9 @@ struct TcArgs {
   size_t part_stride;
   float* attn_f32;       // [rows][128] fp32 window outputs a (read back by pass 2)
   const __nv_bfloat16* v;  // [B*Hkv][n_max][128] values (rare direct-distance path)
-  float* nvbuf;          // [B*Hkv][n_max] ||v_j||^2, written by pass 1, read by pass 2
+  float* nvbuf;          // [B*Hkv][n_max] ||v_j||^2 (pass 1 -> pass 2)
+  float* tmin;           // [B*Hkv][ntmax][chunks] min ||v_j||^2 over a chunk's share of a tile
+  int32_t ntmax;         // ceil(n_max / 128)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -142,18 +148,23 @@ __device__ __forceinline__ uint64_t vmn_desc(uint32_t base, int kk) {
 // =========================== pass 1 =========================================
 // Read-only sweep over a query row of S (pass 1): the row's max of S c over
 // the visible keys.  Warp-collective.
-__device__ __forceinline__ float p1_tile_max(uint32_t tS, int tile0, bool masked, int Prow,
+template <int NC>
+__device__ __forceinline__ float p1_tile_max(uint32_t tS, int tok0, bool masked, int Prow,
                                              float c) {
-  uint32_t sr[128];
-  tmem_ld128(tS, sr);  // one 128-column load: fewer, larger TMEM transfers are faster
-  if (masked) {        // only the last tiles of a sequence: hide keys past P_t
+  uint32_t sr[NC];
+  if constexpr (NC == 64) {
+    tmem_ld32x2(tS, tS + 32, sr);  // one TMEM round trip for the warp's 64 columns
+  } else {
+    tmem_ld128(tS, sr);
+  }
+  if (masked) {  // only the last tiles of a sequence: hide keys past P_t
 #pragma unroll
-    for (int u = 0; u < 128; ++u)
-      if (tile0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
+    for (int u = 0; u < NC; ++u)
+      if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
   }
   float ya = -INFINITY, yb = -INFINITY;
 #pragma unroll
-  for (int u = 0; u < 128; u += 4) {
+  for (int u = 0; u < NC; u += 4) {
     ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
     yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
   }
@@ -164,12 +175,13 @@ __device__ __forceinline__ float p1_tile_max(uint32_t tS, int tile0, bool masked
 // bf16 planes written over the S columns (tokens 16k..16k+15 keep hi in columns
 // [16k, 16k+8) and lo in [16k+8, 16k+16), inside the columns already read);
 // returns the row's sum of P.  Warp-collective.
+template <int NC>
 __device__ __forceinline__ float p1_tile_pass(uint32_t tS, int tile0, bool masked, int Prow,
                                               uint64_t c2, float mu) {
   const uint64_t nmu2 = pk2(-mu, -mu);
   uint64_t l2 = pk2(0.f, 0.f);
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {  // 32 tokens per load
+  for (int cc = 0; cc < NC / 32; ++cc) {  // 32 tokens per load
     uint32_t sr[32];
     tmem_ld32(tS + cc * 32, sr);
     if (masked) {
@@ -205,13 +217,13 @@ __device__ __forceinline__ float p1_tile_pass(uint32_t tS, int tile0, bool maske
 }
 
 // Rare path of pass 1, out of line: the reference max moved for some lanes
-// (factor fac <= 1 for them, 1 for the others), so this warpgroup's O is
-// rescaled once its previous P V has landed.  Warp-collective; nothing is in
-// flight on entry.  Returns false on a timeout.
-__device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, int n, uint32_t od_bar) {
-  if (!warp_wait(od_bar, (n - 1) & 1)) return false;
+// (factor fac <= 1 for them, 1 for the others), so this warp's 64 columns of O
+// are rescaled once the previous P V (the `prev`-th) has landed.
+// Warp-collective.  Returns false on a timeout.
+__device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, int prev, uint32_t od_bar) {
+  if (!warp_wait(od_bar, prev & 1)) return false;
   tc_fence_after();
-  for (int cc = 0; cc < 4; ++cc) {
+  for (int cc = 0; cc < 2; ++cc) {
     uint32_t o[32];
     tmem_ld32(tO + cc * 32, o);
 #pragma unroll
@@ -221,16 +233,17 @@ __device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, int n, uint32_
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads1, 1)
 k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTileBytes;        // 2 stages
-  uint8_t* sV = smem + 3 * kTileBytes;    // 2 stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * kTileBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint8_t* sK = smem + kTileBytes;                // kSt1 stages
+  uint8_t* sV = smem + (1 + kSt1) * kTileBytes;   // kSt1 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (1 + 2 * kSt1) * kTileBytes);  // 19 barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xmax = reinterpret_cast<float*>(tmem_slot + 2);  // [2 tile parities][2 halves][128]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1 KB alignment
     if (threadIdx.x == 0) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
@@ -241,19 +254,23 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int T = t1 - t0;
   const int L = a.L[b];
   const uint32_t BQ = smem_u32(&bars[0]);
-  auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto KE = [&](int s) { return smem_u32(&bars[3 + s]); };
-  auto VF = [&](int s) { return smem_u32(&bars[5 + s]); };
-  auto VE = [&](int s) { return smem_u32(&bars[7 + s]); };
-  auto SF = [&](int s) { return smem_u32(&bars[9 + s]); };
-  auto PF = [&](int s) { return smem_u32(&bars[11 + s]); };
-  auto OD = [&](int s) { return smem_u32(&bars[13 + s]); };
+  auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };   // kSt1 each: K full / empty,
+  auto KE = [&](int s) { return smem_u32(&bars[4 + s]); };   // V full / empty
+  auto VF = [&](int s) { return smem_u32(&bars[7 + s]); };
+  auto VE = [&](int s) { return smem_u32(&bars[10 + s]); };
+  auto SF = [&](int b) { return smem_u32(&bars[13 + b]); };  // 2 TMEM buffers: S ready,
+  auto PF = [&](int b) { return smem_u32(&bars[15 + b]); };  // P written,
+  auto XB = [&](int b) { return smem_u32(&bars[17 + b]); };  // tile-max exchange
+  const uint32_t OD = smem_u32(&bars[19]);                     // P V into O done
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
-    for (int s = 0; s < 2; ++s) {
+    mbar_init(OD, 1);
+    for (int s = 0; s < kSt1; ++s) {
       mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1);
-      mbar_init(VE(s), 1 + 4);  // P V commit + the 4 warps that read ||v||^2 from the tile
-      mbar_init(SF(s), 1); mbar_init(PF(s), 128); mbar_init(OD(s), 1);
+      mbar_init(VE(s), 2);  // P V commit + the ||v||^2 warp's reads
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(SF(b), 1); mbar_init(PF(b), 256); mbar_init(XB(b), 8);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -277,7 +294,7 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
       tma_load_2d(smem_u32(sQ) + kBox, &tmQ, BQ, 64, qrow0);
       auto load = [&](uint8_t* buf, uint32_t full, uint32_t empty, const CUtensorMap* m, int i) {
-        const int s = i & 1, ph = (i >> 1) & 1;
+        const int s = i % kSt1, ph = (i / kSt1) & 1;
         if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); return false; }
         mbar_expect_tx(full, kTileBytes);
         const uint32_t dst = smem_u32(buf + s * kTileBytes);
@@ -287,8 +304,8 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       };
       bool ok = T > 0 ? load(sK, KF(0), KE(0), &tmK, 0) : true;
       for (int j = 0; j < T && ok && !*abort_flag; ++j) {
-        if (j + 1 < T) ok = load(sK, KF((j + 1) & 1), KE((j + 1) & 1), &tmK, j + 1);
-        if (ok) ok = load(sV, VF(j & 1), VE(j & 1), &tmV, j);
+        if (j + 1 < T) ok = load(sK, KF((j + 1) % kSt1), KE((j + 1) % kSt1), &tmK, j + 1);
+        if (ok) ok = load(sV, VF(j % kSt1), VE(j % kSt1), &tmV, j);
       }
     }
   } else if (warp == 9) {
@@ -299,23 +316,23 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (!ok) fail(a, abort_flag);
     const uint32_t qbase = smem_u32(sQ);
     auto issue_S = [&](int i) {
-      const int s = i & 1, ph = (i >> 1) & 1;
+      const int s = i % kSt1, ph = (i / kSt1) & 1, bf = i & 1;
       if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t kb = smem_u32(sK + s * kTileBytes);
-        const uint32_t dS = tbase + (uint32_t)(s * 128);
+        const uint32_t dS = tbase + (uint32_t)(bf * 128);
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(dS, kmajor_desc(qbase, 128, kk), kmajor_desc(kb, 128, kk), IDS, kk > 0);
         mma_commit(KE(s));
-        mma_commit(SF(s));
+        mma_commit(SF(bf));
       }
       __syncwarp();
       return true;
     };
     auto issue_PV = [&](int i) {
-      const int s = i & 1, ph = (i >> 1) & 1;
-      if (!warp_wait(PF(s), ph)) { fail(a, abort_flag); return false; }
+      const int s = i % kSt1, ph = (i / kSt1) & 1, bf = i & 1, bph = (i >> 1) & 1;
+      if (!warp_wait(PF(bf), bph)) { fail(a, abort_flag); return false; }
       if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
       uint8_t* vb = sV + s * kTileBytes;
       const int tile0 = (t0 + i) * kTok;
@@ -334,16 +351,16 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       if (lane == 0) {
         const uint32_t vbase = smem_u32(vb);
-        const uint32_t dO = tbase + 256u + (uint32_t)(s * 128);
-        const uint32_t pS = tbase + (uint32_t)(s * 128);
+        const uint32_t dO = tbase + 256u;  // one O: both halves of every tile feed it
+        const uint32_t pS = tbase + (uint32_t)(bf * 128);
         // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16)
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(dO, pS + (uint32_t)(16 * kk), vmn_desc(vbase, kk), IDP,
-                 (i >= 2 || kk > 0) ? 1u : 0u);
+                 (i > 0 || kk > 0) ? 1u : 0u);
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(dO, pS + (uint32_t)(16 * kk + 8), vmn_desc(vbase, kk), IDP, 1u);
         mma_commit(VE(s));
-        mma_commit(OD(s));
+        mma_commit(OD);
       }
       __syncwarp();
       return true;
@@ -353,59 +370,29 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       if (j + 1 < T) ok = issue_S(j + 1);
       if (ok) ok = issue_PV(j);
     }
-  } else {
-    // ---------------- softmax warpgroups ----------------
-    const int wg = warp >> 2, wl = warp & 3;
-    const int row = wl * 32 + lane;  // query row within the chunk; token row for ||v||^2
-    const bool valid_row = row < a.nqc;
-    const int Prow = valid_row ? L - a.w + (chunk * a.nqc + row) % a.w : L - 1;
-    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-    const uint32_t tS = tbase + (uint32_t)(wg * 128) + lane_off;
-    const uint32_t tO = tbase + 256u + (uint32_t)(wg * 128) + lane_off;
-    const float c = a.c_log2;
-    const uint64_t c2 = pk2(c, c);
-    // this CTA writes ||v_j||^2 for its share of the tile rows (the query
-    // chunks of a KV head cover the same tokens and split the rows)
-    const bool nv_share = (row * a.chunks) / 128 == chunk;
-    float m_ref = -INFINITY, l = 0.f;
-    int n = 0;
-    for (int j = wg; j < T; j += 2, ++n) {
-      if (!warp_wait(SF(wg), n & 1)) { fail(a, abort_flag); break; }
+  } else if (warp == 10) {
+    // ---------------- ||v_j||^2 ----------------
+    // This CTA's share of every V tile's rows (the query chunks of a KV head
+    // cover the same tokens and split the rows), 4 rows per lane; the order of
+    // the squares is free, so the 128-byte swizzle only picks a bank-conflict-
+    // free order.  Arrives on the V stage's empty barrier when done.
+    for (int j = 0; j < T; ++j) {
+      const int s = j % kSt1, ph = (j / kSt1) & 1;
+      if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); break; }
       if (warp_aborted(abort_flag)) break;
-      tc_fence_after();
+      const uint8_t* vb = sV + s * kTileBytes;
       const int tile0 = (t0 + j) * kTok;
-      const bool masked = tile0 + kTok - 1 > L - a.w;
-      // the reference max moves only when a tile exceeds it by more than 8
-      // (so 2^(S c - m) <= 256); then l and this warpgroup's O are rescaled
-      const float mt = p1_tile_max(tS, tile0, masked, Prow, c);
-      float fac = 1.f;
-      bool resc = false;
-      if (mt > m_ref + 8.f) {
-        if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
-        resc = m_ref != -INFINITY && n > 0;
-        m_ref = mt;
-        l *= fac;
-      }
-      // warp-uniform: every lane votes, and all or none call the rescale
-      if (__any_sync(0xffffffffu, resc) && !p1_rescale_o(tO, fac, n, OD(wg))) {
-        fail(a, abort_flag);
-        break;
-      }
-      l += p1_tile_pass(tS, tile0, masked, Prow, c2, m_ref == -INFINITY ? 0.f : m_ref);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(PF(wg));
-      // side job while the tensor core runs P V: ||v||^2 of this tile's rows
-      if (!warp_wait(VF(wg), n & 1)) { fail(a, abort_flag); break; }
-      if (nv_share) {
-        const uint8_t* vrow = sV + wg * kTileBytes + row * 128;
+      float vmin = INFINITY;
+      for (int rr = 0; rr < 4; ++rr) {
+        const int row = rr * 32 + lane;
+        if ((row * a.chunks) / 128 != chunk || tile0 + row >= L) continue;
         uint64_t acc2 = pk2(0.f, 0.f);
 #pragma unroll
         for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int q = 0; q < 8; ++q) {
             const uint4 q4 =
-                *reinterpret_cast<const uint4*>(vrow + bx * kBox + ((i ^ (row & 7)) * 16));
+                *reinterpret_cast<const uint4*>(vb + bx * kBox + row * 128 + ((q ^ (row & 7)) * 16));
             const uint32_t wv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -415,36 +402,88 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           }
         float na, nb;
         upk2(acc2, na, nb);
-        const int tok = tile0 + row;
-        if (tok < L) a.nvbuf[(size_t)z * a.n_max + tok] = na + nb;
+        a.nvbuf[(size_t)z * a.n_max + tile0 + row] = na + nb;
+        vmin = fminf(vmin, na + nb);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(VE(wg));
+      if (lane == 0) mbar_arrive(VE(s));
+      vmin = warp_min(vmin);  // pass 2 decides from it whether A needs its low part
+      if (lane == 0) a.tmin[((size_t)z * a.ntmax + t0 + j) * a.chunks + chunk] = vmin;
     }
-    // partial (m, l, O) of this warpgroup for its row
-    float* out = a.partial + (((size_t)blockIdx.x * 2 + wg) * 128 + row) * kPartStride;
-    bool have = n > 0 && !warp_aborted(abort_flag);
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    // Both warpgroups work on every tile: warpgroup wg owns the tile's tokens
+    // [64 wg, 64 wg + 64) (its S/P columns) and O's head-dim columns
+    // [64 wg, 64 wg + 64); a row's two halves exchange their tile max.
+    const int wg = warp >> 2, wl = warp & 3;
+    const int row = wl * 32 + lane;  // query row within the chunk; token row for ||v||^2
+    const bool valid_row = row < a.nqc;
+    const int Prow = valid_row ? L - a.w + (chunk * a.nqc + row) % a.w : L - 1;
+    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+    const int c0 = wg * 64;
+    const uint32_t tO = tbase + 256u + (uint32_t)c0 + lane_off;
+    const float c = a.c_log2;
+    const uint64_t c2 = pk2(c, c);
+    float m_ref = -INFINITY, l = 0.f;
+    for (int j = 0; j < T; ++j) {
+      const int s = j & 1, ph = (j >> 1) & 1;  // TMEM buffer and its phase
+      if (!warp_wait(SF(s), ph)) { fail(a, abort_flag); break; }
+      if (warp_aborted(abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tS = tbase + (uint32_t)(s * 128) + lane_off + (uint32_t)c0;
+      const int tile0 = (t0 + j) * kTok;
+      const bool masked = tile0 + c0 + 63 > L - a.w;
+      // the reference max moves only when a tile exceeds it by more than 8
+      // (so 2^(S c - m) <= 256); then l and O are rescaled
+      const float mh = p1_tile_max<64>(tS, tile0 + c0, masked, Prow, c);
+      float* xm = xmax + s * 256;
+      xm[wg * 128 + row] = mh;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(XB(s));
+      if (!warp_wait(XB(s), ph)) { fail(a, abort_flag); break; }
+      const float mt = fmaxf(mh, xm[(1 - wg) * 128 + row]);
+      float fac = 1.f;
+      bool resc = false;
+      if (mt > m_ref + 8.f) {
+        if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
+        resc = m_ref != -INFINITY && j > 0;
+        m_ref = mt;
+        l *= fac;
+      }
+      // warp-uniform: every lane votes, and all or none call the rescale
+      if (__any_sync(0xffffffffu, resc) && !p1_rescale_o(tO, fac, j - 1, OD)) {
+        fail(a, abort_flag);
+        break;
+      }
+      l += p1_tile_pass<64>(tS, tile0 + c0, masked, Prow, c2, m_ref == -INFINITY ? 0.f : m_ref);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(PF(s));
+    }
+    // partial row: O half of this warpgroup, the shared max, its normaliser half
+    float* out = a.partial + ((size_t)blockIdx.x * 128 + row) * kPartStride;
+    bool have = T > 0 && !warp_aborted(abort_flag);
     if (have) {
-      if (!warp_wait(OD(wg), (n - 1) & 1)) {
+      if (!warp_wait(OD, (T - 1) & 1)) {
         fail(a, abort_flag);
         have = false;
       }
       tc_fence_after();
     }
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int cc = 0; cc < 2; ++cc) {
       uint32_t o[32];
       if (have) tmem_ld32(tO + cc * 32, o);
       if (valid_row) {
 #pragma unroll
         for (int u = 0; u < 32; u += 4)
-          *reinterpret_cast<float4*>(out + cc * 32 + u) =
+          *reinterpret_cast<float4*>(out + c0 + cc * 32 + u) =
               have ? make_float4(f32(o[u]), f32(o[u + 1]), f32(o[u + 2]), f32(o[u + 3]))
                    : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     if (valid_row) {
-      out[128] = have ? m_ref : -INFINITY;
-      out[129] = have ? l : 0.f;
+      if (wg == 0) out[128] = have ? m_ref : -INFINITY;
+      out[129 + wg] = have ? l : 0.f;
     }
   }
   tc_fence_before();
@@ -469,10 +508,8 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
   const int gr = (hq % a.G) * a.w + t;
   const int chunk = gr / a.nqc, rr = gr % a.nqc;
   const int cta0 = a.cta_base[b] + (h * a.chunks + chunk) * a.splits[b];
-  const int np = 2 * a.splits[b];
-  auto P = [&](int i) {
-    return a.partial + (((size_t)cta0 * 2 + i) * 128 + rr) * kPartStride;
-  };
+  const int np = a.splits[b];
+  auto P = [&](int i) { return a.partial + ((size_t)(cta0 + i) * 128 + rr) * kPartStride; };
   float M = -INFINITY;
   for (int i = lane; i < np; i += 32) M = fmaxf(M, P(i)[128]);
   M = warp_max(M);
@@ -482,7 +519,7 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
     const float* p = P(i);
     const float mi = p[128];
     const float wgt = (mi == -INFINITY) ? 0.f : ex2(mi - M);
-    Lsum += wgt * p[129];
+    Lsum += wgt * (p[129] + p[130]);  // the two warpgroups' normaliser halves
     const float4 o = *reinterpret_cast<const float4*>(p + lane * 4);
     acc.x = fmaf(wgt, o.x, acc.x);
     acc.y = fmaf(wgt, o.y, acc.y);
@@ -599,15 +636,17 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int nqc = a.nqc;
-  uint8_t* sK = smem;                        // 2 stages
-  uint8_t* sV = smem + 2 * kTileBytes;       // 2 stages
-  uint8_t* sQ = smem + 4 * kTileBytes;       // nqc rows x 2 boxes
+  // A ring of kRing2 32 KB slots takes the K and V tiles in turn (K_0, V_0,
+  // K_1, ...).  When A needs its low part, the last slot holds A_lo instead and
+  // the ring runs on the first kRing2 - 1 slots.
+  uint8_t* sRing = smem;
+  uint8_t* sAl = smem + (kRing2 - 1) * kTileBytes;
+  uint8_t* sQ = smem + kRing2 * kTileBytes;  // nqc rows x 2 boxes
   uint8_t* sAh = sQ + nqc * 256;
-  uint8_t* sAl = sAh + nqc * 256;
-  float4* kf = reinterpret_cast<float4*>(sAl + nqc * 256);   // [nqc/2] fast-path constants
+  float4* kf = reinterpret_cast<float4*>(sAh + nqc * 256);   // [nqc/2] fast-path constants
   float* nAmax = reinterpret_cast<float*>(kf + nqc / 2);      // [nqc/16] max ||A||^2 per chunk
-  uint64_t* bars = reinterpret_cast<uint64_t*>(nAmax + 8);    // 13 barriers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(nAmax + 8);    // 5 + 2 kRing2 barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5 + 2 * kRing2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023u) {
@@ -619,18 +658,19 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int T = t1 - t0;
   const int L = a.L[b];
   const uint32_t BQ = smem_u32(&bars[0]);
-  auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto KE = [&](int s) { return smem_u32(&bars[3 + s]); };
-  auto VF = [&](int s) { return smem_u32(&bars[5 + s]); };
-  auto VE = [&](int s) { return smem_u32(&bars[7 + s]); };
-  auto MD = [&](int s) { return smem_u32(&bars[9 + s]); };   // MMAs of a tile done
-  auto TF = [&](int s) { return smem_u32(&bars[11 + s]); };  // TMEM buffer read out
+  auto MD = [&](int s) { return smem_u32(&bars[1 + s]); };   // MMAs of a tile done
+  auto TF = [&](int s) { return smem_u32(&bars[3 + s]); };   // TMEM buffer read out
+  auto FULL = [&](int r) { return smem_u32(&bars[5 + r]); };
+  auto EMPTY = [&](int r) { return smem_u32(&bars[5 + kRing2 + r]); };
   const int qrow0 = (b * a.Hkv + h) * a.G * a.w + chunk * nqc;
+  const int z = b * a.Hkv + h;
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1); mbar_init(VE(s), 1);
-      mbar_init(MD(s), 1); mbar_init(TF(s), 4);
+      mbar_init(MD(s), 1); mbar_init(TF(s), 8);  // both warpgroups read every tile
+    }
+    for (int r = 0; r < kRing2; ++r) {
+      mbar_init(FULL(r), 1); mbar_init(EMPTY(r), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -653,32 +693,50 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     atomicMax(reinterpret_cast<int*>(nAmax) + threadIdx.x / 16,
               __float_as_int(a.qstat[qrow0 + threadIdx.x].w));
   __syncthreads();
+  // Does A need its low part on this CTA's tiles?  Dropping A_lo leaves
+  // -2A rounded to bf16 (relative error <= 2^-8 per component), which moves
+  // -2 A.v by at most 2^-7 ||A|| ||v|| and so the squared distance
+  // ||A - v||^2 >= (||v|| - ||A||)^2 by a relative 2^-7 rho / (1 - rho)^2,
+  // rho = ||A|| / ||v||.  With ||A||^2 <= kLoSkip ||v||^2 for every query of
+  // the chunk and every token of the tiles (rho <= 0.0283) that is <= 2.4e-4.
+  bool lo;
+  {
+    float namx = 0.f;
+    for (int i = 0; i < (nqc + 15) / 16; ++i) namx = fmaxf(namx, nAmax[i]);
+    bool need = false;
+    for (int i = threadIdx.x; i < T * a.chunks; i += blockDim.x) {
+      const float tm = a.tmin[((size_t)z * a.ntmax + t0) * a.chunks + i];
+      if (!(namx <= kLoSkip * tm)) need = true;  // NaN-safe
+    }
+    lo = __syncthreads_or(need) != 0;
+  }
+  const int R = lo ? kRing2 - 1 : kRing2;  // ring slots in use
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const int z = b * a.Hkv + h;
 
   if (warp == 8) {
     if (lane == 0) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmAhi); prefetch_tmap(&tmAlo);
       prefetch_tmap(&tmK); prefetch_tmap(&tmV);
-      mbar_expect_tx(BQ, 3 * nqc * 256);
+      mbar_expect_tx(BQ, (lo ? 3 : 2) * nqc * 256);
       tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
       tma_load_2d(smem_u32(sQ) + nqc * 128, &tmQ, BQ, 64, qrow0);
       tma_load_2d(smem_u32(sAh), &tmAhi, BQ, 0, qrow0);
       tma_load_2d(smem_u32(sAh) + nqc * 128, &tmAhi, BQ, 64, qrow0);
-      tma_load_2d(smem_u32(sAl), &tmAlo, BQ, 0, qrow0);
-      tma_load_2d(smem_u32(sAl) + nqc * 128, &tmAlo, BQ, 64, qrow0);
-      for (int j = 0; j < T && !*abort_flag; ++j) {  // single thread: no warp vote needed
-        const int s = j & 1, ph = (j >> 1) & 1;
-        const uint32_t dk = smem_u32(sK + s * kTileBytes), dv = smem_u32(sV + s * kTileBytes);
-        if (!mbar_wait(KE(s), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
-        mbar_expect_tx(KF(s), kTileBytes);
-        tma_load_3d(dk, &tmK, KF(s), 0, (t0 + j) * kTok, z);
-        tma_load_3d(dk + kBox, &tmK, KF(s), 64, (t0 + j) * kTok, z);
-        if (!mbar_wait(VE(s), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
-        mbar_expect_tx(VF(s), kTileBytes);
-        tma_load_3d(dv, &tmV, VF(s), 0, (t0 + j) * kTok, z);
-        tma_load_3d(dv + kBox, &tmV, VF(s), 64, (t0 + j) * kTok, z);
+      if (lo) {
+        tma_load_2d(smem_u32(sAl), &tmAlo, BQ, 0, qrow0);
+        tma_load_2d(smem_u32(sAl) + nqc * 128, &tmAlo, BQ, 64, qrow0);
+      }
+      // single thread: no warp vote needed
+      for (int i = 0; i < 2 * T && !*abort_flag; ++i) {  // K_j at i = 2j, V_j at 2j + 1
+        const int r = i % R, ph = (i / R) & 1;
+        if (!mbar_wait(EMPTY(r), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
+        mbar_expect_tx(FULL(r), kTileBytes);
+        const uint32_t dst = smem_u32(sRing + r * kTileBytes);
+        const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
+        const int row = (t0 + (i >> 1)) * kTok;
+        tma_load_3d(dst, m, FULL(r), 0, row, z);
+        tma_load_3d(dst + kBox, m, FULL(r), 64, row, z);
       }
     }
   } else if (warp == 9) {
@@ -688,64 +746,70 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t qb = smem_u32(sQ), hb = smem_u32(sAh), lb = smem_u32(sAl);
     for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
+      const int rk = (2 * j) % R, pk = ((2 * j) / R) & 1;
+      const int rv = (2 * j + 1) % R, pv = ((2 * j + 1) / R) & 1;
       const uint32_t dS = tbase + (uint32_t)(s * 256), dD = dS + 128u;
-      if (!warp_wait(TF(s), ph ^ 1) || !warp_wait(KF(s), ph)) {
+      if (!warp_wait(TF(s), ph ^ 1) || !warp_wait(FULL(rk), pk)) {
         fail(a, abort_flag);
         break;
       }
       tc_fence_after();
-      const uint32_t kb = smem_u32(sK + s * kTileBytes), vb = smem_u32(sV + s * kTileBytes);
+      const uint32_t kb = smem_u32(sRing + rk * kTileBytes), vb = smem_u32(sRing + rv * kTileBytes);
       if (lane == 0) {
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(dS, kmajor_desc(kb, 128, kk), kmajor_desc(qb, nqc, kk), IDT, kk > 0);
-        mma_commit(KE(s));
+        mma_commit(EMPTY(rk));
       }
       __syncwarp();
-      if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); break; }
+      if (!warp_wait(FULL(rv), pv)) { fail(a, abort_flag); break; }
       tc_fence_after();
       if (lane == 0) {
         for (int kk = 0; kk < 8; ++kk)
           mma_ss(dD, kmajor_desc(vb, 128, kk), kmajor_desc(hb, nqc, kk), IDT, kk > 0);
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(dD, kmajor_desc(vb, 128, kk), kmajor_desc(lb, nqc, kk), IDT, 1u);
-        mma_commit(VE(s));
+        if (lo)
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(dD, kmajor_desc(vb, 128, kk), kmajor_desc(lb, nqc, kk), IDT, 1u);
+        mma_commit(EMPTY(rv));
         mma_commit(MD(s));
       }
       __syncwarp();
     }
   } else {
+    // Both warpgroups work on every tile: warpgroup wg owns the query columns
+    // [64 wg, min(nqc, 64 wg + 64)) and writes its own partial-score plane.
     const int wg = warp >> 2, wl = warp & 3;
     const int row = wl * 32 + lane;  // token within the tile
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-    const uint32_t tS = tbase + (uint32_t)(wg * 256) + lane_off, tD = tS + 128u;
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
-    const int nch = nqc / 16;
+    const int ch0 = wg * 4, ch1 = min(nqc / 16, ch0 + 4);  // 16-column chunks owned
     const float4* qrows = a.qstat + qrow0;
     const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
+    float* plane = a.parts + (size_t)(chunk * 2 + wg) * a.part_stride + (size_t)z * a.n_max;
     int sing = 0;
-    int n = 0;
-    for (int j = wg; j < T; j += 2, ++n) {
-      const int ph = n & 1;
+    for (int j = 0; j < T; ++j) {
+      const int s = j & 1, ph = (j >> 1) & 1;
       const int tile0 = (t0 + j) * kTok;
       const int tok = tile0 + row;
       const bool valid = tok < L;
-      const float nv = valid ? a.nvbuf[(size_t)z * a.n_max + tok] : 0.f;  // from pass 1
-      const __nv_bfloat16* vrow_g = a.v + ((size_t)z * a.n_max + (valid ? tok : 0)) * kHd;
-      if (!warp_wait(MD(wg), ph)) { fail(a, abort_flag); break; }
+      const size_t ni = (size_t)z * a.n_max + (valid ? tok : 0);
+      const float nv = valid ? a.nvbuf[ni] : 0.f;  // ||v_j||^2 from pass 1
+      const __nv_bfloat16* vrow_g = a.v + ni * kHd;
+      if (!warp_wait(MD(s), ph)) { fail(a, abort_flag); break; }
       if (warp_aborted(abort_flag)) break;
       tc_fence_after();
+      const uint32_t tS = tbase + (uint32_t)(s * 256) + lane_off, tD = tS + 128u;
       const bool masked = tile0 + kTok - 1 > L - a.w;
       float acc = 0.f;
       if (masked) {
-        for (int ch = 0; ch < nch; ++ch)
+        for (int ch = ch0; ch < ch1; ++ch)
           acc += careful16(tS, tD, ch * 16, tok, true, L, a.w, chunk * nqc, qrows, c, nv, arows,
                            vrow_g, &sing);
       } else {
         const uint64_t nv2 = pk2(nv, nv);
-        for (int ch = 0; ch < nch; ch += 2) {
+        for (int ch = ch0; ch < ch1; ch += 2) {
           // 32 columns of S^T and D in one TMEM round trip when available
-          const bool two = ch + 1 < nch;
+          const bool two = ch + 1 < ch1;
           uint32_t r0[32], r1[32];
           if (two) {
             uint32_t rr[64];
@@ -782,8 +846,8 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(TF(wg));
-      if (valid) a.parts[(size_t)chunk * a.part_stride + (size_t)z * a.n_max + tok] = acc;
+      if (lane == 0) mbar_arrive(TF(s));
+      if (valid) plane[tok] = acc;
     }
     if (sing) atomicMax(a.status, (int)DROPKV_ERR_SINGULAR);
   }
@@ -835,9 +899,12 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t pass1_smem() { return 5 * (size_t)kTileBytes + 16 * 8 + 64; }
+size_t pass1_smem() {
+  return (1 + 2 * kSt1) * (size_t)kTileBytes + 20 * 8 + 8 + 2 * 2 * 128 * 4;
+}
 size_t pass2_smem(int nqc) {
-  return 4 * (size_t)kTileBytes + 3 * (size_t)nqc * 256 + (size_t)nqc / 2 * 16 + 8 * 4 + 13 * 8 + 8;
+  return kRing2 * (size_t)kTileBytes + 2 * (size_t)nqc * 256 + (size_t)nqc / 2 * 16 + 8 * 4 +
+         (5 + 2 * kRing2) * 8 + 8;
 }
 
 int num_sms() {
@@ -913,6 +980,8 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   a.attn_f32 = reinterpret_cast<float*>(ws + lay.attn);
   a.v = reinterpret_cast<const __nv_bfloat16*>(v);
   a.nvbuf = reinterpret_cast<float*>(ws + lay.tc_nv);
+  a.tmin = reinterpret_cast<float*>(ws + lay.tc_tmin);
+  a.ntmax = (s.n_max + kTok - 1) / kTok;
 
   const uint64_t rows = (uint64_t)lens.B * s.Hq * s.window;
   a.qbox_rows = (int32_t)std::min<uint64_t>(128, rows);
@@ -932,7 +1001,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   if (e != cudaSuccess) return e;
 
   kev.begin(st);
-  k_tc_pass1<<<ctas, kThreads, sm1, st>>>(mQ1, mK, mV, a);
+  k_tc_pass1<<<ctas, kThreads1, sm1, st>>>(mQ1, mK, mV, a);
   kev.end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kev.begin(st);
