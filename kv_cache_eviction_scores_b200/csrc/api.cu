@@ -86,7 +86,7 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   ScoresLayout l;
   const size_t rows = (size_t)Bs * s.Hq * s.window;
   const bool tc = tc_shape_ok(s);
-  l.nparts = tc ? 2 * tc_plan(s).chunks : 1;  // tensor path: two column halves per chunk
+  l.nparts = tc ? 4 * tc_plan(s).chunks : 1;  // tensor path: four column groups per chunk
   size_t o = 0;
   l.status = o;
   o += kAlign;
@@ -103,7 +103,7 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
     // two warpgroups each, 128 rows of (a[128], max, normaliser, pad).
     const size_t ctas = (size_t)tc_split_target() + (size_t)Bs * s.Hkv * p.chunks;
     l.tc_partial = o;
-    o = align_up(o + ctas * 128 * 132 * sizeof(float), kAlign);
+    o = align_up(o + ctas * 128 * 136 * sizeof(float), kAlign);
     l.tc_ahi = o;
     o = align_up(o + rows * s.d * 2, kAlign);
     l.tc_alo = o;

@@ -61,10 +61,15 @@ constexpr int kTok = 128;          // tokens per tile
 constexpr int kHd = 128;           // head dim
 constexpr int kBox = 128 * 128;    // bytes of a 128-row x 64-col bf16 box (SW128)
 constexpr int kTileBytes = 2 * kBox;
-constexpr int kThreads = 320;      // pass 2: 8 softmax/score warps, TMA warp, MMA warp
-constexpr int kThreads1 = 352;     // pass 1: the same plus the ||v||^2 warp
+constexpr int kSimtWarps = 16;     // softmax / score warps: 4 per TMEM lane quarter
+constexpr int kWarpTma = kSimtWarps, kWarpMma = kSimtWarps + 1, kWarpNv = kSimtWarps + 2;
+constexpr int kThreads2 = (kSimtWarps + 2) * 32;  // pass 2: + TMA warp, MMA warp
+constexpr int kThreads1 = (kSimtWarps + 3) * 32;  // pass 1: + the ||v||^2 warp
+constexpr int kMaxRegs = 96;       // 5 warps share a sub-partition's 16K registers
+constexpr uint32_t kColO = 256;    // pass-1 TMEM columns: S/P buffers [0, 256), O, Q
+constexpr uint32_t kColQ = 384;
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr int kPartStride = 132;   // floats per partial row: O[128], m, l (2 halves), pad
+constexpr int kPartStride = 136;   // floats per partial row: O[128], m, l (4 parts), pad
 constexpr int kMaxCtas = 160;      // split target ceiling (one CTA per SM)
 constexpr int kSt1 = 3;            // pass-1 K and V stages (HBM latency needs > 1 tile in flight)
 constexpr int kRing2 = 5;          // pass-2 ring of 32 KB K/V slots (the last one doubles as A_lo)
@@ -77,6 +82,7 @@ struct TcArgs {
   int32_t splits[kMaxB];
   int32_t cta_base[kMaxB + 1];
   float c_log2;          // log2(e) / sqrt(d)
+  const __nv_bfloat16* q;  // [rows][128] window queries
   float* partial;        // [ctas][128][kPartStride]
   int32_t* status;
   __nv_bfloat16* ahi;    // [rows][128]
@@ -134,82 +140,41 @@ __device__ __forceinline__ bool warp_aborted(volatile int* f) {
   return __any_sync(0xffffffffu, *f != 0);
 }
 
-// K-major SW128 operand of `rows` rows, head dim 128 in two 64-wide boxes:
-// descriptor of the 16-wide K slice kk (0..7).
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int rows, int kk) {
-  return sdesc_sw128(base + (uint32_t)((kk >> 2) * rows * 128 + (kk & 3) * 32), 16, 1024);
+// Descriptor-word offset of the 16-wide K slice kk of a K-major SW128 operand
+// with `rows` rows (kmajor_desc's address offset >> 4).
+__device__ __forceinline__ uint32_t kslice(int kk, uint32_t rows) {
+  return (uint32_t)(kk >> 2) * rows * 8u + (uint32_t)(kk & 3) * 2u;
 }
-// V tile as the MN-major B operand of P V: N = head dim (two 64-wide boxes,
-// 16 KB apart), K = tokens (128-byte rows); slice kk covers tokens 16kk..16kk+15.
-__device__ __forceinline__ uint64_t vmn_desc(uint32_t base, int kk) {
-  return sdesc_sw128(base + (uint32_t)(kk * 16 * 128), kBox, 1024);
-}
-
 // =========================== pass 1 =========================================
-// Read-only sweep over a query row of S (pass 1): the row's max of S c over
-// the visible keys.  Warp-collective.
-template <int NC>
-__device__ __forceinline__ float p1_tile_max(uint32_t tS, int tok0, bool masked, int Prow,
-                                             float c) {
-  uint32_t sr[NC];
-  if constexpr (NC == 64) {
-    tmem_ld32x2(tS, tS + 32, sr);  // one TMEM round trip for the warp's 64 columns
-  } else {
-    tmem_ld128(tS, sr);
-  }
-  if (masked) {  // only the last tiles of a sequence: hide keys past P_t
-#pragma unroll
-    for (int u = 0; u < NC; ++u)
-      if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
-  }
-  float ya = -INFINITY, yb = -INFINITY;
-#pragma unroll
-  for (int u = 0; u < NC; u += 4) {
-    ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
-    yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
-  }
-  return fmaxf(ya, yb) * c;  // c > 0, so the max commutes with the scaling
-}
-
-// Writing sweep over a query row of S (pass 1): P = exp2(S c - mu) as hi/lo
-// bf16 planes written over the S columns (tokens 16k..16k+15 keep hi in columns
-// [16k, 16k+8) and lo in [16k+8, 16k+16), inside the columns already read);
-// returns the row's sum of P.  Warp-collective.
-template <int NC>
-__device__ __forceinline__ float p1_tile_pass(uint32_t tS, int tile0, bool masked, int Prow,
-                                              uint64_t c2, float mu) {
+// Writes P = exp2(S c - mu) for one warp's 32 tokens of a query row (S already
+// in registers, masked keys at -inf) as hi/lo bf16 planes over the same 32
+// TMEM columns: tokens 16k..16k+15 keep hi in columns [16k, 16k+8) and lo in
+// [16k+8, 16k+16).  Returns the row's sum of P over the 32 tokens.
+// Warp-collective.
+__device__ __forceinline__ float p1_exp32(const uint32_t (&sr)[32], uint32_t tS, uint64_t c2,
+                                          float mu) {
   const uint64_t nmu2 = pk2(-mu, -mu);
   uint64_t l2 = pk2(0.f, 0.f);
 #pragma unroll
-  for (int cc = 0; cc < NC / 32; ++cc) {  // 32 tokens per load
-    uint32_t sr[32];
-    tmem_ld32(tS + cc * 32, sr);
-    if (masked) {
+  for (int half = 0; half < 2; ++half) {  // 16 tokens -> 8 hi + 8 lo columns
+    uint32_t hi[8], lo[8];
 #pragma unroll
-      for (int u = 0; u < 32; ++u)
-        if (tile0 + cc * 32 + u > Prow) sr[u] = 0xFF800000u;
+    for (int u2 = 0; u2 < 8; ++u2) {
+      const int u = half * 16 + 2 * u2;
+      float d0, d1;
+      upk2(ffma2(pk2(f32(sr[u]), f32(sr[u + 1])), c2, nmu2), d0, d1);
+      const float e0 = ex2(d0), e1 = ex2(d1);
+      const uint64_t E = pk2(e0, e1);
+      l2 = fadd2(l2, E);
+      hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
+      const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
+      const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
+      float r0, r1;
+      upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
+      lo[u2] = pack_bf16_rn(r0, r1);
     }
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {  // 16 tokens -> 8 hi + 8 lo columns
-      uint32_t hi[8], lo[8];
-#pragma unroll
-      for (int u2 = 0; u2 < 8; ++u2) {
-        const int u = half * 16 + 2 * u2;
-        float d0, d1;
-        upk2(ffma2(pk2(f32(sr[u]), f32(sr[u + 1])), c2, nmu2), d0, d1);
-        const float e0 = ex2(d0), e1 = ex2(d1);
-        const uint64_t E = pk2(e0, e1);
-        l2 = fadd2(l2, E);
-        hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
-        const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
-        const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
-        float r0, r1;
-        upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
-        lo[u2] = pack_bf16_rn(r0, r1);
-      }
-      tmem_st8(tS + cc * 32 + half * 16, hi);
-      tmem_st8(tS + cc * 32 + half * 16 + 8, lo);
-    }
+    tmem_st8(tS + half * 16, hi);
+    tmem_st8(tS + half * 16 + 8, lo);
   }
   float la, lb;
   upk2(l2, la, lb);
@@ -217,33 +182,30 @@ __device__ __forceinline__ float p1_tile_pass(uint32_t tS, int tile0, bool maske
 }
 
 // Rare path of pass 1, out of line: the reference max moved for some lanes
-// (factor fac <= 1 for them, 1 for the others), so this warp's 64 columns of O
+// (factor fac <= 1 for them, 1 for the others), so this warp's 32 columns of O
 // are rescaled once the previous P V (the `prev`-th) has landed.
 // Warp-collective.  Returns false on a timeout.
 __device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, int prev, uint32_t od_bar) {
   if (!warp_wait(od_bar, prev & 1)) return false;
   tc_fence_after();
-  for (int cc = 0; cc < 2; ++cc) {
-    uint32_t o[32];
-    tmem_ld32(tO + cc * 32, o);
+  uint32_t o[32];
+  tmem_ld32(tO, o);
 #pragma unroll
-    for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
-    tmem_st32(tO + cc * 32, o);
-  }
+  for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
+  tmem_st32(tO, o);
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads1, 1)
-k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+__global__ void __maxnreg__(kMaxRegs)
+k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+           const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTileBytes;                // kSt1 stages
-  uint8_t* sV = smem + (1 + kSt1) * kTileBytes;   // kSt1 stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (1 + 2 * kSt1) * kTileBytes);  // 19 barriers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint8_t* sK = smem;                     // kSt1 stages
+  uint8_t* sV = smem + kSt1 * kTileBytes;  // kSt1 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kSt1 * kTileBytes);  // 22 barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xmax = reinterpret_cast<float*>(tmem_slot + 2);  // [2 tile parities][2 halves][128]
+  float* xmax = reinterpret_cast<float*>(tmem_slot + 2);  // [2 tile parities][4 groups][128]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1 KB alignment
     if (threadIdx.x == 0) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
@@ -253,29 +215,33 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   decode_cta(a, blockIdx.x, b, h, chunk, t0, t1);
   const int T = t1 - t0;
   const int L = a.L[b];
-  const uint32_t BQ = smem_u32(&bars[0]);
-  auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };   // kSt1 each: K full / empty,
-  auto KE = [&](int s) { return smem_u32(&bars[4 + s]); };   // V full / empty
-  auto VF = [&](int s) { return smem_u32(&bars[7 + s]); };
-  auto VE = [&](int s) { return smem_u32(&bars[10 + s]); };
-  auto SF = [&](int b) { return smem_u32(&bars[13 + b]); };  // 2 TMEM buffers: S ready,
-  auto PF = [&](int b) { return smem_u32(&bars[15 + b]); };  // P written,
-  auto XB = [&](int b) { return smem_u32(&bars[17 + b]); };  // tile-max exchange
-  const uint32_t OD = smem_u32(&bars[19]);                     // P V into O done
+  auto KF = [&](int s) { return smem_u32(&bars[s]); };       // kSt1 each: K full / empty,
+  auto KE = [&](int s) { return smem_u32(&bars[3 + s]); };   // V full / empty
+  auto VF = [&](int s) { return smem_u32(&bars[6 + s]); };
+  auto VE = [&](int s) { return smem_u32(&bars[9 + s]); };
+  auto SF = [&](int b) { return smem_u32(&bars[12 + b]); };  // 2 TMEM buffers: S ready,
+  auto PF = [&](int b) { return smem_u32(&bars[14 + b]); };  // P written,
+  auto XB = [&](int b) { return smem_u32(&bars[16 + b]); };  // tile-max exchange
+  const uint32_t OD = smem_u32(&bars[18]);                     // P V into O done
+  auto PD = [&](int b) { return smem_u32(&bars[19 + b]); };  // P V of a buffer done
+  // O final: committed once, after the last P V.  (OD's parity alone cannot
+  // tell the last P V from the one before it once the loop has ended.)
+  const uint32_t OF = smem_u32(&bars[21]);
   if (threadIdx.x == 0) {
-    mbar_init(BQ, 1);
     mbar_init(OD, 1);
+    mbar_init(OF, 1);
     for (int s = 0; s < kSt1; ++s) {
       mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1);
       mbar_init(VE(s), 2);  // P V commit + the ||v||^2 warp's reads
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(SF(b), 1); mbar_init(PF(b), 256); mbar_init(XB(b), 8);
+      mbar_init(SF(b), 1); mbar_init(PF(b), kSimtWarps); mbar_init(XB(b), kSimtWarps);
+      mbar_init(PD(b), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
     tc_fence_before();
@@ -285,14 +251,35 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const uint32_t tbase = *tmem_slot;
   const int z = b * a.Hkv + h;
   const int qrow0 = (b * a.Hkv + h) * a.G * a.w + chunk * a.nqc;
+  if (warp < kSimtWarps) {
+    // Q of the chunk into TMEM columns [kColQ, kColQ + 64): row r of the chunk
+    // in lane r, head-dim pair (2c, 2c+1) in column c (the A operand of S = Q K^T);
+    // rows past the chunk are zero.  Warp (g, quarter) moves head dims [32g, 32g+32).
+    const int g = warp >> 2, ql = warp & 3, r = ql * 32 + lane;
+    uint32_t wq[16];
+    if (r < a.nqc) {
+      const uint4* src =
+          reinterpret_cast<const uint4*>(a.q + ((size_t)qrow0 + r) * kHd + g * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 x = src[i];
+        wq[4 * i] = x.x; wq[4 * i + 1] = x.y; wq[4 * i + 2] = x.z; wq[4 * i + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) wq[i] = 0u;
+    }
+    tmem_st16(tbase + kColQ + (uint32_t)(g * 16) + ((uint32_t)(ql * 32) << 16), wq);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
-  if (warp == 8) {
+  if (warp == kWarpTma) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
-      mbar_expect_tx(BQ, 2u * 128u * (uint32_t)a.qbox_rows);
-      tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
-      tma_load_2d(smem_u32(sQ) + kBox, &tmQ, BQ, 64, qrow0);
+      prefetch_tmap(&tmK); prefetch_tmap(&tmV);
       auto load = [&](uint8_t* buf, uint32_t full, uint32_t empty, const CUtensorMap* m, int i) {
         const int s = i % kSt1, ph = (i / kSt1) & 1;
         if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); return false; }
@@ -308,22 +295,30 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (ok) ok = load(sV, VF(j % kSt1), VE(j % kSt1), &tmV, j);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ----------------
-    constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T
+    constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T (Q from TMEM)
     constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);    // O += P V (V MN-major)
-    bool ok = warp_wait(BQ, 0);
-    if (!ok) fail(a, abort_flag);
-    const uint32_t qbase = smem_u32(sQ);
+    bool ok = true;
+    // operand descriptors of stage 0; a stage or K slice only moves the start
+    // address, i.e. adds to the low word (few instructions per MMA: this warp
+    // shares its issue slots with four softmax warps)
+    const SDesc kd0 = sdesc_split(smem_u32(sK), 16, 1024);
+    const SDesc vd0 = sdesc_split(smem_u32(sV), kBox, 1024);
+    const uint32_t tq = tbase + kColQ;
     auto issue_S = [&](int i) {
       const int s = i % kSt1, ph = (i / kSt1) & 1, bf = i & 1;
       if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
+      // S(i) overwrites the buffer whose P the (i-2)-th P V reads from TMEM:
+      // wait until that P V has completed
+      if (i >= 2 && !warp_wait(PD(bf), ((i - 2) >> 1) & 1)) { fail(a, abort_flag); return false; }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t kb = smem_u32(sK + s * kTileBytes);
+        const uint32_t klo = kd0.lo + (uint32_t)s * (kTileBytes >> 4);
         const uint32_t dS = tbase + (uint32_t)(bf * 128);
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(dS, kmajor_desc(qbase, 128, kk), kmajor_desc(kb, 128, kk), IDS, kk > 0);
+          mma_ts_w(dS, tq + (uint32_t)(8 * kk), klo + kslice(kk, 128), kd0.hi, IDS, kk > 0 ? 1u : 0u);
         mma_commit(KE(s));
         mma_commit(SF(bf));
       }
@@ -350,17 +345,22 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       __syncwarp();
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vbase = smem_u32(vb);
-        const uint32_t dO = tbase + 256u;  // one O: both halves of every tile feed it
+        const uint32_t vlo = vd0.lo + (uint32_t)s * (kTileBytes >> 4);
+        const uint32_t dO = tbase + kColO;
         const uint32_t pS = tbase + (uint32_t)(bf * 128);
-        // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16)
+        // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16);
+        // V slice kk starts 16 rows (2048 bytes) further
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dO, pS + (uint32_t)(16 * kk), vmn_desc(vbase, kk), IDP,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_w(dO, pS + (uint32_t)(16 * kk), vlo + (uint32_t)kk * 128u, vd0.hi, IDP,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dO, pS + (uint32_t)(16 * kk + 8), vmn_desc(vbase, kk), IDP, 1u);
+          mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
         mma_commit(VE(s));
         mma_commit(OD);
+        mma_commit(PD(bf));
+        if (i == T - 1) mma_commit(OF);
       }
       __syncwarp();
       return true;
@@ -370,12 +370,13 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       if (j + 1 < T) ok = issue_S(j + 1);
       if (ok) ok = issue_PV(j);
     }
-  } else if (warp == 10) {
+  } else if (warp == kWarpNv) {
     // ---------------- ||v_j||^2 ----------------
     // This CTA's share of every V tile's rows (the query chunks of a KV head
     // cover the same tokens and split the rows), 4 rows per lane; the order of
     // the squares is free, so the 128-byte swizzle only picks a bank-conflict-
-    // free order.  Arrives on the V stage's empty barrier when done.
+    // free order.  Arrives on the V stage's empty barrier when done, and
+    // records the share's minimum for pass 2.
     for (int j = 0; j < T; ++j) {
       const int s = j % kSt1, ph = (j / kSt1) & 1;
       if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); break; }
@@ -410,18 +411,19 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       vmin = warp_min(vmin);  // pass 2 decides from it whether A needs its low part
       if (lane == 0) a.tmin[((size_t)z * a.ntmax + t0 + j) * a.chunks + chunk] = vmin;
     }
-  } else {
-    // ---------------- softmax warpgroups ----------------
-    // Both warpgroups work on every tile: warpgroup wg owns the tile's tokens
-    // [64 wg, 64 wg + 64) (its S/P columns) and O's head-dim columns
-    // [64 wg, 64 wg + 64); a row's two halves exchange their tile max.
-    const int wg = warp >> 2, wl = warp & 3;
-    const int row = wl * 32 + lane;  // query row within the chunk; token row for ||v||^2
+  } else if (warp < kSimtWarps) {
+    // ---------------- softmax warps ----------------
+    // Sixteen warps work on every tile: warp (g, quarter) owns the query rows
+    // [32 quarter, +32) (its TMEM lanes), the tile's tokens [32 g, 32 g + 32)
+    // (its S/P columns) and O's head-dim columns [32 g, 32 g + 32); the four
+    // warps of a row exchange their tile max through shared memory.
+    const int g = warp >> 2, ql = warp & 3;
+    const int row = ql * 32 + lane;  // query row within the chunk
     const bool valid_row = row < a.nqc;
     const int Prow = valid_row ? L - a.w + (chunk * a.nqc + row) % a.w : L - 1;
-    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-    const int c0 = wg * 64;
-    const uint32_t tO = tbase + 256u + (uint32_t)c0 + lane_off;
+    const uint32_t lane_off = (uint32_t)(ql * 32) << 16;
+    const int c0 = g * 32;
+    const uint32_t tO = tbase + kColO + (uint32_t)c0 + lane_off;
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
     float m_ref = -INFINITY, l = 0.f;
@@ -431,17 +433,28 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       if (warp_aborted(abort_flag)) break;
       tc_fence_after();
       const uint32_t tS = tbase + (uint32_t)(s * 128) + lane_off + (uint32_t)c0;
-      const int tile0 = (t0 + j) * kTok;
-      const bool masked = tile0 + c0 + 63 > L - a.w;
+      const int tok0 = (t0 + j) * kTok + c0;
+      uint32_t sr[32];
+      tmem_ld32(tS, sr);
+      if (tok0 + 31 > L - a.w) {  // only the last tiles: hide keys past P_t
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+          if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
+      }
+      float ya = -INFINITY, yb = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 32; u += 4) {
+        ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
+        yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
+      }
       // the reference max moves only when a tile exceeds it by more than 8
       // (so 2^(S c - m) <= 256); then l and O are rescaled
-      const float mh = p1_tile_max<64>(tS, tile0 + c0, masked, Prow, c);
-      float* xm = xmax + s * 256;
-      xm[wg * 128 + row] = mh;
+      float* xm = xmax + s * 512;
+      xm[g * 128 + row] = fmaxf(ya, yb) * c;  // c > 0: the max commutes with the scaling
       __syncwarp();
       if (lane == 0) mbar_arrive(XB(s));
       if (!warp_wait(XB(s), ph)) { fail(a, abort_flag); break; }
-      const float mt = fmaxf(mh, xm[(1 - wg) * 128 + row]);
+      const float mt = fmaxf(fmaxf(xm[row], xm[128 + row]), fmaxf(xm[256 + row], xm[384 + row]));
       float fac = 1.f;
       bool resc = false;
       if (mt > m_ref + 8.f) {
@@ -455,40 +468,37 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         fail(a, abort_flag);
         break;
       }
-      l += p1_tile_pass<64>(tS, tile0 + c0, masked, Prow, c2, m_ref == -INFINITY ? 0.f : m_ref);
+      l += p1_exp32(sr, tS, c2, m_ref == -INFINITY ? 0.f : m_ref);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(PF(s));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(PF(s));
     }
-    // partial row: O half of this warpgroup, the shared max, its normaliser half
+    // partial row: this warp's 32 columns of O, the shared max, its normaliser part
     float* out = a.partial + ((size_t)blockIdx.x * 128 + row) * kPartStride;
     bool have = T > 0 && !warp_aborted(abort_flag);
     if (have) {
-      if (!warp_wait(OD, (T - 1) & 1)) {
+      if (!warp_wait(OF, 0)) {
         fail(a, abort_flag);
         have = false;
       }
       tc_fence_after();
     }
-    for (int cc = 0; cc < 2; ++cc) {
-      uint32_t o[32];
-      if (have) tmem_ld32(tO + cc * 32, o);
-      if (valid_row) {
-#pragma unroll
-        for (int u = 0; u < 32; u += 4)
-          *reinterpret_cast<float4*>(out + c0 + cc * 32 + u) =
-              have ? make_float4(f32(o[u]), f32(o[u + 1]), f32(o[u + 2]), f32(o[u + 3]))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
+    uint32_t o[32];
+    if (have) tmem_ld32(tO, o);
     if (valid_row) {
-      if (wg == 0) out[128] = have ? m_ref : -INFINITY;
-      out[129 + wg] = have ? l : 0.f;
+#pragma unroll
+      for (int u = 0; u < 32; u += 4)
+        *reinterpret_cast<float4*>(out + c0 + u) =
+            have ? make_float4(f32(o[u]), f32(o[u + 1]), f32(o[u + 2]), f32(o[u + 3]))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (g == 0) out[128] = have ? m_ref : -INFINITY;
+      out[129 + g] = have ? l : 0.f;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -519,7 +529,7 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
     const float* p = P(i);
     const float mi = p[128];
     const float wgt = (mi == -INFINITY) ? 0.f : ex2(mi - M);
-    Lsum += wgt * (p[129] + p[130]);  // the two warpgroups' normaliser halves
+    Lsum += wgt * ((p[129] + p[130]) + (p[131] + p[132]));  // the four normaliser parts
     const float4 o = *reinterpret_cast<const float4*>(p + lane * 4);
     acc.x = fmaf(wgt, o.x, acc.x);
     acc.y = fmaf(wgt, o.y, acc.y);
@@ -630,7 +640,7 @@ __device__ __noinline__ float careful16(uint32_t tS, uint32_t tD, int col0, int 
   return acc;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(kMaxRegs)
 k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmAhi,
            const __grid_constant__ CUtensorMap tmAlo, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
@@ -667,7 +677,7 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(MD(s), 1); mbar_init(TF(s), 8);  // both warpgroups read every tile
+      mbar_init(MD(s), 1); mbar_init(TF(s), kSimtWarps);  // every warp reads every tile
     }
     for (int r = 0; r < kRing2; ++r) {
       mbar_init(FULL(r), 1); mbar_init(EMPTY(r), 1);
@@ -683,7 +693,7 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     kff[(i >> 1) * 4 + 2 + (i & 1)] = q.w;
   }
   if (threadIdx.x < 8) nAmax[threadIdx.x] = 0.f;
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
     tc_fence_before();
@@ -714,7 +724,7 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == kWarpTma) {
     if (lane == 0) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmAhi); prefetch_tmap(&tmAlo);
       prefetch_tmap(&tmK); prefetch_tmap(&tmV);
@@ -739,11 +749,14 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         tma_load_3d(dst + kBox, m, FULL(r), 64, row, z);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kWarpMma) {
     const uint32_t IDT = idesc_bf16(128, nqc, false, false);
     bool ok = warp_wait(BQ, 0);
     if (!ok) fail(a, abort_flag);
-    const uint32_t qb = smem_u32(sQ), hb = smem_u32(sAh), lb = smem_u32(sAl);
+    const SDesc rd0 = sdesc_split(smem_u32(sRing), 16, 1024);  // ring slot 0
+    const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024), hd = sdesc_split(smem_u32(sAh), 16, 1024),
+                ld = sdesc_split(smem_u32(sAl), 16, 1024);
+    const uint32_t nq = (uint32_t)nqc;
     for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
       const int rk = (2 * j) % R, pk = ((2 * j) / R) & 1;
@@ -754,38 +767,46 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         break;
       }
       tc_fence_after();
-      const uint32_t kb = smem_u32(sRing + rk * kTileBytes), vb = smem_u32(sRing + rv * kTileBytes);
+      const uint32_t klo = rd0.lo + (uint32_t)rk * (kTileBytes >> 4);
+      const uint32_t vlo = rd0.lo + (uint32_t)rv * (kTileBytes >> 4);
       if (lane == 0) {
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(dS, kmajor_desc(kb, 128, kk), kmajor_desc(qb, nqc, kk), IDT, kk > 0);
+          mma_ss_w(dS, klo + kslice(kk, 128), rd0.hi, qd.lo + kslice(kk, nq), qd.hi, IDT,
+                   kk > 0 ? 1u : 0u);
         mma_commit(EMPTY(rk));
       }
       __syncwarp();
       if (!warp_wait(FULL(rv), pv)) { fail(a, abort_flag); break; }
       tc_fence_after();
       if (lane == 0) {
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(dD, kmajor_desc(vb, 128, kk), kmajor_desc(hb, nqc, kk), IDT, kk > 0);
-        if (lo)
+          mma_ss_w(dD, vlo + kslice(kk, 128), rd0.hi, hd.lo + kslice(kk, nq), hd.hi, IDT,
+                   kk > 0 ? 1u : 0u);
+        if (lo) {
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(dD, kmajor_desc(vb, 128, kk), kmajor_desc(lb, nqc, kk), IDT, 1u);
+            mma_ss_w(dD, vlo + kslice(kk, 128), rd0.hi, ld.lo + kslice(kk, nq), ld.hi, IDT, 1u);
+        }
         mma_commit(EMPTY(rv));
         mma_commit(MD(s));
       }
       __syncwarp();
     }
-  } else {
-    // Both warpgroups work on every tile: warpgroup wg owns the query columns
-    // [64 wg, min(nqc, 64 wg + 64)) and writes its own partial-score plane.
-    const int wg = warp >> 2, wl = warp & 3;
-    const int row = wl * 32 + lane;  // token within the tile
-    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+  } else if (warp < kSimtWarps) {
+    // Sixteen warps work on every tile: warp (g, quarter) owns the tokens
+    // [32 quarter, +32) of the tile (its TMEM lanes) and the query columns
+    // [32 g, min(nqc, 32 g + 32)), and writes its own partial-score plane.
+    const int g = warp >> 2, ql = warp & 3;
+    const int row = ql * 32 + lane;  // token within the tile
+    const uint32_t lane_off = (uint32_t)(ql * 32) << 16;
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
-    const int ch0 = wg * 4, ch1 = min(nqc / 16, ch0 + 4);  // 16-column chunks owned
+    const int ch0 = min(nqc / 16, 2 * g), ch1 = min(nqc / 16, 2 * g + 2);  // 16-column chunks
     const float4* qrows = a.qstat + qrow0;
     const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
-    float* plane = a.parts + (size_t)(chunk * 2 + wg) * a.part_stride + (size_t)z * a.n_max;
+    float* plane = a.parts + (size_t)(chunk * 4 + g) * a.part_stride + (size_t)z * a.n_max;
     int sing = 0;
     for (int j = 0; j < T; ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
@@ -807,40 +828,21 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                            vrow_g, &sing);
       } else {
         const uint64_t nv2 = pk2(nv, nv);
-        for (int ch = ch0; ch < ch1; ch += 2) {
-          // 32 columns of S^T and D in one TMEM round trip when available
-          const bool two = ch + 1 < ch1;
-          uint32_t r0[32], r1[32];
-          if (two) {
-            uint32_t rr[64];
-            tmem_ld32x2(tS + ch * 16, tD + ch * 16, rr);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              r0[u] = rr[u];            // S^T columns ch*16 .. +15
-              r0[16 + u] = rr[32 + u];  // D columns ch*16 .. +15
-              r1[u] = rr[16 + u];
-              r1[16 + u] = rr[48 + u];
-            }
+        for (int ch = ch0; ch < ch1; ++ch) {
+          uint32_t r[32];
+          tmem_ld16x2(tS + ch * 16, tD + ch * 16, r);  // 16 columns of S^T and of D
+          uint64_t a2 = pk2(0.f, 0.f);
+          float pmax = 0.f;
+          fast16(r, kf + ch * 8, c2, nv2, a2, pmax);
+          // dominant token (p >= 2^-8) or possible cancellation (||A||^2 >= 0.6 ||v||^2)
+          const bool redo = pmax >= 0.00390625f || nAmax[ch] >= 0.6f * nv;
+          if (__any_sync(0xffffffffu, redo)) {
+            acc += careful16(tS, tD, ch * 16, tok, false, L, a.w, chunk * nqc, qrows, c, nv,
+                             arows, vrow_g, &sing);
           } else {
-            tmem_ld16x2(tS + ch * 16, tD + ch * 16, r0);
-          }
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            if (k == 1 && !two) break;
-            const int cw = ch + k;
-            uint64_t a2 = pk2(0.f, 0.f);
-            float pmax = 0.f;
-            fast16(k ? r1 : r0, kf + cw * 8, c2, nv2, a2, pmax);
-            // dominant token (p >= 2^-8) or possible cancellation (||A||^2 >= 0.6 ||v||^2)
-            const bool redo = pmax >= 0.00390625f || nAmax[cw] >= 0.6f * nv;
-            if (__any_sync(0xffffffffu, redo)) {
-              acc += careful16(tS, tD, cw * 16, tok, false, L, a.w, chunk * nqc, qrows, c, nv,
-                               arows, vrow_g, &sing);
-            } else {
-              float x0, x1;
-              upk2(a2, x0, x1);
-              acc += x0 + x1;
-            }
+            float x0, x1;
+            upk2(a2, x0, x1);
+            acc += x0 + x1;
           }
         }
       }
@@ -853,7 +855,7 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -900,7 +902,7 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
 }
 
 size_t pass1_smem() {
-  return (1 + 2 * kSt1) * (size_t)kTileBytes + 20 * 8 + 8 + 2 * 2 * 128 * 4;
+  return 2 * kSt1 * (size_t)kTileBytes + 22 * 8 + 8 + 2 * 4 * 128 * 4;
 }
 size_t pass2_smem(int nqc) {
   return kRing2 * (size_t)kTileBytes + 2 * (size_t)nqc * 256 + (size_t)nqc / 2 * 16 + 8 * 4 +
@@ -968,6 +970,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   for (int i = 0; i < lens.B; ++i) a.cta_base[i + 1] = a.cta_base[i] + units * a.splits[i];
   const int ctas = a.cta_base[lens.B];
   a.c_log2 = (float)(1.4426950408889634 / sqrt((double)s.d));
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
   a.partial = reinterpret_cast<float*>(ws + lay.tc_partial);
   a.status = status;
   a.ahi = reinterpret_cast<__nv_bfloat16*>(ws + lay.tc_ahi);
@@ -1001,7 +1004,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   if (e != cudaSuccess) return e;
 
   kev.begin(st);
-  k_tc_pass1<<<ctas, kThreads1, sm1, st>>>(mQ1, mK, mV, a);
+  k_tc_pass1<<<ctas, kThreads1, sm1, st>>>(mK, mV, a);
   kev.end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kev.begin(st);
@@ -1009,7 +1012,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   kev.end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kev.begin(st);
-  k_tc_pass2<<<ctas, kThreads, sm2, st>>>(mQ2, mAh, mAl, mK, mV, a);
+  k_tc_pass2<<<ctas, kThreads2, sm2, st>>>(mQ2, mAh, mAl, mK, mV, a);
   kev.end(st);
   return cudaGetLastError();
 }
