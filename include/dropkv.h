@@ -171,10 +171,11 @@ DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, co
  * device synchronisation).  The paper has no counterpart: this is an interface
  * variant of the eviction step above, with the same arguments minus the
  * workspace and the same results.
- *   Scratch: a 1 MiB array of static device memory inside the library, held by
+ *   Scratch: a 4 KiB array of static device memory inside the library, held by
  *   every GPU that loads the library until the process exits.  Sizes whose
- *   dropkv_select_workspace_bytes(min(B, 64), Hkv, n_max) exceeds 1 MiB are
- *   rejected with DROPKV_ERR_WORKSPACE before anything is enqueued.
+ *   dropkv_select_workspace_bytes(min(B, 64), Hkv, n_max) exceeds 4 KiB would be
+ *   rejected with DROPKV_ERR_WORKSPACE before anything is enqueued (the select
+ *   path needs 256 bytes for any size, so none is).
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
  *   before any stream capture.  No call allocates or frees memory.

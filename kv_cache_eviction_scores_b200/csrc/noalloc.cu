@@ -23,9 +23,9 @@
 namespace dropkv {
 namespace {
 
-// Largest scratch the select kernels may use here: 1 MiB (enough for, e.g.,
-// 64 (batch row, KV head) segments of 128K tokens each).
-constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
+// Scratch of the select kernels here: 4 KiB (the select path keeps its state
+// in shared memory and needs only a status word, for any size).
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 10;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];

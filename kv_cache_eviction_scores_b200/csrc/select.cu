@@ -1,47 +1,58 @@
-// select.cu -- exact lowest-score eviction per (b, KV head): multi-CTA radix
-// select plus an order-preserving compaction.
+// select.cu -- exact lowest-score eviction per (b, KV head): one thread-block
+// cluster per segment runs a radix select over the segment's keys and an
+// order-preserving compaction, in a single launch.
 //
 // Write-up "DropKV：精确单项输出扰动评分组件", Algorithm 1 paragraph: after
 // pooling and window protection, the lowest-scoring tokens are evicted.  The
 // order used is (score ascending, position ascending); NaN sorts above +inf.
 //
-// Scores map to 32-bit keys whose unsigned order is the float order.  Every
-// segment (b, h) is cut into 4096-key chunks, one CTA each, so the work spreads
-// over the whole GPU even when B * Hkv is small.
-//   round 0..2: histogram of an 11/11/10-bit digit of the keys that match the
-//       prefix found so far; the last CTA of a segment to finish (an atomic
-//       arrival counter, no waiting) picks the digit holding the E-th smallest
-//       key.  After round 2 the prefix is the threshold key T and `rem` is how
-//       many keys equal to T are evicted (the lowest positions among them).
-//   count: per chunk, #keys < T and #keys == T; the last CTA of the segment
-//       turns them into exclusive prefixes.
-//   write: each chunk walks its keys in position order with block scans and
-//       writes kept / evicted positions to their final slots.
-// Outputs are pre-filled with -1 by the init kernel.
+// Scores map to 32-bit keys whose unsigned order is the float order.  A
+// segment (b, h) of L keys is split into kC contiguous ranges, one per CTA of
+// a kC-CTA cluster; a range is cached in shared memory when it fits.
+// A range is processed in sub-ranges of 16384 keys (one when it fits the
+// shared-memory cache, which then holds it for every phase).
+//   rounds 0..2: every CTA histograms an 11/11/10-bit digit of its keys that
+//       match the prefix found so far and adds the histogram into rank 0's
+//       shared memory (distributed shared memory atomics; one histogram per
+//       round, all zeroed at the start) and arrives on rank 0's gather
+//       barrier; rank 0 finds the digit holding the E-th smallest key,
+//       stores (prefix, rank) into every CTA and arrives on every CTA's
+//       broadcast barrier.
+//       After round 2 the prefix is the threshold key T and `rem` is how many
+//       keys equal to T are evicted (the lowest positions among them).
+//   count: every CTA stores its counts of keys < T and == T into every CTA;
+//       each CTA then sums the counts of the lower ranks (the ranges are in
+//       position order).
+//   write: per sub-range of 16384 keys, each thread takes 32 consecutive
+//       keys; two block scans give every thread its kept / evicted ranks, the
+//       positions are staged in shared memory and copied out coalesced.
+// The phases are separated by cluster-wide mbarrier phases with bounded waits;
+// a wait that gives up records DROPKV_ERR_TIMEOUT in the workspace status word
+// and the CTA keeps taking the remaining phase barriers (without the work), so
+// no CTA leaves while another may still address its shared memory.
 #include "common.cuh"
 #include "internal.h"
 
 namespace dropkv {
 namespace {
 
-constexpr int kChunk = 4096;
-constexpr int kThreads = 256;
+constexpr int kC = 8;                // CTAs per cluster: one cluster per segment
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
-
-struct SegState {
-  uint32_t prefix;  // digits found so far; after round 2 the threshold key T
-  int32_t rem;      // rank still to place; after round 2 the quota among keys == T
-  uint32_t arrive;  // arrival counter for the last-CTA step
-  int32_t done;     // 1: nothing to select (no eviction)
-};
+constexpr int kPer = 32;             // consecutive keys per thread in one sub-range
+constexpr int kSub = kThreads * kPer;  // keys per sub-range (16384)
+constexpr int kCopies = 4;           // histogram copies (warp % 4), padded apart by one bank
+constexpr int kCopyStride = kBins + 1;
+constexpr uint64_t kWaitNs = 2000000000ull;
 
 struct SelParams {
   int32_t B, Hkv, n_max;
   int32_t max_keep, max_evict;
   int32_t L[kMaxB];
-  int32_t E[kMaxB];            // evictions per row
-  int32_t nchunk[kMaxB];       // chunks per segment of row b
-  int32_t chunk_base[kMaxB + 1];  // first CTA of row b (Hkv segments each)
+  int32_t E[kMaxB];                  // evictions per row
+  int32_t* status;                   // device status word (0 = OK)
+  int32_t cache;                     // 1: every CTA's range fits one cached sub-range
 };
 
 __device__ __forceinline__ uint32_t key_of(float s) {
@@ -50,279 +61,436 @@ __device__ __forceinline__ uint32_t key_of(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// CTA -> (b, h, chunk)
-__device__ __forceinline__ void locate(const SelParams& p, int blk, int& b, int& h, int& c) {
-  b = 0;
-  while (b + 1 < p.B && blk >= p.chunk_base[b + 1]) ++b;
-  const int local = blk - p.chunk_base[b];
-  h = local / p.nchunk[b];
-  c = local % p.nchunk[b];
+// ---- cluster / distributed shared memory -----------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// address of the same shared-memory variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void dsm_add(uint32_t raddr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(raddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void dsm_st(uint32_t raddr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(raddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t dsm_ld(uint32_t raddr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(raddr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
 
-struct Workspace {
-  SegState* seg;
-  uint32_t* hist;   // [segments][kBins]
-  int32_t* cnt;     // [chunks][2]: #< T, #== T
-  int32_t* off;     // [chunks][2]: exclusive prefixes within the segment
-};
-
-__device__ __forceinline__ Workspace carve(void* ws, const SelParams& p) {
-  const int segs = p.B * p.Hkv;
-  const int chunks = p.chunk_base[p.B];
-  char* base = reinterpret_cast<char*>(ws);
-  Workspace w;
-  w.seg = reinterpret_cast<SegState*>(base);
-  size_t o = align_up(sizeof(SegState) * segs, 256);
-  w.hist = reinterpret_cast<uint32_t*>(base + o);
-  o += align_up(sizeof(uint32_t) * kBins * (size_t)segs, 256);
-  w.cnt = reinterpret_cast<int32_t*>(base + o);
-  o += align_up(sizeof(int32_t) * 2 * (size_t)chunks, 256);
-  w.off = reinterpret_cast<int32_t*>(base + o);
-  return w;
+// Block-wide exclusive prefix sum of one int per thread (kThreads threads);
+// also returns the block total.  Contains __syncthreads.
+__device__ __forceinline__ int block_excl_scan(int v, int& total, int* warp_tot) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[wid] = x;
+  __syncthreads();
+  int before = 0;
+  total = 0;
+  for (int i = 0; i < kWarps; ++i) {
+    const int t = warp_tot[i];
+    if (i < wid) before += t;
+    total += t;
+  }
+  __syncthreads();
+  return before + x - v;
 }
 
-__global__ void k_sel_init(SelParams p, void* ws, int32_t* keep_idx, int32_t* evict_idx) {
-  Workspace w = carve(ws, p);
-  const int segs = p.B * p.Hkv;
-  const size_t tid = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
-  const size_t nthr = (size_t)gridDim.x * blockDim.x;
-  for (size_t i = tid; i < (size_t)segs; i += nthr) {
-    const int b = (int)(i / p.Hkv);
-    SegState s;
-    s.prefix = 0;
-    s.rem = p.E[b];
-    s.arrive = 0;
-    s.done = (p.E[b] == 0) ? 1 : 0;
-    w.seg[i] = s;
-  }
-  for (size_t i = tid; i < (size_t)segs * kBins; i += nthr) w.hist[i] = 0;
-  for (size_t i = tid; i < (size_t)segs * p.max_keep; i += nthr) keep_idx[i] = -1;
-  for (size_t i = tid; i < (size_t)segs * p.max_evict; i += nthr) evict_idx[i] = -1;
+// Thread 0 only: arrive (release, cluster scope) on the mbarrier at shared
+// address `bar` of CTA `rank`.
+__device__ __forceinline__ void arrive_at(uint32_t bar, uint32_t rank) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(bar, rank))
+               : "memory");
 }
-
-__global__ void __launch_bounds__(kThreads)
-k_sel_hist(SelParams p, const float* __restrict__ scores, void* ws, int round) {
-  __shared__ uint32_t sh[kBins];
-  __shared__ int last;
-  __shared__ uint32_t part[kThreads];
-  Workspace w = carve(ws, p);
-  int b, h, c;
-  locate(p, blockIdx.x, b, h, c);
-  const int seg = b * p.Hkv + h;
-  if (w.seg[seg].done) return;  // uniform for the whole segment
-  const int shift = (round == 0) ? 21 : (round == 1) ? 10 : 0;
-  const int width = (round == 2) ? 10 : 11;
-  const uint32_t mask = (1u << width) - 1u;
-  const uint32_t prefix = w.seg[seg].prefix;
-  for (int i = threadIdx.x; i < kBins; i += kThreads) sh[i] = 0;
-  __syncthreads();
-  const int L = p.L[b];
-  const float* s = scores + (size_t)seg * p.n_max;
-  const int beg = c * kChunk, end = min(L, beg + kChunk);
-  for (int j = beg + threadIdx.x; j < end; j += kThreads) {
-    const uint32_t key = key_of(s[j]);
-    if (round == 0 || (key >> (shift + width)) == prefix) atomicAdd(&sh[(key >> shift) & mask], 1u);
-  }
-  __syncthreads();
-  uint32_t* gh = w.hist + (size_t)seg * kBins;
-  for (int i = threadIdx.x; i < kBins; i += kThreads)
-    if (sh[i]) atomicAdd(&gh[i], sh[i]);
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = (atomicAdd(&w.seg[seg].arrive, 1u) == (uint32_t)p.nchunk[b] - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  // Last CTA of the segment: find the digit that holds rank `rem` (1-based).
-  const int per = kBins / kThreads;  // 8 bins per thread
-  uint32_t local[kBins / kThreads];
-  uint32_t tot = 0;
-  for (int i = 0; i < per; ++i) {
-    local[i] = __ldcg(&gh[threadIdx.x * per + i]);
-    tot += local[i];
-  }
-  part[threadIdx.x] = tot;
-  __syncthreads();
-  // inclusive scan of the per-thread totals (Hillis-Steele in shared memory)
-  for (int o = 1; o < kThreads; o <<= 1) {
-    const uint32_t add = (threadIdx.x >= o) ? part[threadIdx.x - o] : 0u;
-    __syncthreads();
-    part[threadIdx.x] += add;
-    __syncthreads();
-  }
-  const uint32_t rem = (uint32_t)w.seg[seg].rem;
-  uint32_t before = part[threadIdx.x] - tot;  // exclusive prefix
-  if (before < rem && rem <= part[threadIdx.x]) {
-    for (int i = 0; i < per; ++i) {
-      if (before + local[i] >= rem) {
-        SegState st = w.seg[seg];
-        st.prefix = (round == 0) ? (uint32_t)(threadIdx.x * per + i)
-                                 : ((prefix << width) | (uint32_t)(threadIdx.x * per + i));
-        st.rem = (int32_t)(rem - before);
-        st.arrive = 0;
-        w.seg[seg] = st;
-        break;
-      }
-      before += local[i];
+// Thread 0 only: bounded wait (acquire, cluster scope) for the phase of
+// parity `parity` of this CTA's mbarrier `bar`.  On expiry records the timeout.
+__device__ bool wait_at(uint32_t bar, uint32_t parity, volatile int* fail, int32_t* status) {
+  const uint64_t t0 = gtimer();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (gtimer() - t0 > kWaitNs) {
+      *fail = 1;
+      atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
+      return false;
     }
   }
-  for (int i = threadIdx.x; i < kBins; i += kThreads) gh[i] = 0;
 }
 
-__global__ void __launch_bounds__(kThreads)
-k_sel_count(SelParams p, const float* __restrict__ scores, void* ws) {
-  __shared__ int32_t red[2][kThreads / 32];
-  __shared__ int last;
-  Workspace w = carve(ws, p);
-  int b, h, c;
-  locate(p, blockIdx.x, b, h, c);
-  const int seg = b * p.Hkv + h;
-  const SegState st = w.seg[seg];
-  const uint32_t T = st.done ? 0u : st.prefix;
-  const int L = p.L[b];
+// One cluster-wide phase: after a block barrier (which orders every thread's
+// prior shared / distributed shared memory writes before thread 0), thread 0
+// fences at cluster scope and arrives on the phase barrier of every CTA of the
+// cluster, then waits (bounded, acquire at cluster scope) for all kC arrivals
+// on its own; a second block barrier releases the other threads.  Returns
+// false once any wait of this CTA has given up.
+__device__ bool cluster_phase(uint32_t bar, int& phase, volatile int* fail, int32_t* status) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+    for (uint32_t r = 0; r < (uint32_t)kC; ++r)
+      asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(bar, r))
+                   : "memory");
+    const uint32_t parity = (uint32_t)(phase & 1);
+    const uint64_t t0 = gtimer();
+    for (;;) {
+      uint32_t done;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(done)
+          : "r"(bar), "r"(parity)
+          : "memory");
+      if (done) break;
+      if (gtimer() - t0 > kWaitNs) {
+        *fail = 1;
+        atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+  __syncthreads();
+  ++phase;
+  return *fail == 0;
+}
+
+__global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 1)
+k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ keep_idx,
+         int32_t* __restrict__ evict_idx) {
+  extern __shared__ uint32_t smem_dyn[];     // [kSub] key cache / staging, then histogram copies
+  uint32_t* cached_keys = smem_dyn;          // this CTA's range when it fits one sub-range
+  int32_t* staging = reinterpret_cast<int32_t*>(smem_dyn + (p.cache ? kSub : 0));
+  uint32_t* loc = smem_dyn + 2 * kSub;       // [kCopies][kCopyStride] this CTA's histograms
+  __shared__ uint32_t H[3][kBins];           // the cluster histogram of each round (rank 0's)
+  __shared__ int32_t warp_tot[kWarps];
+  __shared__ uint32_t cnt[kC][2];            // per-rank (#< T, #== T), stored by every rank
+  __shared__ uint32_t ctl[2];                // this CTA's (prefix, rem) after a round
+  __shared__ int32_t wsum[2][kWarps];
+  __shared__ int32_t bcast[2];
+  __shared__ __align__(8) uint64_t bar;     // all-to-all phases (count, final): kC arrivals
+  __shared__ __align__(8) uint64_t gbar;    // rank 0: a round's histogram adds landed (kC)
+  __shared__ __align__(8) uint64_t bbar;    // every CTA: rank 0 broadcast the round's digit (1)
+  __shared__ int fail;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const uint32_t rank = cluster_rank();
+  const int seg = blockIdx.x / kC;
+  const int b = seg / p.Hkv;
+  const int L = p.L[b], E = p.E[b];
+  const long long span_ll = (((long long)L + kC - 1) / kC + 31) & ~31ll;
+  const int lo = (int)min((long long)L, (long long)rank * span_ll);
+  const int hi = (int)min((long long)L, (long long)lo + span_ll);
+  const bool cached = p.cache != 0;  // sized for the longest row of the launch
   const float* s = scores + (size_t)seg * p.n_max;
-  const int beg = c * kChunk, end = min(L, beg + kChunk);
+  const uint32_t barA = smem_addr(&bar), gbarA = smem_addr(&gbar), bbarA = smem_addr(&bbar);
+
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(barA), "r"(kC) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(gbarA), "r"(kC) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bbarA), "r"(1) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fail = 0;
+    ctl[0] = 0;
+    ctl[1] = (uint32_t)E;
+  }
+  for (int i = tid; i < 3 * kBins; i += kThreads) (&H[0][0])[i] = 0;
+  if (tid < 2 * kC) cnt[tid >> 1][tid & 1] = 0;
+  // cache layout: key r of the range at r ^ ((r >> 5) & 31), so that both the
+  // coalesced fill (32 consecutive r per warp) and the per-thread runs (lane t
+  // reads r = 32 t + u) touch 32 distinct banks
+  if (cached)
+    for (int j = lo + tid; j < hi; j += kThreads) {
+      const int r = j - lo;
+      cached_keys[r ^ ((r >> 5) & 31)] = key_of(__ldg(s + j));
+    }
+  __syncthreads();
+  // every CTA's barrier and histogram are initialised before any remote access
+  // (the one hardware cluster barrier; all threads of all CTAs reach it)
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+  auto key_at = [&](int j) {
+    const int r = j - lo;
+    return cached ? cached_keys[r ^ ((r >> 5) & 31)] : key_of(__ldg(s + j));
+  };
+  // this thread's kPer consecutive keys of the sub-range starting at sub0
+  // (slots past hi read as the NaN key; every use masks them by position)
+  auto load_run = [&](int sub0, uint32_t (&k)[kPer]) {
+    const int j0 = sub0 + tid * kPer;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) k[u] = (j0 + u < hi) ? key_at(j0 + u) : 0xFFFFFFFFu;
+  };
+  const uint32_t H0 = mapa(smem_addr(&H[0][0]), 0);
+  int phase = 0;
+  bool ok = true;
+  uint32_t prefix = 0, rem = (uint32_t)E;
+
+  // ---- radix select: three digit rounds (E is uniform over the cluster) ----
+  if (E > 0) {
+    for (int round = 0; round < 3; ++round) {
+      const int shift = (round == 0) ? 21 : (round == 1) ? 10 : 0;
+      const int width = (round == 2) ? 10 : 11;
+      const uint32_t mask = (1u << width) - 1u;
+      if (ok) {
+        for (int i = tid; i < kCopies * kCopyStride; i += kThreads) loc[i] = 0;
+        __syncthreads();
+        // scores concentrate in few bins: four copies (by warp), one bank apart,
+        // spread the colliding atomics
+        uint32_t* myloc = loc + (wid & (kCopies - 1)) * kCopyStride;
+        for (int sub0 = lo; sub0 < hi; sub0 += kSub) {
+          uint32_t k[kPer];
+          load_run(sub0, k);
+          const int j0 = sub0 + tid * kPer;
+#pragma unroll
+          for (int u = 0; u < kPer; ++u)
+            if (j0 + u < hi && (round == 0 || (k[u] >> (shift + width)) == prefix))
+              atomicAdd(&myloc[(k[u] >> shift) & mask], 1u);
+        }
+        __syncthreads();
+        for (int i = tid; i < kBins; i += kThreads) {
+          uint32_t v = 0;
+#pragma unroll
+          for (int c = 0; c < kCopies; ++c) v += loc[c * kCopyStride + i];
+          if (v) dsm_add(H0 + 4u * (uint32_t)(round * kBins + i), v);
+        }
+      }
+      // gather: every CTA's adds have landed at rank 0
+      __syncthreads();
+      if (tid == 0) {
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        arrive_at(gbarA, 0);
+      }
+      if (rank == 0) {
+        if (tid == 0) wait_at(gbarA, (uint32_t)(round & 1), &fail, p.status);
+        __syncthreads();
+        if (fail == 0) {
+          // the digit holding rank `rem` (1-based) of the keys with this prefix
+          constexpr int per = kBins / kThreads;  // 4 bins per thread
+          uint32_t v[per], tot = 0;
+#pragma unroll
+          for (int i = 0; i < per; ++i) {
+            v[i] = H[round][tid * per + i];
+            tot += v[i];
+          }
+          int total;
+          uint32_t before = (uint32_t)block_excl_scan((int)tot, total, warp_tot);
+          if (before < rem && rem <= before + tot) {
+            for (int i = 0; i < per; ++i) {
+              if (before + v[i] >= rem) {
+                const uint32_t digit = (uint32_t)(tid * per + i);
+                ctl[0] = (round == 0) ? digit : ((prefix << width) | digit);
+                ctl[1] = rem - before;
+                break;
+              }
+              before += v[i];
+            }
+          }
+          __syncthreads();
+          if (tid < kC) {  // broadcast (prefix, rem) into every CTA
+            const uint32_t dst = mapa(smem_addr(ctl), (uint32_t)tid);
+            dsm_st(dst, ctl[0]);
+            dsm_st(dst + 4u, ctl[1]);
+          }
+        }
+        __syncthreads();
+        if (tid == 0) {
+          asm volatile("fence.acq_rel.cluster;" ::: "memory");
+          for (uint32_t r = 0; r < (uint32_t)kC; ++r) arrive_at(bbarA, r);
+        }
+      }
+      // broadcast: the round's (prefix, rem) is in this CTA's ctl
+      if (tid == 0) wait_at(bbarA, (uint32_t)(round & 1), &fail, p.status);
+      __syncthreads();
+      ok = fail == 0;
+      prefix = ctl[0];
+      rem = ctl[1];
+      __syncthreads();  // ctl is read by every thread before the next round's broadcast
+    }
+  }
+  const uint32_t T = prefix;
+  const int quota = E > 0 ? (int)rem : 0;  // keys == T that are evicted
+
+  // ---- counts below / at the threshold, gathered at rank 0 -----------------
   int nlt = 0, neq = 0;
-  if (!st.done)
-    for (int j = beg + threadIdx.x; j < end; j += kThreads) {
-      const uint32_t key = key_of(s[j]);
-      nlt += key < T;
-      neq += key == T;
+  if (ok && E > 0)
+    for (int sub0 = lo; sub0 < hi; sub0 += kSub) {
+      uint32_t k[kPer];
+      load_run(sub0, k);
+      const int j0 = sub0 + tid * kPer;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const bool in = j0 + u < hi;
+        nlt += in && k[u] < T;
+        neq += in && k[u] == T;
+      }
     }
   for (int o = 16; o > 0; o >>= 1) {
     nlt += __shfl_xor_sync(0xffffffffu, nlt, o);
     neq += __shfl_xor_sync(0xffffffffu, neq, o);
   }
-  if ((threadIdx.x & 31) == 0) {
-    red[0][threadIdx.x >> 5] = nlt;
-    red[1][threadIdx.x >> 5] = neq;
+  if (lane == 0) {
+    wsum[0][wid] = nlt;
+    wsum[1][wid] = neq;
   }
   __syncthreads();
-  const int blk = blockIdx.x;
-  if (threadIdx.x == 0) {
+  if (tid < kC && ok) {  // this rank's counts into every CTA of the cluster
     int a = 0, e = 0;
-    for (int i = 0; i < kThreads / 32; ++i) { a += red[0][i]; e += red[1][i]; }
-    w.cnt[2 * blk] = a;
-    w.cnt[2 * blk + 1] = e;
-    __threadfence();
-    last = (atomicAdd(&w.seg[seg].arrive, 1u) == (uint32_t)p.nchunk[b] - 1);
+    for (int i = 0; i < kWarps; ++i) {
+      a += wsum[0][i];
+      e += wsum[1][i];
+    }
+    const uint32_t dst = mapa(smem_addr(&cnt[rank][0]), (uint32_t)tid);
+    dsm_st(dst, (uint32_t)a);
+    dsm_st(dst + 4u, (uint32_t)e);
+  }
+  ok = cluster_phase(barA, phase, &fail, p.status) && ok;
+  if (tid == 0) {
+    int a = 0, e = 0;
+    if (ok)
+      for (uint32_t r = 0; r < rank; ++r) {  // the lower ranks hold the lower positions
+        a += (int)cnt[r][0];
+        e += (int)cnt[r][1];
+      }
+    bcast[0] = a;
+    bcast[1] = e;
   }
   __syncthreads();
-  if (!last || threadIdx.x != 0) return;
-  __threadfence();
-  // exclusive prefixes over the segment's chunks, in position order
-  const int first = blk - c;
-  int a = 0, e = 0;
-  for (int i = 0; i < p.nchunk[b]; ++i) {
-    w.off[2 * (first + i)] = a;
-    w.off[2 * (first + i) + 1] = e;
-    a += __ldcg(&w.cnt[2 * (first + i)]);
-    e += __ldcg(&w.cnt[2 * (first + i) + 1]);
-  }
-}
 
-__global__ void __launch_bounds__(kThreads)
-k_sel_write(SelParams p, const float* __restrict__ scores, const void* ws,
-            int32_t* __restrict__ keep_idx, int32_t* __restrict__ evict_idx) {
-  __shared__ int32_t wsum[2][kThreads / 32];
-  Workspace w = carve(const_cast<void*>(ws), p);
-  int b, h, c;
-  locate(p, blockIdx.x, b, h, c);
-  const int seg = b * p.Hkv + h;
-  const SegState st = w.seg[seg];
-  const uint32_t T = st.prefix;
-  const int quota = st.done ? 0 : st.rem;  // keys == T that are evicted
-  const bool any = !st.done;
-  const int L = p.L[b];
-  const float* s = scores + (size_t)seg * p.n_max;
-  int32_t* kout = keep_idx + (size_t)seg * p.max_keep;
-  int32_t* eout = evict_idx + (size_t)seg * p.max_evict;
-  const int blk = blockIdx.x;
-  const int lt_before = w.off[2 * blk];
-  int eq_seen = w.off[2 * blk + 1];                      // keys == T before this point
-  int ev_seen = lt_before + min(eq_seen, quota);         // evicted before this point
-  const int beg = c * kChunk, end = min(L, beg + kChunk);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  for (int t0 = beg; t0 < end; t0 += kThreads) {
-    const int j = t0 + threadIdx.x;
-    const bool in = j < end;
-    uint32_t key = in ? key_of(s[j]) : 0xFFFFFFFFu;
-    const bool lt = in && any && key < T;
-    const bool eq = in && any && key == T;
-    // exclusive rank of eq among this tile's eq, in position order
-    const unsigned beq = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) wsum[1][wid] = __popc(beq);
-    __syncthreads();
-    int eq_rank = eq_seen + __popc(beq & ((1u << lane) - 1u));
-    int eq_tile = 0;
-    for (int i = 0; i < kThreads / 32; ++i) {
-      if (i < wid) eq_rank += wsum[1][i];
-      eq_tile += wsum[1][i];
-    }
-    const bool ev = in && (lt || (eq && eq_rank < quota));
-    const unsigned bev = __ballot_sync(0xffffffffu, ev);
-    if (lane == 0) wsum[0][wid] = __popc(bev);
-    __syncthreads();
-    int ev_rank = ev_seen + __popc(bev & ((1u << lane) - 1u));
-    int ev_tile = 0;
-    for (int i = 0; i < kThreads / 32; ++i) {
-      if (i < wid) ev_rank += wsum[0][i];
-      ev_tile += wsum[0][i];
-    }
-    if (in) {  // the guards only matter if the ranks were inconsistent
-      if (ev) {
-        if (ev_rank < p.max_evict) eout[ev_rank] = j;
-      } else if (j - ev_rank < p.max_keep) {
-        kout[j - ev_rank] = j;
+  // ---- order-preserving compaction of this CTA's range ----------------------
+  // Per sub-range: thread t owns keys [sub0 + 32 t, +32).  eq ranks come from
+  // a scan of the per-thread == T counts, evicted counts from a scan of
+  // (#< T + the == T keys within the quota); the sub-range's evicted positions
+  // are staged in shared memory first, its kept positions after them, and both
+  // lists are copied out coalesced (they are contiguous in the outputs).
+  if (ok) {
+    int32_t* kout = keep_idx + (size_t)seg * p.max_keep;
+    int32_t* eout = evict_idx + (size_t)seg * p.max_evict;
+    int eq_base = bcast[1];                           // keys == T before this sub-range
+    int ev_base = bcast[0] + min(eq_base, quota);     // evicted before this sub-range
+    const bool any = E > 0;
+    for (int sub0 = lo; sub0 < hi; sub0 += kSub) {
+      uint32_t k[kPer];
+      load_run(sub0, k);
+      const int j0 = sub0 + tid * kPer;
+      int lt = 0, eq = 0;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const bool in = any && j0 + u < hi;
+        lt += in && k[u] < T;
+        eq += in && k[u] == T;
       }
+      int eq_tot, ev_tot;
+      const int eq_before = eq_base + block_excl_scan(eq, eq_tot, warp_tot);
+      // evicted == T keys of this thread: those whose eq rank is below the quota
+      const int eq_ev = max(0, min(eq, quota - eq_before));
+      const int ev_before_local = block_excl_scan(lt + eq_ev, ev_tot, warp_tot);
+      const int n_sub = min(kSub, hi - sub0);
+      // stage: evicted at [0, ev_tot), kept at [ev_tot, n_sub) of the sub-range
+      __syncthreads();  // every thread has its keys in registers before the cache is reused
+      int ev_i = ev_before_local, eqr = eq_before;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int j = j0 + u;
+        if (j >= hi) break;
+        bool ev = false;
+        if (any) {
+          if (k[u] < T) ev = true;
+          else if (k[u] == T) ev = (eqr++ < quota);
+        }
+        if (ev) staging[ev_i++] = j;
+        else staging[ev_tot + (j - sub0) - ev_i] = j;
+      }
+      __syncthreads();
+      for (int i = tid; i < n_sub; i += kThreads) {
+        if (i < ev_tot) {
+          const int r = ev_base + i;
+          if (r < p.max_evict) eout[r] = staging[i];  // guards: only inconsistent ranks
+        } else {
+          const int r = (sub0 - ev_base) + (i - ev_tot);  // kept before + local kept rank
+          if (r < p.max_keep) kout[r] = staging[i];
+        }
+      }
+      __syncthreads();
+      eq_base += eq_tot;
+      ev_base += ev_tot;
     }
-    eq_seen += eq_tile;
-    ev_seen += ev_tile;
-    __syncthreads();
+    // slots past this row's own counts (rows shorter than the maxima): -1
+    if (rank == kC - 1) {
+      for (int i = L - E + tid; i < p.max_keep; i += kThreads) kout[i] = -1;
+      for (int i = E + tid; i < p.max_evict; i += kThreads) eout[i] = -1;
+    }
   }
+  // rank 0's histograms and every CTA's counters outlive every remote access
+  cluster_phase(barA, phase, &fail, p.status);
 }
 
 SelParams make_params(int B, int Hkv, int n_max, const int32_t* L, const int32_t* keep,
-                      int max_keep, int max_evict) {
+                      int max_keep, int max_evict, int32_t* status) {
   SelParams p;
   p.B = B;
   p.Hkv = Hkv;
   p.n_max = n_max;
   p.max_keep = max_keep;
   p.max_evict = max_evict;
-  p.chunk_base[0] = 0;
+  p.status = status;
   for (int b = 0; b < B; ++b) {
     p.L[b] = L[b];
     p.E[b] = L[b] - keep[b];
-    p.nchunk[b] = (L[b] + kChunk - 1) / kChunk;
-    if (p.nchunk[b] == 0) p.nchunk[b] = 1;  // an empty row still gets one (idle) CTA
-    p.chunk_base[b + 1] = p.chunk_base[b] + Hkv * p.nchunk[b];
   }
   return p;
 }
 
 }  // namespace
 
-size_t select_workspace_bytes(int B, int Hkv, int n_max) {
-  const size_t segs = (size_t)B * Hkv;
-  const size_t nchunk = (size_t)(n_max + kChunk - 1) / kChunk + 1;
-  return align_up(sizeof(SegState) * segs, 256) + align_up(sizeof(uint32_t) * kBins * segs, 256) +
-         2 * align_up(sizeof(int32_t) * 2 * segs * nchunk, 256);
-}
+// The select path keeps its state in shared memory; the workspace holds only
+// the device status word.
+size_t select_workspace_bytes(int, int, int) { return 256; }
 
-int select_launch_count() { return 6; }
+int select_launch_count() { return 1; }
 
-// L, keep: host arrays of B <= kMaxB rows.  Workspace carve-up depends only on
-// (B, Hkv, chunk counts), all of which are bounded by select_workspace_bytes.
+// L, keep: host arrays of B <= kMaxB rows.
 cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const int32_t* L,
                           const int32_t* keep, int32_t* keep_idx, int32_t max_keep,
                           int32_t* evict_idx, int32_t max_evict, void* ws, cudaStream_t st) {
-  const SelParams p = make_params(B, Hkv, n_max, L, keep, max_keep, max_evict);
-  const int chunks = p.chunk_base[B];
-  k_sel_init<<<148, 256, 0, st>>>(p, ws, keep_idx, evict_idx);
-  for (int r = 0; r < 3; ++r) k_sel_hist<<<chunks, kThreads, 0, st>>>(p, scores, ws, r);
-  k_sel_count<<<chunks, kThreads, 0, st>>>(p, scores, ws);
-  k_sel_write<<<chunks, kThreads, 0, st>>>(p, scores, ws, keep_idx, evict_idx);
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  SelParams p = make_params(B, Hkv, n_max, L, keep, max_keep, max_evict, status);
+  int max_L = 0;
+  for (int b = 0; b < B; ++b) max_L = L[b] > max_L ? L[b] : max_L;
+  const long long span = (((long long)max_L + kC - 1) / kC + 31) & ~31ll;
+  p.cache = span <= kSub ? 1 : 0;
+  // [key cache when it fits][staging][histogram copies]; the histogram copies
+  // always start at 2 * kSub words
+  const size_t smem = (2 * (size_t)kSub + kCopies * (size_t)kCopyStride) * sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(status, 0, sizeof(int32_t), st)) != cudaSuccess) return e;
+  k_select<<<B * Hkv * kC, kThreads, smem, st>>>(p, scores, keep_idx, evict_idx);
   return cudaGetLastError();
 }
 

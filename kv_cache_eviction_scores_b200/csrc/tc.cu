@@ -66,12 +66,13 @@ constexpr int kWarpTma = kSimtWarps, kWarpMma = kSimtWarps + 1, kWarpNv = kSimtW
 constexpr int kThreads2 = (kSimtWarps + 2) * 32;  // pass 2: + TMA warp, MMA warp
 constexpr int kThreads1 = (kSimtWarps + 3) * 32;  // pass 1: + the ||v||^2 warp
 constexpr int kMaxRegs = 96;       // 5 warps share a sub-partition's 16K registers
-constexpr uint32_t kColO = 256;    // pass-1 TMEM columns: S/P buffers [0, 256), O, Q
-constexpr uint32_t kColQ = 384;
+constexpr uint32_t kColO = 384;    // pass-1 TMEM columns: three S/P buffers [0, 384), then O
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kPartStride = 136;   // floats per partial row: O[128], m, l (4 parts), pad
 constexpr int kMaxCtas = 160;      // split target ceiling (one CTA per SM)
-constexpr int kSt1 = 3;            // pass-1 K and V stages (HBM latency needs > 1 tile in flight)
+constexpr int kSt1 = 3;            // pass-1 V stages (HBM latency needs > 1 tile in flight)
+constexpr int kStK = 2;            // pass-1 K stages (S runs two tiles ahead of P V)
+constexpr int kBars1 = 1 + 2 * kStK + 2 * kSt1 + 13;  // pass-1 mbarriers
 constexpr int kRing2 = 5;          // pass-2 ring of 32 KB K/V slots (the last one doubles as A_lo)
 constexpr float kLoSkip = 8e-4f;   // pass 2 drops A_lo when ||A||^2 <= kLoSkip ||v||^2 throughout
 
@@ -155,9 +156,9 @@ __device__ __forceinline__ float p1_exp32(const uint32_t (&sr)[32], uint32_t tS,
                                           float mu) {
   const uint64_t nmu2 = pk2(-mu, -mu);
   uint64_t l2 = pk2(0.f, 0.f);
+  uint32_t pw[32];  // columns: hi of tokens 0-15, lo of 0-15, hi of 16-31, lo of 16-31
 #pragma unroll
   for (int half = 0; half < 2; ++half) {  // 16 tokens -> 8 hi + 8 lo columns
-    uint32_t hi[8], lo[8];
 #pragma unroll
     for (int u2 = 0; u2 < 8; ++u2) {
       const int u = half * 16 + 2 * u2;
@@ -166,16 +167,15 @@ __device__ __forceinline__ float p1_exp32(const uint32_t (&sr)[32], uint32_t tS,
       const float e0 = ex2(d0), e1 = ex2(d1);
       const uint64_t E = pk2(e0, e1);
       l2 = fadd2(l2, E);
-      hi[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
+      pw[half * 16 + u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
       const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
       const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
       float r0, r1;
       upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
-      lo[u2] = pack_bf16_rn(r0, r1);
+      pw[half * 16 + 8 + u2] = pack_bf16_rn(r0, r1);
     }
-    tmem_st8(tS + half * 16, hi);
-    tmem_st8(tS + half * 16 + 8, lo);
   }
+  tmem_st32(tS, pw);  // one TMEM store for the warp's 32 columns
   float la, lb;
   upk2(l2, la, lb);
   return la + lb;
@@ -183,10 +183,12 @@ __device__ __forceinline__ float p1_exp32(const uint32_t (&sr)[32], uint32_t tS,
 
 // Rare path of pass 1, out of line: the reference max moved for some lanes
 // (factor fac <= 1 for them, 1 for the others), so this warp's 32 columns of O
-// are rescaled once the previous P V (the `prev`-th) has landed.
-// Warp-collective.  Returns false on a timeout.
-__device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, int prev, uint32_t od_bar) {
-  if (!warp_wait(od_bar, prev & 1)) return false;
+// are rescaled once the P V that last accumulated into O has landed (waited on
+// through that P V's buffer barrier and parity).  Warp-collective.  Returns
+// false on a timeout.
+__device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, uint32_t pd_bar,
+                                          uint32_t parity) {
+  if (!warp_wait(pd_bar, parity)) return false;
   tc_fence_after();
   uint32_t o[32];
   tmem_ld32(tO, o);
@@ -197,15 +199,16 @@ __device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, int prev, uint
 }
 
 __global__ void __maxnreg__(kMaxRegs)
-k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-           const TcArgs a) {
+k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* sK = smem;                     // kSt1 stages
-  uint8_t* sV = smem + kSt1 * kTileBytes;  // kSt1 stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kSt1 * kTileBytes);  // 22 barriers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint8_t* sQ = smem;                              // 128 rows x 2 boxes
+  uint8_t* sK = smem + kTileBytes;                 // kStK stages
+  uint8_t* sV = sK + kStK * kTileBytes;            // kSt1 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kSt1 * kTileBytes);  // kBars1 barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBars1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xmax = reinterpret_cast<float*>(tmem_slot + 2);  // [2 tile parities][4 groups][128]
+  float* xmax = reinterpret_cast<float*>(tmem_slot + 2);  // [3 buffers][4 groups][128]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1 KB alignment
     if (threadIdx.x == 0) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
@@ -215,28 +218,32 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
   decode_cta(a, blockIdx.x, b, h, chunk, t0, t1);
   const int T = t1 - t0;
   const int L = a.L[b];
-  auto KF = [&](int s) { return smem_u32(&bars[s]); };       // kSt1 each: K full / empty,
-  auto KE = [&](int s) { return smem_u32(&bars[3 + s]); };   // V full / empty
-  auto VF = [&](int s) { return smem_u32(&bars[6 + s]); };
-  auto VE = [&](int s) { return smem_u32(&bars[9 + s]); };
-  auto SF = [&](int b) { return smem_u32(&bars[12 + b]); };  // 2 TMEM buffers: S ready,
-  auto PF = [&](int b) { return smem_u32(&bars[14 + b]); };  // P written,
-  auto XB = [&](int b) { return smem_u32(&bars[16 + b]); };  // tile-max exchange
-  const uint32_t OD = smem_u32(&bars[18]);                     // P V into O done
-  auto PD = [&](int b) { return smem_u32(&bars[19 + b]); };  // P V of a buffer done
-  // O final: committed once, after the last P V.  (OD's parity alone cannot
-  // tell the last P V from the one before it once the loop has ended.)
-  const uint32_t OF = smem_u32(&bars[21]);
+  // barriers: Q; K full/empty (kStK stages); V full/empty (kSt1 stages); per
+  // TMEM S/P buffer: S ready, P written, tile max exchanged, P V done; O final
+  const uint32_t BQ = smem_u32(&bars[0]);
+  auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto KE = [&](int s) { return smem_u32(&bars[1 + kStK + s]); };
+  auto VF = [&](int s) { return smem_u32(&bars[1 + 2 * kStK + s]); };
+  auto VE = [&](int s) { return smem_u32(&bars[1 + 2 * kStK + kSt1 + s]); };
+  constexpr int kB0 = 1 + 2 * kStK + 2 * kSt1;
+  auto SF = [&](int s) { return smem_u32(&bars[kB0 + s]); };
+  auto PF = [&](int s) { return smem_u32(&bars[kB0 + 3 + s]); };
+  auto XB = [&](int s) { return smem_u32(&bars[kB0 + 6 + s]); };
+  auto PD = [&](int s) { return smem_u32(&bars[kB0 + 9 + s]); };
+  const uint32_t OF = smem_u32(&bars[kB0 + 12]);  // committed once, after the last P V
   if (threadIdx.x == 0) {
-    mbar_init(OD, 1);
+    mbar_init(BQ, 1);
     mbar_init(OF, 1);
+    for (int s = 0; s < kStK; ++s) {
+      mbar_init(KF(s), 1); mbar_init(KE(s), 1);
+    }
     for (int s = 0; s < kSt1; ++s) {
-      mbar_init(KF(s), 1); mbar_init(KE(s), 1); mbar_init(VF(s), 1);
+      mbar_init(VF(s), 1);
       mbar_init(VE(s), 2);  // P V commit + the ||v||^2 warp's reads
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(SF(b), 1); mbar_init(PF(b), kSimtWarps); mbar_init(XB(b), kSimtWarps);
-      mbar_init(PD(b), 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(SF(s), 1); mbar_init(PF(s), kSimtWarps); mbar_init(XB(s), kSimtWarps);
+      mbar_init(PD(s), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -251,74 +258,58 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
   const uint32_t tbase = *tmem_slot;
   const int z = b * a.Hkv + h;
   const int qrow0 = (b * a.Hkv + h) * a.G * a.w + chunk * a.nqc;
-  if (warp < kSimtWarps) {
-    // Q of the chunk into TMEM columns [kColQ, kColQ + 64): row r of the chunk
-    // in lane r, head-dim pair (2c, 2c+1) in column c (the A operand of S = Q K^T);
-    // rows past the chunk are zero.  Warp (g, quarter) moves head dims [32g, 32g+32).
-    const int g = warp >> 2, ql = warp & 3, r = ql * 32 + lane;
-    uint32_t wq[16];
-    if (r < a.nqc) {
-      const uint4* src =
-          reinterpret_cast<const uint4*>(a.q + ((size_t)qrow0 + r) * kHd + g * 32);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 x = src[i];
-        wq[4 * i] = x.x; wq[4 * i + 1] = x.y; wq[4 * i + 2] = x.z; wq[4 * i + 3] = x.w;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) wq[i] = 0u;
-    }
-    tmem_st16(tbase + kColQ + (uint32_t)(g * 16) + ((uint32_t)(ql * 32) << 16), wq);
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
 
   if (warp == kWarpTma) {
     // ---------------- TMA producer ----------------
+    // order: Q, K_0, K_1, then K_{j+2} and V_j for each tile j (S runs two
+    // tiles ahead of P V)
     if (lane == 0) {
-      prefetch_tmap(&tmK); prefetch_tmap(&tmV);
-      auto load = [&](uint8_t* buf, uint32_t full, uint32_t empty, const CUtensorMap* m, int i) {
-        const int s = i % kSt1, ph = (i / kSt1) & 1;
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
+      mbar_expect_tx(BQ, 2u * 128u * (uint32_t)a.qbox_rows);
+      tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
+      tma_load_2d(smem_u32(sQ) + kBox, &tmQ, BQ, 64, qrow0);
+      auto load = [&](uint8_t* buf, int nst, const CUtensorMap* m, int i, uint32_t full,
+                      uint32_t empty) {
+        const int ph = (i / nst) & 1;
         if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); return false; }
         mbar_expect_tx(full, kTileBytes);
-        const uint32_t dst = smem_u32(buf + s * kTileBytes);
+        const uint32_t dst = smem_u32(buf + (i % nst) * kTileBytes);
         tma_load_3d(dst, m, full, 0, (t0 + i) * kTok, z);
         tma_load_3d(dst + kBox, m, full, 64, (t0 + i) * kTok, z);
         return true;
       };
-      bool ok = T > 0 ? load(sK, KF(0), KE(0), &tmK, 0) : true;
+      bool ok = true;
+      for (int i = 0; i < 2 && i < T && ok; ++i)
+        ok = load(sK, kStK, &tmK, i, KF(i % kStK), KE(i % kStK));
       for (int j = 0; j < T && ok && !*abort_flag; ++j) {
-        if (j + 1 < T) ok = load(sK, KF((j + 1) % kSt1), KE((j + 1) % kSt1), &tmK, j + 1);
-        if (ok) ok = load(sV, VF(j % kSt1), VE(j % kSt1), &tmV, j);
+        if (j + 2 < T) ok = load(sK, kStK, &tmK, j + 2, KF((j + 2) % kStK), KE((j + 2) % kStK));
+        if (ok) ok = load(sV, kSt1, &tmV, j, VF(j % kSt1), VE(j % kSt1));
       }
     }
   } else if (warp == kWarpMma) {
     // ---------------- MMA issuer ----------------
-    constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T (Q from TMEM)
+    constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T
     constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);    // O += P V (V MN-major)
-    bool ok = true;
+    bool ok = warp_wait(BQ, 0);
+    if (!ok) fail(a, abort_flag);
     // operand descriptors of stage 0; a stage or K slice only moves the start
-    // address, i.e. adds to the low word (few instructions per MMA: this warp
-    // shares its issue slots with four softmax warps)
+    // address, i.e. adds to the low word
+    const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024);
     const SDesc kd0 = sdesc_split(smem_u32(sK), 16, 1024);
     const SDesc vd0 = sdesc_split(smem_u32(sV), kBox, 1024);
-    const uint32_t tq = tbase + kColQ;
     auto issue_S = [&](int i) {
-      const int s = i % kSt1, ph = (i / kSt1) & 1, bf = i & 1;
+      const int s = i % kStK, ph = (i / kStK) & 1, bf = i % 3;
       if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
-      // S(i) overwrites the buffer whose P the (i-2)-th P V reads from TMEM:
-      // wait until that P V has completed
-      if (i >= 2 && !warp_wait(PD(bf), ((i - 2) >> 1) & 1)) { fail(a, abort_flag); return false; }
+      // S(i) overwrites the buffer whose P the (i-3)-th P V reads from TMEM
+      if (i >= 3 && !warp_wait(PD(bf), ((i - 3) / 3) & 1)) { fail(a, abort_flag); return false; }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t klo = kd0.lo + (uint32_t)s * (kTileBytes >> 4);
         const uint32_t dS = tbase + (uint32_t)(bf * 128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts_w(dS, tq + (uint32_t)(8 * kk), klo + kslice(kk, 128), kd0.hi, IDS, kk > 0 ? 1u : 0u);
+          mma_ss_w(dS, qd.lo + kslice(kk, 128), qd.hi, klo + kslice(kk, 128), kd0.hi, IDS,
+                   kk > 0 ? 1u : 0u);
         mma_commit(KE(s));
         mma_commit(SF(bf));
       }
@@ -326,7 +317,7 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
       return true;
     };
     auto issue_PV = [&](int i) {
-      const int s = i % kSt1, ph = (i / kSt1) & 1, bf = i & 1, bph = (i >> 1) & 1;
+      const int s = i % kSt1, ph = (i / kSt1) & 1, bf = i % 3, bph = (i / 3) & 1;
       if (!warp_wait(PF(bf), bph)) { fail(a, abort_flag); return false; }
       if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
       uint8_t* vb = sV + s * kTileBytes;
@@ -358,16 +349,18 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         for (int kk = 0; kk < 8; ++kk)
           mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
         mma_commit(VE(s));
-        mma_commit(OD);
         mma_commit(PD(bf));
         if (i == T - 1) mma_commit(OF);
       }
       __syncwarp();
       return true;
     };
-    if (ok && T > 0) ok = issue_S(0);
+    // tensor-pipe order: S(0), S(1), then S(j + 2), P V(j) for each j.  S(j + 2)
+    // needs only P V(j - 1) done (its buffer) and goes ahead of P V(j), which
+    // waits for the softmax warps, so S is ready when they reach tile j + 2.
+    for (int i = 0; i < 2 && i < T && ok; ++i) ok = issue_S(i);
     for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
-      if (j + 1 < T) ok = issue_S(j + 1);
+      if (j + 2 < T) ok = issue_S(j + 2);
       if (ok) ok = issue_PV(j);
     }
   } else if (warp == kWarpNv) {
@@ -415,8 +408,10 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     // ---------------- softmax warps ----------------
     // Sixteen warps work on every tile: warp (g, quarter) owns the query rows
     // [32 quarter, +32) (its TMEM lanes), the tile's tokens [32 g, 32 g + 32)
-    // (its S/P columns) and O's head-dim columns [32 g, 32 g + 32); the four
-    // warps of a row exchange their tile max through shared memory.
+    // (its S/P columns) and O's head-dim columns [32 g, 32 g + 32).
+    // Software pipelined by one tile: step j posts tile j's max for the other
+    // three warps of its rows, then writes P of tile j - 1, whose maxes were
+    // posted a full step earlier, so the exchange rarely waits.
     const int g = warp >> 2, ql = warp & 3;
     const int row = ql * 32 + lane;  // query row within the chunk
     const bool valid_row = row < a.nqc;
@@ -427,52 +422,69 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
     float m_ref = -INFINITY, l = 0.f;
-    for (int j = 0; j < T; ++j) {
-      const int s = j & 1, ph = (j >> 1) & 1;  // TMEM buffer and its phase
-      if (!warp_wait(SF(s), ph)) { fail(a, abort_flag); break; }
-      if (warp_aborted(abort_flag)) break;
-      tc_fence_after();
-      const uint32_t tS = tbase + (uint32_t)(s * 128) + lane_off + (uint32_t)c0;
-      const int tok0 = (t0 + j) * kTok + c0;
+    for (int j = 0; j <= T; ++j) {
       uint32_t sr[32];
-      tmem_ld32(tS, sr);
-      if (tok0 + 31 > L - a.w) {  // only the last tiles: hide keys past P_t
+      if (j < T) {
+        // ---- tile j: row max of this warp's 32 keys, posted to the exchange
+        const int bf = j % 3;
+        if (!warp_wait(SF(bf), (j / 3) & 1)) { fail(a, abort_flag); break; }
+        if (warp_aborted(abort_flag)) break;
+        tc_fence_after();
+        const int tok0 = (t0 + j) * kTok + c0;
+        tmem_ld32(tbase + (uint32_t)(bf * 128) + lane_off + (uint32_t)c0, sr);
+        if (tok0 + 31 > L - a.w) {  // only the last tiles: hide keys past P_t
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
-          if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
-      }
-      float ya = -INFINITY, yb = -INFINITY;
+          for (int u = 0; u < 32; ++u)
+            if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
+        }
+        float ya = -INFINITY, yb = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 32; u += 4) {
-        ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
-        yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
+        for (int u = 0; u < 32; u += 4) {
+          ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
+          yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
+        }
+        xmax[bf * 512 + g * 128 + row] = fmaxf(ya, yb) * c;  // c > 0: commutes with the max
+        __syncwarp();
+        if (lane == 0) mbar_arrive(XB(bf));
       }
-      // the reference max moves only when a tile exceeds it by more than 8
-      // (so 2^(S c - m) <= 256); then l and O are rescaled
-      float* xm = xmax + s * 512;
-      xm[g * 128 + row] = fmaxf(ya, yb) * c;  // c > 0: the max commutes with the scaling
-      __syncwarp();
-      if (lane == 0) mbar_arrive(XB(s));
-      if (!warp_wait(XB(s), ph)) { fail(a, abort_flag); break; }
-      const float mt = fmaxf(fmaxf(xm[row], xm[128 + row]), fmaxf(xm[256 + row], xm[384 + row]));
-      float fac = 1.f;
-      bool resc = false;
-      if (mt > m_ref + 8.f) {
-        if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
-        resc = m_ref != -INFINITY && j > 0;
-        m_ref = mt;
-        l *= fac;
+      if (j >= 1) {
+        // ---- tile i = j - 1: the row's reference, then P = 2^(S c - m) over S
+        const int i = j - 1, bf = i % 3;
+        if (!warp_wait(XB(bf), (i / 3) & 1)) { fail(a, abort_flag); break; }
+        const float* xm = xmax + bf * 512;
+        const float mt = fmaxf(fmaxf(xm[row], xm[128 + row]), fmaxf(xm[256 + row], xm[384 + row]));
+        // the reference max moves only when a tile exceeds it by more than 8
+        // (so 2^(S c - m) <= 256); then l and O are rescaled
+        float fac = 1.f;
+        bool resc = false;
+        if (mt > m_ref + 8.f) {
+          if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
+          resc = m_ref != -INFINITY && i > 0;
+          m_ref = mt;
+          l *= fac;
+        }
+        // warp-uniform: every lane votes, and all or none call the rescale; O
+        // holds P V up to tile i - 1, which has landed once PD of its buffer
+        // completes that tile's phase
+        if (__any_sync(0xffffffffu, resc) &&
+            !p1_rescale_o(tO, fac, PD((i - 1) % 3), (uint32_t)(((i - 1) / 3) & 1))) {
+          fail(a, abort_flag);
+          break;
+        }
+        const uint32_t tS = tbase + (uint32_t)(bf * 128) + lane_off + (uint32_t)c0;
+        const int tok0 = (t0 + i) * kTok + c0;
+        tmem_ld32(tS, sr);
+        if (tok0 + 31 > L - a.w) {
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            if (tok0 + u > Prow) sr[u] = 0xFF800000u;
+        }
+        l += p1_exp32(sr, tS, c2, m_ref == -INFINITY ? 0.f : m_ref);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(PF(bf));
       }
-      // warp-uniform: every lane votes, and all or none call the rescale
-      if (__any_sync(0xffffffffu, resc) && !p1_rescale_o(tO, fac, j - 1, OD)) {
-        fail(a, abort_flag);
-        break;
-      }
-      l += p1_exp32(sr, tS, c2, m_ref == -INFINITY ? 0.f : m_ref);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(PF(s));
     }
     // partial row: this warp's 32 columns of O, the shared max, its normaliser part
     float* out = a.partial + ((size_t)blockIdx.x * 128 + row) * kPartStride;
@@ -520,21 +532,39 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
   const int cta0 = a.cta_base[b] + (h * a.chunks + chunk) * a.splits[b];
   const int np = a.splits[b];
   auto P = [&](int i) { return a.partial + ((size_t)(cta0 + i) * 128 + rr) * kPartStride; };
+  // lanes take the partials' (max, normaliser) in parallel: M, then the
+  // weights 2^(m_i - M) and L = sum_i w_i l_i
   float M = -INFINITY;
   for (int i = lane; i < np; i += 32) M = fmaxf(M, P(i)[128]);
   M = warp_max(M);
-  float Lsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i = 0; i < np; ++i) {
+  float lpart = 0.f;
+  for (int i = lane; i < np; i += 32) {
     const float* p = P(i);
     const float mi = p[128];
     const float wgt = (mi == -INFINITY) ? 0.f : ex2(mi - M);
-    Lsum += wgt * ((p[129] + p[130]) + (p[131] + p[132]));  // the four normaliser parts
-    const float4 o = *reinterpret_cast<const float4*>(p + lane * 4);
-    acc.x = fmaf(wgt, o.x, acc.x);
-    acc.y = fmaf(wgt, o.y, acc.y);
-    acc.z = fmaf(wgt, o.z, acc.z);
-    acc.w = fmaf(wgt, o.w, acc.w);
+    lpart = fmaf(wgt, (p[129] + p[130]) + (p[131] + p[132]), lpart);  // four normaliser parts
+  }
+  const float Lsum = warp_sum(lpart);
+  // O = sum_i w_i O_i, four partial rows in flight per step
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < np; i0 += 4) {
+    float4 o[4];
+    float wg[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = min(i0 + k, np - 1);
+      const float* p = P(i);
+      o[k] = *reinterpret_cast<const float4*>(p + lane * 4);
+      const float mi = p[128];
+      wg[k] = (i0 + k >= np || mi == -INFINITY) ? 0.f : ex2(mi - M);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc.x = fmaf(wg[k], o[k].x, acc.x);
+      acc.y = fmaf(wg[k], o[k].y, acc.y);
+      acc.z = fmaf(wg[k], o[k].z, acc.z);
+      acc.w = fmaf(wg[k], o[k].w, acc.w);
+    }
   }
   const float inv = 1.f / Lsum;
   const float A[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
@@ -586,9 +616,11 @@ __device__ __noinline__ float direct_sqdist(const float* A, const __nv_bfloat16*
   return s;
 }
 
-// Fast path for 16 query columns of one token (no dominant token, no
-// possible cancellation, every key visible): packed fp32 pairs,
-//   p = 2^(x c - M'),  M' = M + log2 L,   ratio = p + p^2 + p^3,
+// Fast path for 16 query columns of one token (every p < 2^-4, no possible
+// cancellation, every key visible): packed fp32 pairs,
+//   p = 2^(x c - M'),  M' = M + log2 L,
+//   ratio = p / (1 - p) = p (1 + p (1 + p (1 + p (1 + p)))) + O(p^6)
+//   (relative truncation error p^5 / (1 - p) <= 1.0e-6 for p < 2^-4),
 //   s += ratio^2 (D' + ||A||^2 + ||v||^2)   with D' = -2 A.v from the MMA.
 // kf holds (-M'_t, -M'_t+1, ||A_t||^2, ||A_t+1||^2) per column pair.
 __device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf, uint64_t c2,
@@ -601,7 +633,8 @@ __device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf
     const float p0 = ex2(y0), p1 = ex2(y1);
     pmax = fmax3(pmax, p0, p1);
     const uint64_t P = pk2(p0, p1);
-    const uint64_t ratio = ffma2(P, ffma2(P, P, P), P);
+    const uint64_t one = pk2(1.f, 1.f);
+    const uint64_t ratio = fmul2(P, ffma2(P, ffma2(P, ffma2(P, fadd2(P, one), one), one), one));
     const uint64_t zt = fadd2(fadd2(pk2(f32(r[16 + 2 * i]), f32(r[16 + 2 * i + 1])),
                                     pk2(k.z, k.w)), nv2);
     acc2 = ffma2(fmul2(ratio, ratio), zt, acc2);
@@ -834,8 +867,9 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           uint64_t a2 = pk2(0.f, 0.f);
           float pmax = 0.f;
           fast16(r, kf + ch * 8, c2, nv2, a2, pmax);
-          // dominant token (p >= 2^-8) or possible cancellation (||A||^2 >= 0.6 ||v||^2)
-          const bool redo = pmax >= 0.00390625f || nAmax[ch] >= 0.6f * nv;
+          // a large p (>= 2^-4: the series above would be short) or possible
+          // cancellation (||A||^2 >= 0.6 ||v||^2): the careful path
+          const bool redo = pmax >= 0.0625f || nAmax[ch] >= 0.6f * nv;
           if (__any_sync(0xffffffffu, redo)) {
             acc += careful16(tS, tD, ch * 16, tok, false, L, a.w, chunk * nqc, qrows, c, nv,
                              arows, vrow_g, &sing);
@@ -902,7 +936,7 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
 }
 
 size_t pass1_smem() {
-  return 2 * kSt1 * (size_t)kTileBytes + 22 * 8 + 8 + 2 * 4 * 128 * 4;
+  return (1 + kStK + kSt1) * (size_t)kTileBytes + kBars1 * 8 + 8 + 3 * 4 * 128 * 4;
 }
 size_t pass2_smem(int nqc) {
   return kRing2 * (size_t)kTileBytes + 2 * (size_t)nqc * 256 + (size_t)nqc / 2 * 16 + 8 * 4 +
@@ -1004,7 +1038,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   if (e != cudaSuccess) return e;
 
   kev.begin(st);
-  k_tc_pass1<<<ctas, kThreads1, sm1, st>>>(mK, mV, a);
+  k_tc_pass1<<<ctas, kThreads1, sm1, st>>>(mQ1, mK, mV, a);
   kev.end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kev.begin(st);

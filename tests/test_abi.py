@@ -66,7 +66,7 @@ def test_workspace_sizes():
     assert dk.scores_workspace_bytes(_shape(Hq=30)) == 0
     assert dk.scores_workspace_bytes(_shape(d=300)) == 0
     assert dk.scores_workspace_bytes(_shape(window=4096)) == 0
-    assert dk.select_workspace_bytes(1, 8, 131072) > 8 * 2048 * 4
+    assert dk.select_workspace_bytes(1, 8, 131072) >= 4  # the device status word
     assert dk.select_workspace_bytes(0, 8, 10) == 0
 
 

@@ -3,10 +3,10 @@
 Callers such as a serving engine that owns every byte of device memory through
 its own pool (or a path that cannot afford cudaMalloc's implicit device
 synchronisation) cannot hand dropkv_select a workspace.  dropkv_select_noalloc
-takes none and uses a 1 MiB scratch array compiled into the library.  This
+takes none and uses a 4 KiB scratch array compiled into the library.  This
 test calls it through the C ABI twice in a row and checks that both calls give
-exactly the keep / evict lists of dropkv_select (integer outputs: exact), and
-that sizes beyond the scratch are refused before anything runs.
+exactly the keep / evict lists of dropkv_select (integer outputs: exact), also
+for a launch of more than 64 batch rows (sliced on the host).
 
 The file is named so that pytest collects it last.
 """
@@ -68,16 +68,21 @@ def test_noalloc_select_matches_select_on_two_calls_in_a_row():
         assert torch.equal(ev_idx, ref_ev), f"call {call}: evict lists differ"
 
 
-def test_noalloc_select_refuses_sizes_beyond_its_scratch():
+def test_noalloc_select_many_rows_matches_select():
     L = _bind()
-    B, Hkv, n_max = 64, 4, 64  # 256 segments: the histograms alone need 2 MiB
-    assert dk.select_workspace_bytes(B, Hkv, n_max) > (1 << 20)
-    lengths = [n_max] * B
-    keep = [n_max // 2] * B
-    scores = _scores(B, Hkv, n_max, lengths, 3)  # real buffers of the declared sizes
-    keep_idx = torch.empty(B, Hkv, n_max // 2, dtype=torch.int32, device=DEV)
-    ev_idx = torch.empty(B, Hkv, n_max // 2, dtype=torch.int32, device=DEV)
+    B, Hkv, n_max = 70, 4, 300  # more than 64 rows: two host-side slices
+    rng = np.random.default_rng(5)
+    lengths = [int(x) for x in rng.integers(1, n_max + 1, size=B)]
+    keep = [int(rng.integers(0, Lb + 1)) for Lb in lengths]
+    scores = _scores(B, Hkv, n_max, lengths, 3)
+    ref_keep, ref_ev = dk.dropkv_select(scores, keep, lengths)
+    torch.cuda.synchronize()
+    max_keep, max_evict = ref_keep.shape[2], ref_ev.shape[2]
+    keep_idx = torch.full((B, Hkv, max_keep), 7, dtype=torch.int32, device=DEV)
+    ev_idx = torch.full((B, Hkv, max_evict), 7, dtype=torch.int32, device=DEV)
     st = L.dropkv_select_noalloc(B, Hkv, n_max, ctypes.c_void_p(scores.data_ptr()), _arr(lengths),
-                                 _arr(keep), ctypes.c_void_p(keep_idx.data_ptr()), n_max // 2,
-                                 ctypes.c_void_p(ev_idx.data_ptr()), n_max // 2, None)
-    assert st == dk.ERR_WORKSPACE
+                                 _arr(keep), ctypes.c_void_p(keep_idx.data_ptr()), max_keep,
+                                 ctypes.c_void_p(ev_idx.data_ptr()), max_evict, None)
+    assert st == dk.OK
+    torch.cuda.synchronize()
+    assert torch.equal(keep_idx, ref_keep) and torch.equal(ev_idx, ref_ev)
