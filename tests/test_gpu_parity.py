@@ -180,17 +180,24 @@ def test_nonsingular_async_status_is_ok():
 
 # ---- selection on constructed scores (ties, +inf, NaN padding) --------------
 
-@pytest.mark.parametrize("case", ["ties", "keep_all", "evict_all", "long"])
+@pytest.mark.parametrize("case", ["ties", "keep_all", "evict_all", "long", "huge", "nan_in_range"])
 def test_select_exact_on_constructed_scores(case):
     rng = np.random.default_rng(3)
     if case == "long":
         B, Hkv, n_max, lengths = 2, 3, 20000, [20000, 13001]
+    elif case == "huge":
+        # per-CTA ranges of 37500 keys: past the shared-memory key cache, three
+        # sub-ranges per CTA read from global memory
+        B, Hkv, n_max, lengths = 2, 2, 300000, [300000, 140001]
     else:
         B, Hkv, n_max, lengths = 3, 2, 5000, [5000, 4097, 1]
     s = rng.integers(0, 50, size=(B, Hkv, n_max)).astype(np.float32) / 8.0
     for b, L in enumerate(lengths):
         s[b, :, max(0, L - 3): L] = np.inf
         s[b, :, L:] = np.nan
+    if case == "nan_in_range":  # NaN scores inside [0, L) order above +inf
+        s[0, :, 17:40] = np.nan
+        s[1, 1, :100] = np.nan
     if case == "keep_all":
         keep = list(lengths)
     elif case == "evict_all":
