@@ -1,0 +1,107 @@
+"""Joint-removal objective on tiny inputs: DropKV's evicted set against the
+brute-force optimum (CPU only).
+
+The write-up ("DropKV：精确单项输出扰动评分组件", sections 核心公式 and
+结果与独立对照) scores every token by the exact output change its removal
+alone causes, and evicts the lowest-scoring ones.  The joint objective of an
+evicted set S is J(S) = sum over the KV head's window queries t of
+||a_S^(t) - a^(t)||^2, where a_S is the attention output with every token of S
+deleted.  Here:
+
+* J(S) is computed by actually deleting the tokens and re-softmaxing (numpy,
+  fp64), and the closed form a_S = (a - sum_{j in S} p_j v_j) / (1 - sum_{j in S} p_j)
+  is pinned against it;
+* for |S| = 1 and pool kernel 1 the DropKV score of token j is J({j}) / G, so
+  the oracle's eviction must be the brute-force optimum (exact pin);
+* for |S| = 2, 3 the ratio J(S_dropkv) / min_S J(S) is >= 1; the pages quote a
+  median ratio on real models, which synthetic inputs do not reproduce, so
+  the ratio itself is only reported.
+"""
+
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+
+G, HKV, D, L, W = 2, 1, 4, 11, 2          # history tokens [0, L - W) are evictable
+HIST = L - W
+
+
+def _inputs(seed):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, G * HKV, W, D))
+    k = rng.standard_normal((1, HKV, L, D)) * 1.3
+    v = rng.standard_normal((1, HKV, L, D))
+    return q, k, v
+
+
+def _softmax_out(qt, K, V):
+    x = K @ qt / np.sqrt(qt.shape[0])
+    e = np.exp(x - x.max())
+    return (e / e.sum()) @ V, e / e.sum()
+
+
+def joint_objective(q, k, v, S):
+    """J(S) by deletion: sum over the group's window queries of ||a_S - a||^2."""
+    keep = np.ones(L, dtype=bool)
+    keep[list(S)] = False
+    total = 0.0
+    for hq in range(G * HKV):
+        for t in range(W):
+            P = L - W + t  # causal limit of window query t (tail-aligned)
+            K, V = k[0, 0, : P + 1], v[0, 0, : P + 1]
+            a, _ = _softmax_out(q[0, hq, t], K, V)
+            a_s, _ = _softmax_out(q[0, hq, t], K[keep[: P + 1]], V[keep[: P + 1]])
+            total += float(np.sum((a_s - a) ** 2))
+    return total
+
+
+def dropkv_evicted(q, k, v, n_evict):
+    s = oracle.scores(q, k, v, [L], W, 1)
+    _, ev = oracle.select(s, [L], [L - n_evict])
+    return tuple(int(j) for j in ev[0, 0])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_closed_form_joint_removal_matches_deletion(seed):
+    q, k, v = _inputs(seed)
+    rng = np.random.default_rng(100 + seed)
+    S = sorted(rng.choice(HIST, size=3, replace=False).tolist())
+    for hq in range(G):
+        for t in range(W):
+            P = L - W + t
+            K, V = k[0, 0, : P + 1], v[0, 0, : P + 1]
+            a, p = _softmax_out(q[0, hq, t], K, V)
+            mass = p[S].sum()
+            closed = (a - p[S] @ V[S]) / (1.0 - mass)
+            keep = np.ones(P + 1, dtype=bool)
+            keep[S] = False
+            direct, _ = _softmax_out(q[0, hq, t], K[keep], V[keep])
+            np.testing.assert_allclose(closed, direct, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_single_eviction_is_the_brute_force_optimum(seed):
+    q, k, v = _inputs(seed)
+    J = np.array([joint_objective(q, k, v, (j,)) for j in range(HIST)])
+    # the DropKV score of a history token is J({j}) / G (pool 1, one KV head)
+    s = oracle.scores(q, k, v, [L], W, 1)
+    np.testing.assert_allclose(s[0, 0, :HIST], J / G, rtol=1e-10)
+    assert dropkv_evicted(q, k, v, 1) == (int(np.argmin(J)),)
+
+
+@pytest.mark.parametrize("n_evict", [2, 3])
+def test_multi_eviction_ratio_against_brute_force(n_evict):
+    ratios = []
+    for seed in range(6):
+        q, k, v = _inputs(seed)
+        S = dropkv_evicted(q, k, v, n_evict)
+        assert len(S) == n_evict and all(j < HIST for j in S)  # the window is never evicted
+        J_drop = joint_objective(q, k, v, S)
+        J_opt = min(joint_objective(q, k, v, c) for c in itertools.combinations(range(HIST), n_evict))
+        assert J_drop >= J_opt * (1 - 1e-12)
+        ratios.append(J_drop / J_opt)
+    print(f"|S| = {n_evict}: J(DropKV) / J(optimum) over 6 seeds: "
+          f"median {np.median(ratios):.3f}, max {max(ratios):.3f}")
