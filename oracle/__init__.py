@@ -49,6 +49,8 @@ def lib():
         L.oracle_scores_at.restype = i
         L.oracle_select.argtypes = [i, i, i, dp, ip, ip, i, i, ip, ip]
         L.oracle_select.restype = i
+        L.oracle_attn_raw.argtypes = [i, i, i, i, i, i, dp, dp, ip, dp]
+        L.oracle_attn_raw.restype = i
         _lib = L
     return _lib
 
@@ -141,6 +143,31 @@ def scores(q, k, v, lengths, window, pool, *, raise_singular=True, intermediates
     if intermediates:
         return out, merged, raw, st
     return out
+
+
+def attn_raw(q, k, lengths):
+    """Attention-only raw score per query head: sum over the window queries of
+    the attention probability each token receives (NaN padding)."""
+    q, k = _f64(q), _f64(k)
+    B, Hq, w, d = q.shape
+    _, Hkv, n_max, _ = k.shape
+    lens = _i32(lengths)
+    raw = np.empty((B, Hq, n_max))
+    st = lib().oracle_attn_raw(B, Hq, Hkv, n_max, d, w, _p(q, ctypes.c_double),
+                               _p(k, ctypes.c_double), _p(lens, ctypes.c_int32),
+                               _p(raw, ctypes.c_double))
+    if st == ERR_ARG:
+        raise ValueError("oracle: bad shape or lengths")
+    return raw
+
+
+def attn_scores(q, k, lengths, window, pool):
+    """Final attention-only scores [B, Hkv, n_max]: merged, pooled, window = +inf."""
+    q = _f64(q)
+    if q.shape[2] != window:
+        raise ValueError("q must hold exactly the window rows")
+    Hkv = np.asarray(k).shape[1]
+    return pool_protect(merge(attn_raw(q, k, lengths), Hkv, lengths), window, pool, lengths)
 
 
 def scores_at(Qg, K, V, window, pool, positions: Sequence[int]):

@@ -155,6 +155,49 @@ int oracle_raw_scores(int B, int Hq, int Hkv, int n_max, int d, int w, const dou
   return status;
 }
 
+/*
+ * Attention-only score, the negative control of the write-up
+ * "DropKV：精确单项输出扰动评分组件", section 结果与独立对照: the pages name an
+ * "attention-only" control beside the perturbation score without defining
+ * it; the reading taken here is the plainest one, the attention mass each
+ * token receives from the window queries,
+ *     raw[b, hq, j] = sum over window queries t with j <= P_t of p_j^(t),
+ * passed through the same merge / pool / protect / select as the perturbation
+ * score.  Nothing is singular here.  Padding positions are NaN.
+ */
+int oracle_attn_raw(int B, int Hq, int Hkv, int n_max, int d, int w, const double* q,
+                    const double* k, const int32_t* lengths, double* raw) {
+  if (check_shape(B, Hq, Hkv, n_max, d, w, 1, lengths)) return ORACLE_ERR_ARG;
+  const int G = Hq / Hkv;
+
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int bh = 0; bh < B * Hq; ++bh) {
+    const int b = bh / Hq, hq = bh % Hq, h = hq / G;
+    const int L = lengths[b];
+    const double* K = k + ((size_t)b * Hkv + h) * n_max * d;
+    double* s = raw + ((size_t)b * Hq + hq) * n_max;
+    double* x = malloc(sizeof(double) * L);
+    for (int j = 0; j < n_max; ++j) s[j] = (j < L) ? 0.0 : NAN;
+    for (int t = 0; t < w; ++t) {
+      const int P = L - w + t; /* causal tail alignment */
+      const double* qt = q + (((size_t)b * Hq + hq) * w + t) * d;
+      /* p = softmax over keys 0..P of q.k / sqrt(d) */
+      double m = -INFINITY;
+      for (int j = 0; j <= P; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += qt[c] * K[(size_t)j * d + c];
+        x[j] = dot / sqrt((double)d);
+        if (x[j] > m) m = x[j];
+      }
+      double l = 0.0;
+      for (int j = 0; j <= P; ++j) l += exp(x[j] - m);
+      for (int j = 0; j <= P; ++j) s[j] += exp(x[j] - m) / l;
+    }
+    free(x);
+  }
+  return ORACLE_OK;
+}
+
 /* GQA mean-merge: merged[b, h, j] = mean over g of raw[b, h*G + g, j]. */
 void oracle_merge(int B, int Hq, int Hkv, int n_max, const double* raw, const int32_t* lengths,
                   double* merged) {

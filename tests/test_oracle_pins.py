@@ -298,3 +298,55 @@ def test_scores_at_equals_full_oracle():
         got = oracle.scores_at(wl.q[0, 2 * h: 2 * h + 2], wl.k[0, h, :90], wl.v[0, h, :90],
                                5, 5, pos)
         np.testing.assert_allclose(got, full[0, h, pos], rtol=1e-13)
+
+
+# ---- attention-only score (the write-up's negative control) -----------------
+
+def test_attention_only_mass_sums_to_the_window():
+    # every window query spreads probability 1 over the keys it sees
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((2, 4, 5, 16))
+    k = rng.standard_normal((2, 2, 40, 16)) * 2.0
+    raw = oracle.attn_raw(q, k, [40, 23])
+    for b, L in enumerate([40, 23]):
+        np.testing.assert_allclose(raw[b, :, :L].sum(axis=1), 5.0, rtol=1e-13)
+        assert np.all(np.isnan(raw[b, :, L:]))
+
+
+def test_attention_only_uniform_keys_closed_form():
+    # equal keys: query t sees P_t + 1 keys, each with p = 1 / (P_t + 1)
+    L, w, d = 12, 4, 8
+    q = np.random.default_rng(1).standard_normal((1, 1, w, d))
+    k = np.tile(np.random.default_rng(2).standard_normal(d), (1, 1, L, 1))
+    raw = oracle.attn_raw(q, k, [L])[0, 0]
+    want = np.zeros(L)
+    for t in range(w):
+        P = L - w + t
+        want[: P + 1] += 1.0 / (P + 1)
+    np.testing.assert_allclose(raw, want, rtol=1e-13)
+
+
+def test_attention_only_three_key_closed_form():
+    # d = 4, q = (2,0,0,0), keys (1,0,0,0), 0, (-1,0,0,0): logits / sqrt(4) = 1, 0, -1
+    q = np.zeros((1, 1, 1, 4)); q[0, 0, 0, 0] = 2.0
+    k = np.zeros((1, 1, 3, 4)); k[0, 0, 0, 0] = 1.0; k[0, 0, 2, 0] = -1.0
+    raw = oracle.attn_raw(q, k, [3])[0, 0]
+    e = np.array([math.e, 1.0, 1.0 / math.e])
+    np.testing.assert_allclose(raw, e / e.sum(), rtol=1e-14)
+
+
+def test_attention_only_dominant_key_and_pipeline():
+    # a key far above the rest takes (almost) all the mass of every query that
+    # sees it; after merge / pool / protect the window is +inf and padding NaN
+    rng = np.random.default_rng(3)
+    L, w, d, G = 20, 3, 8, 2
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    q = u + 0.01 * rng.standard_normal((1, G, w, d))  # every query points along u
+    k = rng.standard_normal((1, 1, L, d)) * 0.1
+    k[0, 0, 5] = 60.0 * u  # logit about 60 / sqrt(8) = 21 above the others
+    raw = oracle.attn_raw(q, k, [L])
+    assert np.all(raw[0, :, 5] > w - 1e-3)
+    s = oracle.attn_scores(q, k, [L], w, 1)
+    np.testing.assert_allclose(s[0, 0, : L - w], raw[0, :, : L - w].mean(axis=0), rtol=1e-14)
+    assert np.all(np.isposinf(s[0, 0, L - w: L]))
