@@ -84,10 +84,23 @@ typedef struct dropkv_shape {
   int32_t dtype;        /* dropkv_dtype of q, k and v                         */
 } dropkv_shape;
 
+/* What is scored (dropkv_options.score). */
+typedef enum dropkv_score {
+  /* the exact single-removal output perturbation, sum over the window of
+     ||p_j/(1-p_j) (a - v_j)||^2 (write-up section 核心公式); the default      */
+  DROPKV_SCORE_PERTURBATION = 0,
+  /* the attention-only negative control the write-up reports beside it
+     (section 结果与独立对照): the attention mass sum_t p_j^(t) each token
+     receives from the window queries.  Same merge, pooling, window protection
+     and scores layout; never singular.  Only the first pass reads v (it
+     still produces the window outputs); the second pass reads only k.       */
+  DROPKV_SCORE_ATTENTION = 1
+} dropkv_score;
+
 /* Optional extras for dropkv_scores_ex.  Zero-initialise for defaults. */
 typedef struct dropkv_options {
   int32_t path;        /* dropkv_path                                                  */
-  int32_t reserved;
+  int32_t score;       /* dropkv_score; other values are DROPKV_ERR_ARG                */
   float* attn_out;     /* device fp32 [B, Hq, w, d] or NULL: each window query's
                           attention output a (the write-up's result also returns the
                           window attention/output, section 代码映射与边界)              */

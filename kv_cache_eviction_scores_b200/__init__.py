@@ -31,6 +31,8 @@ __all__ = [
 OK, ERR_ARG, ERR_SINGULAR, ERR_CUDA, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TIMEOUT = range(7)
 PATH_AUTO, PATH_SIMT, PATH_TENSOR = 0, 1, 2
 _PATHS = {"auto": PATH_AUTO, "simt": PATH_SIMT, "tensor": PATH_TENSOR}
+SCORE_PERTURBATION, SCORE_ATTENTION = 0, 1
+_SCORES = {"perturbation": SCORE_PERTURBATION, "attention": SCORE_ATTENTION}
 BF16, F32 = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -57,7 +59,7 @@ class Shape(ctypes.Structure):
 
 
 class Options(ctypes.Structure):
-    _fields_ = [("path", ctypes.c_int32), ("reserved", ctypes.c_int32),
+    _fields_ = [("path", ctypes.c_int32), ("score", ctypes.c_int32),
                 ("attn_out", ctypes.c_void_p), ("stats_out", ctypes.c_void_p),
                 ("events", ctypes.c_void_p), ("n_events", ctypes.c_int32),
                 ("reserved2", ctypes.c_int32)]
@@ -189,7 +191,8 @@ def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int
                   pool_kernel: int, lengths: Optional[Sequence[int]] = None, *,
                   path: str = "auto", out: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, return_attn: bool = False,
-                  status: Optional[torch.Tensor] = None, kernel_events=None):
+                  status: Optional[torch.Tensor] = None, kernel_events=None,
+                  score: str = "perturbation"):
     """fp32 scores [B, Hkv, n_max] (pooled, window = +inf, padding = NaN).
 
     q: [B, Hq, window, d] window queries; k, v: [B, Hkv, n_max, d]; lengths:
@@ -200,7 +203,12 @@ def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int
     [B, Hq, window, d] and (max logit, normaliser) stats [B, Hq, window, 2].
     ``kernel_events``: torch.cuda.Event objects (each recorded once already so
     that its handle exists); events 2i / 2i+1 bracket the i-th kernel launch.
+    ``score``: "perturbation" (DropKV's exact single-removal score) or
+    "attention" (the accumulated window attention probability, the control
+    score), same merge / pool / window handling.
     """
+    if score not in _SCORES:
+        raise ValueError(f"score must be one of {sorted(_SCORES)}")
     _check_inputs(q, k, v)
     shape = make_shape(q, k, window, pool_kernel)
     dev = q.device
@@ -211,7 +219,7 @@ def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int
         raise DropKVError(ERR_ARG, "dropkv_scores_workspace_bytes")
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    opts = Options(_PATHS[path], 0, None, None, None, 0, 0)
+    opts = Options(_PATHS[path], _SCORES[score], None, None, None, 0, 0)
     ev_arr = None
     if kernel_events:
         # raw cudaEvent_t handles of (already recorded once) torch.cuda.Event objects
@@ -265,8 +273,9 @@ def dropkv_select(scores: torch.Tensor, keep_counts: Sequence[int],
 
 
 def evict(q, k, v, window: int, pool_kernel: int, keep_counts: Sequence[int],
-          lengths: Optional[Sequence[int]] = None, *, path: str = "auto"):
+          lengths: Optional[Sequence[int]] = None, *, path: str = "auto",
+          score: str = "perturbation"):
     """Scores and the keep / evict lists in one call: (scores, keep_idx, evict_idx)."""
-    s = dropkv_scores(q, k, v, window, pool_kernel, lengths, path=path)
+    s = dropkv_scores(q, k, v, window, pool_kernel, lengths, path=path, score=score)
     keep_idx, evict_idx = dropkv_select(s, keep_counts, lengths)
     return s, keep_idx, evict_idx

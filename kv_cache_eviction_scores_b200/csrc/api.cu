@@ -133,6 +133,8 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
   if (status_dev && ((uintptr_t)status_dev & 3u)) return DROPKV_ERR_ARG;
   if (opt && opt->attn_out && !aligned16(opt->attn_out)) return DROPKV_ERR_ARG;
   if (opt && opt->stats_out && !aligned16(opt->stats_out)) return DROPKV_ERR_ARG;
+  const int score = opt ? opt->score : DROPKV_SCORE_PERTURBATION;
+  if (score != DROPKV_SCORE_PERTURBATION && score != DROPKV_SCORE_ATTENTION) return DROPKV_ERR_ARG;
   const int path = resolve_path(s, opt ? opt->path : DROPKV_PATH_AUTO);
   if (path == -2) return DROPKV_ERR_ARG;
   if (path == -1) return DROPKV_ERR_UNSUPPORTED;
@@ -179,7 +181,8 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
       kev.end(st);
       if (e == cudaSuccess) {
         kev.begin(st);
-        e = launch_simt_pass2(s, qs, ks, vs, lens, stats_ws, attn_ws, parts, status_word, st);
+        e = launch_simt_pass2(s, qs, ks, vs, lens, stats_ws, attn_ws, parts, status_word, score,
+                              st);
         kev.end(st);
       }
       if (e == cudaSuccess) {
@@ -188,8 +191,8 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
         kev.end(st);
       }
     } else {
-      e = launch_tc_scores(s, qs, ks, vs, lens, lay, ws, attn_user, stats_user, status_word, st,
-                           kev);
+      e = launch_tc_scores(s, qs, ks, vs, lens, lay, ws, attn_user, stats_user, status_word, score,
+                           st, kev);
       if (e == cudaSuccess) {
         kev.begin(st);
         e = launch_epilogue(s, lens, parts, lay.nparts, part_stride, sc, st);

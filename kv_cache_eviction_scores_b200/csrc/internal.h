@@ -73,7 +73,7 @@ cudaError_t launch_simt_pass1(const dropkv_shape& s, const void* q, const void* 
                               float* stats_user, float* attn_user, cudaStream_t st);
 cudaError_t launch_simt_pass2(const dropkv_shape& s, const void* q, const void* k,
                               const void* v, const Lens& lens, const double* stats_ws,
-                              const void* attn_ws, float* part, int32_t* status,
+                              const void* attn_ws, float* part, int32_t* status, int score,
                               cudaStream_t st);
 cudaError_t launch_epilogue(const dropkv_shape& s, const Lens& lens, const float* parts,
                             int nparts, size_t part_stride, float* scores, cudaStream_t st);
@@ -83,7 +83,7 @@ cudaError_t launch_epilogue(const dropkv_shape& s, const Lens& lens, const float
 cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k,
                              const void* v, const Lens& lens, const ScoresLayout& lay,
                              char* ws, float* attn_out, float* stats_out, int32_t* status,
-                             cudaStream_t st, KernelEvents& kev);
+                             int score, cudaStream_t st, KernelEvents& kev);
 int tc_launch_count();
 int tc_split_target();
 bool tc_available();

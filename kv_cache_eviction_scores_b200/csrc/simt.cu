@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(TPB)
 k_simt_pass2(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, Lens lens,
              int Hq, int Hkv, int n_max, int d, int w, const double* __restrict__ stats,
              const acc_t<T>* __restrict__ attn, float* __restrict__ part,
-             int32_t* __restrict__ status) {
+             int32_t* __restrict__ status, int attn_only) {
   using A = acc_t<T>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   A* qa = reinterpret_cast<A*>(smem_raw);                    // [kQB][2][d]
@@ -194,6 +194,10 @@ k_simt_pass2(const T* __restrict__ q, const T* __restrict__ k, const T* __restri
         const A m = (A)stats[2 * (qrow0 + r)], l = (A)stats[2 * (qrow0 + r) + 1];
         const A x = logit(qa + 2 * i * d, ks + tid, TPB, d, isd);
         const A e = exp_acc(x - m);
+        if (attn_only) {  // attention-only score: the probability itself
+          s += e / l;
+          continue;
+        }
         const A den = l - e;  // (1 - p_j) * l
         if (!(den > A(0))) {  // p_j rounds to 1: removal is singular
           atomicMax(status, kStatusSingular);
@@ -231,14 +235,15 @@ cudaError_t pass1_launch(const dropkv_shape& s, const void* q, const void* k, co
 template <typename T, int TPB>
 cudaError_t pass2_launch(const dropkv_shape& s, const void* q, const void* k, const void* v,
                          const Lens& lens, const double* stats, const void* attn, float* part,
-                         int32_t* status, cudaStream_t st) {
+                         int32_t* status, int attn_only, cudaStream_t st) {
   const size_t smem = 2 * (size_t)s.d * TPB * sizeof(T) + (size_t)kQB * 2 * s.d * sizeof(acc_t<T>);
   auto fn = k_simt_pass2<T, TPB>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((s.n_max + TPB - 1) / TPB, lens.B * s.Hkv);
   fn<<<grid, TPB, smem, st>>>((const T*)q, (const T*)k, (const T*)v, lens, s.Hq, s.Hkv, s.n_max,
-                              s.d, s.window, stats, (const acc_t<T>*)attn, part, status);
+                              s.d, s.window, stats, (const acc_t<T>*)attn, part, status,
+                              attn_only);
   return cudaGetLastError();
 }
 
@@ -255,13 +260,15 @@ cudaError_t launch_simt_pass1(const dropkv_shape& s, const void* q, const void* 
 
 cudaError_t launch_simt_pass2(const dropkv_shape& s, const void* q, const void* k,
                               const void* v, const Lens& lens, const double* stats_ws,
-                              const void* attn_ws, float* part, int32_t* status,
+                              const void* attn_ws, float* part, int32_t* status, int score,
                               cudaStream_t st) {
+  const int ao = score == DROPKV_SCORE_ATTENTION ? 1 : 0;
   if (s.dtype == DROPKV_BF16)
-    return pass2_launch<__nv_bfloat16, 128>(s, q, k, v, lens, stats_ws, attn_ws, part, status, st);
+    return pass2_launch<__nv_bfloat16, 128>(s, q, k, v, lens, stats_ws, attn_ws, part, status,
+                                            ao, st);
   if (s.d <= 128)
-    return pass2_launch<float, 128>(s, q, k, v, lens, stats_ws, attn_ws, part, status, st);
-  return pass2_launch<float, 64>(s, q, k, v, lens, stats_ws, attn_ws, part, status, st);
+    return pass2_launch<float, 128>(s, q, k, v, lens, stats_ws, attn_ws, part, status, ao, st);
+  return pass2_launch<float, 64>(s, q, k, v, lens, stats_ws, attn_ws, part, status, ao, st);
 }
 
 }  // namespace dropkv

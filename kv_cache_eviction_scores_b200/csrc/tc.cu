@@ -34,12 +34,14 @@
 //   s += ratio^2 * (||A||^2 + ||v_j||^2 - 2 D); where that expansion cancels by
 //   more than 32x (A close to v_j: a dominant token) the squared distance is
 //   recomputed directly from fp32 A and v_j.
-//   Two warpgroups take alternate tiles.
+//   The attention-only control score (section 结果与独立对照) is the same
+//   kernel instantiated with kAttn: K tiles only, S^T only, s += p.
 //
-// Warp roles (320 threads): warps 0-3 and 4-7 are the two warpgroups, warp 8
-// issues TMA loads, warp 9 allocates TMEM and issues MMAs (lane 0).  Every
-// wait on an mbarrier is bounded (2 s of %globaltimer); on expiry the kernel
-// records DROPKV_ERR_TIMEOUT, every role leaves its loop and TMEM is freed.
+// Warp roles: sixteen score / softmax warps (4 per TMEM lane quarter), one
+// warp issuing TMA loads, one allocating TMEM and issuing MMAs (lane 0), and in
+// pass 1 one more warp computing ||v_j||^2.  Every wait on an mbarrier is
+// bounded (2 s of %globaltimer); on expiry the kernel records
+// DROPKV_ERR_TIMEOUT, every role leaves its loop and TMEM is freed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -673,6 +675,37 @@ __device__ __noinline__ float careful16(uint32_t tS, uint32_t tD, int col0, int 
   return acc;
 }
 
+// Attention-only score (the write-up's control, section 结果与独立对照) for 16
+// query columns of one token: sum of p = 2^(x c - M') over the columns that see
+// the token (all of them when `masked` is false).  r[0..15] holds S^T.
+__device__ __forceinline__ float attn16(const uint32_t* r, const float4* kf, uint64_t c2,
+                                        bool masked, int tok, int L, int w, int crow0, int col0,
+                                        float c) {
+  if (!masked) {
+    uint64_t acc2 = pk2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 k = kf[i];
+      float y0, y1;
+      upk2(ffma2(pk2(f32(r[2 * i]), f32(r[2 * i + 1])), c2, pk2(k.x, k.y)), y0, y1);
+      acc2 = fadd2(acc2, pk2(ex2(y0), ex2(y1)));
+    }
+    float x0, x1;
+    upk2(acc2, x0, x1);
+    return x0 + x1;
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const float nM = reinterpret_cast<const float*>(kf)[(u >> 1) * 4 + (u & 1)];
+    if (tok <= L - w + (crow0 + col0 + u) % w) acc += ex2(fmaf(f32(r[u]), c, nM));
+  }
+  return acc;
+}
+
+// kAttn = false: the DropKV perturbation score.  kAttn = true: the attention-
+// only score; the CTA then streams K alone and issues only the S^T MMA.
+template <bool kAttn>
 __global__ void __maxnreg__(kMaxRegs)
 k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmAhi,
            const __grid_constant__ CUtensorMap tmAlo, const __grid_constant__ CUtensorMap tmK,
@@ -742,8 +775,8 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   // ||A - v||^2 >= (||v|| - ||A||)^2 by a relative 2^-7 rho / (1 - rho)^2,
   // rho = ||A|| / ||v||.  With ||A||^2 <= kLoSkip ||v||^2 for every query of
   // the chunk and every token of the tiles (rho <= 0.0283) that is <= 2.4e-4.
-  bool lo;
-  {
+  bool lo = false;
+  if constexpr (!kAttn) {
     float namx = 0.f;
     for (int i = 0; i < (nqc + 15) / 16; ++i) namx = fmaxf(namx, nAmax[i]);
     bool need = false;
@@ -761,23 +794,27 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     if (lane == 0) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmAhi); prefetch_tmap(&tmAlo);
       prefetch_tmap(&tmK); prefetch_tmap(&tmV);
-      mbar_expect_tx(BQ, (lo ? 3 : 2) * nqc * 256);
+      mbar_expect_tx(BQ, (kAttn ? 1 : lo ? 3 : 2) * nqc * 256);
       tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
       tma_load_2d(smem_u32(sQ) + nqc * 128, &tmQ, BQ, 64, qrow0);
-      tma_load_2d(smem_u32(sAh), &tmAhi, BQ, 0, qrow0);
-      tma_load_2d(smem_u32(sAh) + nqc * 128, &tmAhi, BQ, 64, qrow0);
+      if (!kAttn) {
+        tma_load_2d(smem_u32(sAh), &tmAhi, BQ, 0, qrow0);
+        tma_load_2d(smem_u32(sAh) + nqc * 128, &tmAhi, BQ, 64, qrow0);
+      }
       if (lo) {
         tma_load_2d(smem_u32(sAl), &tmAlo, BQ, 0, qrow0);
         tma_load_2d(smem_u32(sAl) + nqc * 128, &tmAlo, BQ, 64, qrow0);
       }
-      // single thread: no warp vote needed
-      for (int i = 0; i < 2 * T && !*abort_flag; ++i) {  // K_j at i = 2j, V_j at 2j + 1
+      // single thread: no warp vote needed.  Perturbation: K_j at i = 2j and
+      // V_j at 2j + 1; attention-only: K_j at i = j.
+      const int nload = kAttn ? T : 2 * T;
+      for (int i = 0; i < nload && !*abort_flag; ++i) {
         const int r = i % R, ph = (i / R) & 1;
         if (!mbar_wait(EMPTY(r), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
         mbar_expect_tx(FULL(r), kTileBytes);
         const uint32_t dst = smem_u32(sRing + r * kTileBytes);
-        const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
-        const int row = (t0 + (i >> 1)) * kTok;
+        const CUtensorMap* m = (!kAttn && (i & 1)) ? &tmV : &tmK;
+        const int row = (t0 + (kAttn ? i : i >> 1)) * kTok;
         tma_load_3d(dst, m, FULL(r), 0, row, z);
         tma_load_3d(dst + kBox, m, FULL(r), 64, row, z);
       }
@@ -792,7 +829,8 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t nq = (uint32_t)nqc;
     for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
-      const int rk = (2 * j) % R, pk = ((2 * j) / R) & 1;
+      const int ik = kAttn ? j : 2 * j;  // ring position of K_j
+      const int rk = ik % R, pk = (ik / R) & 1;
       const int rv = (2 * j + 1) % R, pv = ((2 * j + 1) / R) & 1;
       const uint32_t dS = tbase + (uint32_t)(s * 256), dD = dS + 128u;
       if (!warp_wait(TF(s), ph ^ 1) || !warp_wait(FULL(rk), pk)) {
@@ -808,8 +846,10 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           mma_ss_w(dS, klo + kslice(kk, 128), rd0.hi, qd.lo + kslice(kk, nq), qd.hi, IDT,
                    kk > 0 ? 1u : 0u);
         mma_commit(EMPTY(rk));
+        if (kAttn) mma_commit(MD(s));
       }
       __syncwarp();
+      if (kAttn) continue;
       if (!warp_wait(FULL(rv), pv)) { fail(a, abort_flag); break; }
       tc_fence_after();
       if (lane == 0) {
@@ -847,7 +887,7 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const int tok = tile0 + row;
       const bool valid = tok < L;
       const size_t ni = (size_t)z * a.n_max + (valid ? tok : 0);
-      const float nv = valid ? a.nvbuf[ni] : 0.f;  // ||v_j||^2 from pass 1
+      const float nv = (!kAttn && valid) ? a.nvbuf[ni] : 0.f;  // ||v_j||^2 from pass 1
       const __nv_bfloat16* vrow_g = a.v + ni * kHd;
       if (!warp_wait(MD(s), ph)) { fail(a, abort_flag); break; }
       if (warp_aborted(abort_flag)) break;
@@ -855,7 +895,13 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const uint32_t tS = tbase + (uint32_t)(s * 256) + lane_off, tD = tS + 128u;
       const bool masked = tile0 + kTok - 1 > L - a.w;
       float acc = 0.f;
-      if (masked) {
+      if (kAttn) {
+        for (int ch = ch0; ch < ch1; ++ch) {
+          uint32_t r[16];
+          tmem_ld16(tS + ch * 16, r);
+          acc += attn16(r, kf + ch * 8, c2, masked, tok, L, a.w, chunk * nqc, ch * 16, c);
+        }
+      } else if (masked) {
         for (int ch = ch0; ch < ch1; ++ch)
           acc += careful16(tS, tD, ch * 16, tok, true, L, a.w, chunk * nqc, qrows, c, nv, arows,
                            vrow_g, &sing);
@@ -983,8 +1029,10 @@ void tc_splits(const Lens& lens, int units_per_row, int budget, int32_t* splits)
 
 cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k, const void* v,
                              const Lens& lens, const ScoresLayout& lay, char* ws, float* attn_out,
-                             float* stats_out, int32_t* status, cudaStream_t st,
+                             float* stats_out, int32_t* status, int score, cudaStream_t st,
                              KernelEvents& kev) {
+  const bool attn_only = score == DROPKV_SCORE_ATTENTION;
+  auto pass2 = attn_only ? k_tc_pass2<true> : k_tc_pass2<false>;
   const TcPlan plan = tc_plan(s);
   TcArgs a;
   memset(&a, 0, sizeof(a));
@@ -1034,7 +1082,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   cudaError_t e = cudaFuncSetAttribute(k_tc_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sm1);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_tc_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    e = cudaFuncSetAttribute(pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
   if (e != cudaSuccess) return e;
 
   kev.begin(st);
@@ -1046,7 +1094,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   kev.end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kev.begin(st);
-  k_tc_pass2<<<ctas, kThreads2, sm2, st>>>(mQ2, mAh, mAl, mK, mV, a);
+  pass2<<<ctas, kThreads2, sm2, st>>>(mQ2, mAh, mAl, mK, mV, a);
   kev.end(st);
   return cudaGetLastError();
 }

@@ -166,8 +166,8 @@ def attn_scores(q, k, lengths, window, pool):
     q = _f64(q)
     if q.shape[2] != window:
         raise ValueError("q must hold exactly the window rows")
-    Hkv = np.asarray(k).shape[1]
-    return pool_protect(merge(attn_raw(q, k, lengths), Hkv, lengths), window, pool, lengths)
+    k = _f64(k)
+    return pool_protect(merge(attn_raw(q, k, lengths), k.shape[1], lengths), window, pool, lengths)
 
 
 def scores_at(Qg, K, V, window, pool, positions: Sequence[int]):

@@ -101,6 +101,19 @@ def test_bad_lengths_and_pointers_are_rejected_on_the_host():
                                  None, None) == dk.ERR_ARG
 
 
+def test_unknown_score_kind_is_rejected_on_the_host():
+    s = _shape()
+    fake = ctypes.c_void_p(0x100000)
+    L = dk.lib()
+    for bad in (-1, 2, 99):
+        opts = dk.Options(dk.PATH_AUTO, bad, None, None, None, 0, 0)
+        assert L.dropkv_scores_ex(ctypes.byref(s), fake, fake, fake, None, fake, fake, 1 << 30,
+                                  None, None, ctypes.byref(opts)) == dk.ERR_ARG
+    with pytest.raises(ValueError):
+        dk.dropkv_scores(torch.zeros(1, 4, 2, 8), torch.zeros(1, 2, 8, 8), torch.zeros(1, 2, 8, 8),
+                         2, 1, score="bogus")
+
+
 def test_small_or_missing_workspace_is_rejected_on_the_host():
     s = _shape()
     fake = ctypes.c_void_p(0x100000)

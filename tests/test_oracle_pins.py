@@ -350,3 +350,13 @@ def test_attention_only_dominant_key_and_pipeline():
     s = oracle.attn_scores(q, k, [L], w, 1)
     np.testing.assert_allclose(s[0, 0, : L - w], raw[0, :, : L - w].mean(axis=0), rtol=1e-14)
     assert np.all(np.isposinf(s[0, 0, L - w: L]))
+
+
+def test_attention_only_accepts_bf16_tensors_as_their_exact_upcast():
+    # bf16 torch inputs are read as their exact fp64 values
+    g = torch.Generator().manual_seed(4)
+    q = torch.randn(1, 4, 3, 16, generator=g).to(torch.bfloat16)
+    k = torch.randn(1, 2, 30, 16, generator=g).to(torch.bfloat16)
+    s_t = oracle.attn_scores(q, k, [30], 3, 3)
+    s_n = oracle.attn_scores(q.double().numpy(), k.double().numpy(), [30], 3, 3)
+    assert np.array_equal(s_t, s_n, equal_nan=True)
