@@ -215,6 +215,12 @@ DROPKV_API int32_t dropkv_select_launches(int32_t B, int32_t Hkv, int32_t n_max,
 /* Static description of a status code. */
 DROPKV_API const char* dropkv_status_string(dropkv_status status);
 
+/* The cudaError_t code (as an int) behind the last DROPKV_ERR_CUDA that a call
+ * made on this host thread returned, and its name; 0 / "cudaSuccess" before
+ * any.  Host-only, never fails. */
+DROPKV_API int32_t dropkv_last_cuda_error(void);
+DROPKV_API const char* dropkv_last_cuda_error_string(void);
+
 /* DROPKV_ABI_VERSION of the loaded library. */
 DROPKV_API int32_t dropkv_abi_version(void);
 

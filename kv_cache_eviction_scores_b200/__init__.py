@@ -104,6 +104,10 @@ def lib():
     L.dropkv_status_string.restype = ctypes.c_char_p
     L.dropkv_abi_version.argtypes = []
     L.dropkv_abi_version.restype = i32
+    L.dropkv_last_cuda_error.argtypes = []
+    L.dropkv_last_cuda_error.restype = i32
+    L.dropkv_last_cuda_error_string.argtypes = []
+    L.dropkv_last_cuda_error_string.restype = ctypes.c_char_p
     _lib = L
     return L
 
@@ -120,6 +124,8 @@ def _check(status: int, what: str):
         return
     if status == ERR_SINGULAR:
         raise SingularError(status, what)
+    if status == ERR_CUDA:
+        what = f"{what} [{lib().dropkv_last_cuda_error_string().decode()}]"
     raise DropKVError(status, what)
 
 

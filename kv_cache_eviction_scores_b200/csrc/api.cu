@@ -110,14 +110,22 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
     o = align_up(o + rows * s.d * 2, kAlign);
     l.tc_qstat = o;
     o = align_up(o + rows * 4 * sizeof(float), kAlign);
-    l.tc_nv = o;
-    o = align_up(o + (size_t)Bs * s.Hkv * (size_t)s.n_max * sizeof(float), kAlign);
+    l.tc_nv = o;  // per head padded to whole 128-token tiles (512-byte rows per tile)
+    o = align_up(o + (size_t)Bs * s.Hkv * (size_t)((s.n_max + 127) / 128) * 128 * sizeof(float),
+                 kAlign);
     l.tc_tmin = o;
     o = align_up(o + (size_t)Bs * s.Hkv * (size_t)((s.n_max + 127) / 128) * p.chunks * sizeof(float),
                  kAlign);
   }
   l.total = o;
   return l;
+}
+
+// The CUDA error behind the last DROPKV_ERR_CUDA returned to this thread.
+static thread_local cudaError_t g_last_cuda = cudaSuccess;
+static dropkv_status cuda_fail(cudaError_t e) {
+  g_last_cuda = e == cudaSuccess ? cudaErrorUnknown : e;
+  return DROPKV_ERR_CUDA;
 }
 
 // Runs the scoring pipeline; `sync` selects the synchronous contract.
@@ -148,7 +156,7 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
   const int Bs_max = s.B < kMaxB ? s.B : kMaxB;
   const ScoresLayout lay = scores_layout(s, Bs_max);
   int32_t* status_word = status_dev ? status_dev : reinterpret_cast<int32_t*>(ws + lay.status);
-  if (cudaMemsetAsync(status_word, 0, sizeof(int32_t), st) != cudaSuccess) return DROPKV_ERR_CUDA;
+  if (cudaError_t e0 = cudaMemsetAsync(status_word, 0, sizeof(int32_t), st)) return cuda_fail(e0);
 
   KernelEvents kev;
   if (opt && opt->events && opt->n_events > 0) {
@@ -199,15 +207,14 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
         kev.end(st);
       }
     }
-    if (e != cudaSuccess) return e == cudaErrorNotSupported ? DROPKV_ERR_UNSUPPORTED
-                                                            : DROPKV_ERR_CUDA;
+    if (e != cudaSuccess) return e == cudaErrorNotSupported ? DROPKV_ERR_UNSUPPORTED : cuda_fail(e);
   }
   if (!sync) return DROPKV_OK;
   int32_t host_status = 0;
-  if (cudaMemcpyAsync(&host_status, status_word, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
-          cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess)
-    return DROPKV_ERR_CUDA;
+  if (cudaError_t e1 =
+          cudaMemcpyAsync(&host_status, status_word, sizeof(int32_t), cudaMemcpyDeviceToHost, st))
+    return cuda_fail(e1);
+  if (cudaError_t e2 = cudaStreamSynchronize(st)) return cuda_fail(e2);
   if (host_status != 0) return static_cast<dropkv_status>(host_status);
   return DROPKV_OK;
 }
@@ -287,7 +294,7 @@ dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* 
     cudaError_t e = launch_select(Bs, Hkv, n_max, scores + seg0 * n_max, L, K,
                                   keep_idx + seg0 * max_keep, max_keep,
                                   evict_idx + seg0 * max_evict, max_evict, workspace, st);
-    if (e != cudaSuccess) return DROPKV_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   return DROPKV_OK;
 }
@@ -311,6 +318,9 @@ int32_t dropkv_select_launches(int32_t B, int32_t Hkv, int32_t n_max, const int3
   if (B < 1 || Hkv < 1 || n_max < 1) return -1;
   return ((B + kMaxB - 1) / kMaxB) * select_launch_count();
 }
+
+int32_t dropkv_last_cuda_error(void) { return (int32_t)g_last_cuda; }
+const char* dropkv_last_cuda_error_string(void) { return cudaGetErrorName(g_last_cuda); }
 
 const char* dropkv_status_string(dropkv_status status) {
   switch (status) {

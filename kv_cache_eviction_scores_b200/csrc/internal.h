@@ -47,7 +47,7 @@ struct ScoresLayout {
   size_t tc_ahi;     // bf16 [B, Hq, w, d] high part of a (tensor path)
   size_t tc_alo;     // bf16 [B, Hq, w, d] low part of a (tensor path)
   size_t tc_qstat;   // fp32 [B, Hq, w, 4] per-query pass-2 constants (tensor path)
-  size_t tc_nv;      // fp32 [B, Hkv, n_max] ||v_j||^2 (tensor path, pass 1 -> pass 2)
+  size_t tc_nv;      // fp32 [B, Hkv, ceil(n_max/128)*128] ||v_j||^2 (tensor path, pass 1 -> pass 2)
   size_t tc_tmin;    // fp32 [B, Hkv, ceil(n_max/128), chunks] min ||v_j||^2 per tile share
   size_t total;
   int nparts;

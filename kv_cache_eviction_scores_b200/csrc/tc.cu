@@ -67,7 +67,8 @@ constexpr int kSimtWarps = 16;     // softmax / score warps: 4 per TMEM lane qua
 constexpr int kWarpTma = kSimtWarps, kWarpMma = kSimtWarps + 1, kWarpNv = kSimtWarps + 2;
 constexpr int kThreads2 = (kSimtWarps + 2) * 32;  // pass 2: + TMA warp, MMA warp
 constexpr int kThreads1 = (kSimtWarps + 3) * 32;  // pass 1: + the ||v||^2 warp
-constexpr int kMaxRegs = 96;       // 5 warps share a sub-partition's 16K registers
+constexpr int kMaxRegs = 96;       // pass 1: 19 warps share the SM's 64K registers
+constexpr int kMaxRegs2 = 96;      // pass 2: 18 warps, 5 on a sub-partition (16K registers)
 constexpr uint32_t kColO = 384;    // pass-1 TMEM columns: three S/P buffers [0, 384), then O
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kPartStride = 136;   // floats per partial row: O[128], m, l (4 parts), pad
@@ -97,7 +98,7 @@ struct TcArgs {
   size_t part_stride;
   float* attn_f32;       // [rows][128] fp32 window outputs a (read back by pass 2)
   const __nv_bfloat16* v;  // [B*Hkv][n_max][128] values (rare direct-distance path)
-  float* nvbuf;          // [B*Hkv][n_max] ||v_j||^2 (pass 1 -> pass 2)
+  float* nvbuf;          // [B*Hkv][ntmax*128] ||v_j||^2 (pass 1 -> pass 2), tile-padded rows
   float* tmin;           // [B*Hkv][ntmax][chunks] min ||v_j||^2 over a chunk's share of a tile
   int32_t ntmax;         // ceil(n_max / 128)
 };
@@ -398,7 +399,7 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           }
         float na, nb;
         upk2(acc2, na, nb);
-        a.nvbuf[(size_t)z * a.n_max + tile0 + row] = na + nb;
+        a.nvbuf[(size_t)z * a.ntmax * kTok + tile0 + row] = na + nb;
         vmin = fminf(vmin, na + nb);
       }
       __syncwarp();
@@ -643,16 +644,14 @@ __device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf
   }
 }
 
-// Careful path for 16 query columns of one token, re-read from TMEM: the
-// causal mask, ratio = e / (L - e) with the singular check when p >= 2^-8, and
-// the direct squared distance where the expansion cancels by more than 32x.
-// Warp-uniform call (the TMEM loads are warp-collective).
-__device__ __noinline__ float careful16(uint32_t tS, uint32_t tD, int col0, int tok, bool masked,
-                                        int L, int w, int crow0, const float4* qstat_rows,
-                                        float c, float nv, const float* arows,
-                                        const __nv_bfloat16* vrow, int* sing) {
-  uint32_t r[32];
-  tmem_ld16x2(tS + col0, tD + col0, r);
+// Careful path for 16 query columns of one token (r[0..15] = S^T, r[16..31] =
+// D): the causal mask, ratio = e / (L - e) with the singular check when
+// p >= 2^-8, and the direct squared distance where the expansion cancels by
+// more than 32x.
+__device__ __noinline__ float careful16(const uint32_t* r, int col0, int tok, bool masked, int L,
+                                        int w, int crow0, const float4* qstat_rows, float c,
+                                        float nv, const float* arows, const __nv_bfloat16* vrow,
+                                        int* sing) {
   float acc = 0.f;
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
@@ -706,7 +705,7 @@ __device__ __forceinline__ float attn16(const uint32_t* r, const float4* kf, uin
 // kAttn = false: the DropKV perturbation score.  kAttn = true: the attention-
 // only score; the CTA then streams K alone and issues only the S^T MMA.
 template <bool kAttn>
-__global__ void __maxnreg__(kMaxRegs)
+__global__ void __maxnreg__(kMaxRegs2)
 k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmAhi,
            const __grid_constant__ CUtensorMap tmAlo, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
@@ -880,55 +879,83 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const float4* qrows = a.qstat + qrow0;
     const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
     float* plane = a.parts + (size_t)(chunk * 4 + g) * a.part_stride + (size_t)z * a.n_max;
+    const int nch = ch1 - ch0;  // this warp's 16-column chunks: 0, 1 or 2 (warp-uniform)
+    // ||v_j||^2 of the next tile is fetched one tile ahead: under the streaming
+    // traffic a global load takes of the order of a tile's work to return
+    auto nv_at = [&](int jj) -> float {
+      const int tk = (t0 + jj) * kTok + row;
+      return (!kAttn && jj < T && tk < L) ? a.nvbuf[(size_t)z * a.ntmax * kTok + tk] : 0.f;
+    };
+    float nv_next = nv_at(0);
     int sing = 0;
+    // A warp with no columns (nch = 0) still walks the tiles: it hands every
+    // buffer back and writes zeros to its plane.
     for (int j = 0; j < T; ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
       const int tile0 = (t0 + j) * kTok;
       const int tok = tile0 + row;
       const bool valid = tok < L;
-      const size_t ni = (size_t)z * a.n_max + (valid ? tok : 0);
-      const float nv = (!kAttn && valid) ? a.nvbuf[ni] : 0.f;  // ||v_j||^2 from pass 1
-      const __nv_bfloat16* vrow_g = a.v + ni * kHd;
+      const float nv = nv_next;
+      nv_next = nv_at(j + 1);
+      const __nv_bfloat16* vrow_g = a.v + ((size_t)z * a.n_max + (valid ? tok : 0)) * kHd;
       if (!warp_wait(MD(s), ph)) { fail(a, abort_flag); break; }
       if (warp_aborted(abort_flag)) break;
       tc_fence_after();
-      const uint32_t tS = tbase + (uint32_t)(s * 256) + lane_off, tD = tS + 128u;
+      const uint32_t tS = tbase + (uint32_t)(s * 256) + lane_off + (uint32_t)(ch0 * 16);
+      const uint32_t tD = tS + 128u;
       const bool masked = tile0 + kTok - 1 > L - a.w;
-      float acc = 0.f;
-      if (kAttn) {
-        for (int ch = ch0; ch < ch1; ++ch) {
-          uint32_t r[16];
-          tmem_ld16(tS + ch * 16, r);
-          acc += attn16(r, kf + ch * 8, c2, masked, tok, L, a.w, chunk * nqc, ch * 16, c);
-        }
-      } else if (masked) {
-        for (int ch = ch0; ch < ch1; ++ch)
-          acc += careful16(tS, tD, ch * 16, tok, true, L, a.w, chunk * nqc, qrows, c, nv, arows,
-                           vrow_g, &sing);
-      } else {
-        const uint64_t nv2 = pk2(nv, nv);
-        for (int ch = ch0; ch < ch1; ++ch) {
-          uint32_t r[32];
-          tmem_ld16x2(tS + ch * 16, tD + ch * 16, r);  // 16 columns of S^T and of D
-          uint64_t a2 = pk2(0.f, 0.f);
+      // The buffer goes back to the MMA warp as soon as its last columns this
+      // warp needs are in registers (before the last chunk's arithmetic), so
+      // that the MMAs of tile j + 2 overlap the rest of this tile's work.
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(TF(s));
+      };
+      // score of 16 columns (chunk ch) from S^T in r[0..15] and D in r[16..31]
+      auto chunk_score = [&](const uint32_t(&r)[32], int ch) -> float {
+        bool redo = masked;
+        uint64_t a2 = pk2(0.f, 0.f);
+        if (!masked) {
           float pmax = 0.f;
-          fast16(r, kf + ch * 8, c2, nv2, a2, pmax);
+          fast16(r, kf + ch * 8, c2, pk2(nv, nv), a2, pmax);
           // a large p (>= 2^-4: the series above would be short) or possible
           // cancellation (||A||^2 >= 0.6 ||v||^2): the careful path
-          const bool redo = pmax >= 0.0625f || nAmax[ch] >= 0.6f * nv;
-          if (__any_sync(0xffffffffu, redo)) {
-            acc += careful16(tS, tD, ch * 16, tok, false, L, a.w, chunk * nqc, qrows, c, nv,
-                             arows, vrow_g, &sing);
-          } else {
-            float x0, x1;
-            upk2(a2, x0, x1);
-            acc += x0 + x1;
-          }
+          redo = pmax >= 0.0625f || nAmax[ch] >= 0.6f * nv;
+        }
+        if (__any_sync(0xffffffffu, redo)) {
+          uint32_t rc[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) rc[k] = r[k];
+          return careful16(rc, ch * 16, tok, masked, L, a.w, chunk * nqc, qrows, c, nv, arows,
+                           vrow_g, &sing);
+        }
+        float x0, x1;
+        upk2(a2, x0, x1);
+        return x0 + x1;
+      };
+      float acc = 0.f;
+      if (nch == 0) {
+        release();
+      } else if (kAttn) {
+        uint32_t r[32];
+        tmem_ld32(tS, r);  // S^T of chunks ch0, ch0 + 1 (the second unused when nch = 1)
+        release();
+        acc = attn16(r, kf + ch0 * 8, c2, masked, tok, L, a.w, chunk * nqc, ch0 * 16, c);
+        if (nch > 1)
+          acc += attn16(r + 16, kf + ch0 * 8 + 8, c2, masked, tok, L, a.w, chunk * nqc,
+                        ch0 * 16 + 16, c);
+      } else {
+        uint32_t r[32];
+        tmem_ld16x2(tS, tD, r);  // chunk ch0: 16 columns of S^T and of D
+        if (nch == 1) release();
+        acc = chunk_score(r, ch0);
+        if (nch > 1) {
+          tmem_ld16x2(tS + 16u, tD + 16u, r);  // chunk ch0 + 1
+          release();
+          acc += chunk_score(r, ch0 + 1);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(TF(s));
       if (valid) plane[tok] = acc;
     }
     if (sing) atomicMax(a.status, (int)DROPKV_ERR_SINGULAR);

@@ -161,3 +161,9 @@ def test_no_device_means_unsupported_not_a_cpu_fallback():
     need = dk.scores_workspace_bytes(s)
     st = dk.lib().dropkv_scores(ctypes.byref(s), fake, fake, fake, None, fake, fake, need, None)
     assert st == dk.ERR_UNSUPPORTED
+
+
+def test_last_cuda_error_starts_clear():
+    L = dk.lib()
+    assert L.dropkv_last_cuda_error() == 0
+    assert L.dropkv_last_cuda_error_string() == b"cudaSuccess"
