@@ -19,6 +19,7 @@ scaled by 32) on the host cores.
 """
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -61,6 +62,9 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", type=int, default=3, help="workload index (3 = 128K headline)")
     p.add_argument("--path", choices=["auto", "simt", "tensor"], default="auto")
+    p.add_argument("--seq", type=int, default=None,
+                   help="override the configuration's sequence length (one batch row; profiling "
+                        "a smaller case of the same shape)")
     p.add_argument("--score", choices=["perturbation", "attention"], default="perturbation",
                    help="DropKV's perturbation score, or the attention-only control score")
     p.add_argument("--e2e-steps", type=int, default=None)
@@ -77,6 +81,15 @@ def peaks():
             "measured"
     except Exception:
         return 6650.0, 1590.0, 1965.0, "fallback"
+
+
+def bench_spec(args):
+    spec = W.config_spec(args.config)
+    if args.seq is not None:
+        frac = spec.keep[0] / spec.lengths[0]
+        spec = dataclasses.replace(spec, name=f"{spec.name}@n{args.seq}", B=1, lengths=[args.seq],
+                                   n_max=args.seq, keep=[int(frac * args.seq)])
+    return spec
 
 
 def workload_desc(spec):
@@ -199,7 +212,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    spec = W.config_spec(args.config)
+    spec = bench_spec(args)
     wl = W.generate(spec, 42)
     tokens = sum(wl.lengths)
     times = []
@@ -354,7 +367,7 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     dk.lib()
 
-    spec = W.config_spec(args.config)
+    spec = bench_spec(args)
     wl = W.generate(spec, rank_seed(rank))
     q, k, v = wl.q.to(dev), wl.k.to(dev), wl.v.to(dev)
     shape = dk.make_shape(q, k, spec.window, spec.pool)
