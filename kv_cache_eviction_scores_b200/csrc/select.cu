@@ -181,12 +181,15 @@ __device__ bool cluster_phase(uint32_t bar, int& phase, volatile int* fail, int3
   return *fail == 0;
 }
 
+// kCached: every CTA's range fits one sub-range and is read from the
+// shared-memory key cache in every phase (no global loads after the fill).
+template <bool kCached>
 __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 1)
 k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ keep_idx,
          int32_t* __restrict__ evict_idx) {
   extern __shared__ uint32_t smem_dyn[];     // [kSub] key cache / staging, then histogram copies
   uint32_t* cached_keys = smem_dyn;          // this CTA's range when it fits one sub-range
-  int32_t* staging = reinterpret_cast<int32_t*>(smem_dyn + (p.cache ? kSub : 0));
+  int32_t* staging = reinterpret_cast<int32_t*>(smem_dyn + (kCached ? kSub : 0));
   uint32_t* loc = smem_dyn + 2 * kSub;       // [kCopies][kCopyStride] this CTA's histograms
   __shared__ uint32_t H[3][kBins];           // the cluster histogram of each round (rank 0's)
   __shared__ int32_t warp_tot[kWarps];
@@ -206,7 +209,6 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   const long long span_ll = (((long long)L + kC - 1) / kC + 31) & ~31ll;
   const int lo = (int)min((long long)L, (long long)rank * span_ll);
   const int hi = (int)min((long long)L, (long long)lo + span_ll);
-  const bool cached = p.cache != 0;  // sized for the longest row of the launch
   const float* s = scores + (size_t)seg * p.n_max;
   const uint32_t barA = smem_addr(&bar), gbarA = smem_addr(&gbar), bbarA = smem_addr(&bbar);
 
@@ -224,7 +226,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   // cache layout: key r of the range at r ^ ((r >> 5) & 31), so that both the
   // coalesced fill (32 consecutive r per warp) and the per-thread runs (lane t
   // reads r = 32 t + u) touch 32 distinct banks
-  if (cached)
+  if (kCached)
     for (int j = lo + tid; j < hi; j += kThreads) {
       const int r = j - lo;
       cached_keys[r ^ ((r >> 5) & 31)] = key_of(__ldg(s + j));
@@ -236,7 +238,8 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
                    "memory");
   auto key_at = [&](int j) {
     const int r = j - lo;
-    return cached ? cached_keys[r ^ ((r >> 5) & 31)] : key_of(__ldg(s + j));
+    if constexpr (kCached) return cached_keys[r ^ ((r >> 5) & 31)];
+    else return key_of(__ldg(s + j));
   };
   // this thread's kPer consecutive keys of the sub-range starting at sub0
   // (slots past hi read as the NaN key; every use masks them by position)
@@ -486,11 +489,11 @@ cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const 
   // [key cache when it fits][staging][histogram copies]; the histogram copies
   // always start at 2 * kSub words
   const size_t smem = (2 * (size_t)kSub + kCopies * (size_t)kCopyStride) * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  auto kern = p.cache ? k_select<true> : k_select<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(status, 0, sizeof(int32_t), st)) != cudaSuccess) return e;
-  k_select<<<B * Hkv * kC, kThreads, smem, st>>>(p, scores, keep_idx, evict_idx);
+  kern<<<B * Hkv * kC, kThreads, smem, st>>>(p, scores, keep_idx, evict_idx);
   return cudaGetLastError();
 }
 
