@@ -54,6 +54,9 @@ KERNEL_SRC = {
 }
 
 
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e nominal (DGX figure), context beside the measured peak
+
+
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -454,10 +457,15 @@ def run_ours(args):
                    "seq_len": max(spec.lengths),
                    "parallelism": f"replicas x{world} (independent inputs per GPU)",
                    "l2": f"inputs {kv_bytes / 1e6:.0f} MB > 126 MB L2; no flush"},
+        "token_heads_per_s": value * spec.Hkv,
         "hbm": {"alg_bytes_per_step": alg_bytes,
                 "achieved_gbs": alg_bytes / (ms * 1e-3) / 1e9 * 1.0,
                 "peak_gbs": hbm_peak, "frac": alg_bytes / (ms * 1e-3) / 1e9 / hbm_peak,
-                "of": peak_src},
+                "of": peak_src,
+                "frac_nominal": alg_bytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+                "nominal_gbs": NOMINAL_HBM_GBS},
+        "phases_us": {"scores": sum(kern_us[n] for n in names),
+                      "select": kern_us["select (all launches)"]},
         "roofline": roof,
         "kernels_us": kern_us,
         "e2e": e2e,

@@ -360,3 +360,22 @@ def test_attention_only_accepts_bf16_tensors_as_their_exact_upcast():
     s_t = oracle.attn_scores(q, k, [30], 3, 3)
     s_n = oracle.attn_scores(q.double().numpy(), k.double().numpy(), [30], 3, 3)
     assert np.array_equal(s_t, s_n, equal_nan=True)
+
+
+def test_negative_control_differs_from_dropkv():
+    # the attention-only score is a different ranking from DropKV's: on a seeded
+    # workload the two orders are not the same and the evict sets differ
+    spec = W.small_spec(1)
+    wl = W.generate(spec, 42)
+    s_dk = oracle.scores(wl.q, wl.k, wl.v, wl.lengths, spec.window, spec.pool)
+    s_at = oracle.attn_scores(wl.q, wl.k, wl.lengths, spec.window, spec.pool)
+    L = wl.lengths[0]
+    hist = L - spec.window
+    for h in range(spec.Hkv):
+        a, b = s_dk[0, h, :hist], s_at[0, h, :hist]
+        ra, rb = np.argsort(np.argsort(a)), np.argsort(np.argsort(b))
+        rho = np.corrcoef(ra, rb)[0, 1]  # Spearman rank correlation
+        assert rho < 0.9, (h, rho)
+    _, ev_dk = oracle.select(s_dk, wl.lengths, wl.keep)
+    _, ev_at = oracle.select(s_at, wl.lengths, wl.keep)
+    assert not np.array_equal(ev_dk, ev_at)
