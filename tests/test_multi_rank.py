@@ -64,3 +64,17 @@ def test_rank_seeds_are_distinct_and_single_rank_is_identity():
     assert bench.rank_seed(0) != bench.rank_seed(1)
     assert bench.max_over_ranks(3.5, None, torch.device("cpu")) == 3.5
     assert bench.whole_job_value(1, 1000, 2.0) == pytest.approx(5e5)
+
+
+def test_sequence_override_keeps_the_shape_and_budget_fraction():
+    import argparse
+
+    spec = bench.bench_spec(argparse.Namespace(config=3, seq=32768))
+    full = W.config_spec(3)
+    assert (spec.Hq, spec.Hkv, spec.d, spec.window, spec.pool) == \
+        (full.Hq, full.Hkv, full.d, full.window, full.pool)
+    assert spec.lengths == [32768] and spec.n_max == 32768 and spec.B == 1
+    assert spec.keep[0] == int(full.keep[0] / full.lengths[0] * 32768)
+    assert spec.outlier_channels == full.outlier_channels
+    assert bench.bench_spec(argparse.Namespace(config=3, seq=None)) == full
+    assert bench.NOMINAL_HBM_GBS == 8000.0
