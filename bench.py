@@ -23,6 +23,7 @@ import dataclasses
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -244,8 +245,12 @@ def run_reference(args):
 # ------------------------------------------------------------------ ours ----
 
 def source_hash(fname):
-    with open(os.path.join(CSRC, fname), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    """sha256 of a kernel source's code: line comments and blank lines removed,
+    so that a comment edit does not invalidate the stored DRAM traffic."""
+    with open(os.path.join(CSRC, fname), encoding="utf-8") as f:
+        lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in f)
+        code = "\n".join(ln for ln in lines if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()
 
 
 def traffic_for(kernel):

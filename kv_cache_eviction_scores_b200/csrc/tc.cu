@@ -15,25 +15,28 @@
 //
 // k_tc_pass1 (query-major, one CTA per (b, h, chunk, split)):
 //   S = Q_chunk K_tile^T      tcgen05 M=128 (queries) N=128 (tokens) K=128
-//   online softmax per query row in registers (log2 domain; the reference max
-//   only moves up by more than 8, so exp2 stays <= 256 and O rarely rescales)
-//   P = exp2(S*c - m) written back over S in TMEM as two bf16 planes,
+//   online softmax per query row (log2 domain; the reference max only moves up
+//   by more than 8, so exp2 stays <= 256 and O rarely rescales).  Sixteen
+//   softmax warps share every tile: each owns 32 rows x 32 tokens, posts its
+//   row maxima for the other three warps of its rows and, one tile behind,
+//   writes P = exp2(S*c - m) back over S in TMEM as two bf16 planes,
 //   P_hi = P truncated to bf16 and P_lo = bf16(P - P_hi), so P_hi + P_lo holds
 //   P to 2^-16 relative;  O += P_hi V + P_lo V   (A from TMEM, V MN-major).
-//   Two softmax warpgroups take alternate tiles, each with its own S/P buffer,
-//   O accumulator and (m, l): each writes one partial (m, l, O) per row.
+//   Three S/P buffers let S run two tiles ahead of P V.  Each CTA writes one
+//   partial (m, l, O) per row.
 // k_tc_combine: merges the partials of a row into the final max M, normaliser
-//   L and output A = O / L; writes A as bf16 hi/lo planes (same 2^-16 split)
-//   plus the per-query constants (M, 1/L, L, ||A||^2) for pass 2.
+//   L and output A = O / L; writes -2A as bf16 hi/lo planes (same split) plus
+//   the per-query constants (M, 1/L, L, ||A||^2) for pass 2.
 // k_tc_pass2 (token-major, one CTA per (b, h, chunk, split)):
-//   S^T = K_tile Q^T and D = V_tile A_hi^T + V_tile A_lo^T, tcgen05 M=128
-//   (tokens) N=nqc (queries) K=128; each thread owns one token and sums over
-//   the chunk's queries:  e = exp2(S*c - M), p = e / L,
-//   ratio = p + p^2 + p^3 when p < 2^-8 (exact to fp32 rounding), otherwise
-//   e / (L - e) with the singular check (L - e not > 0 => rejected),
-//   s += ratio^2 * (||A||^2 + ||v_j||^2 - 2 D); where that expansion cancels by
-//   more than 32x (A close to v_j: a dominant token) the squared distance is
-//   recomputed directly from fp32 A and v_j.
+//   S^T = K_tile Q^T and D = V_tile (-2A_hi)^T [+ V_tile (-2A_lo)^T], tcgen05
+//   M=128 (tokens) N=nqc (queries) K=128, into two TMEM buffers; each thread
+//   owns one token and sums over its warp's 32 queries:  p = exp2(S*c - M'),
+//   M' = M + log2 L; while p < 2^-4 the series p(1 + p(1 + p(1 + p(1 + p))))
+//   gives p / (1 - p); otherwise ratio = e / (L - e) with the singular check
+//   (L - e not > 0 => rejected); s += ratio^2 * (||A||^2 + ||v_j||^2 + D);
+//   where that expansion cancels by more than 32x (A close to v_j: a dominant
+//   token) the squared distance is recomputed directly from fp32 A and v_j.
+//   A warp hands its TMEM buffer back once its last columns are in registers.
 //   The attention-only control score (section 结果与独立对照) is the same
 //   kernel instantiated with kAttn: K tiles only, S^T only, s += p.
 //
