@@ -82,11 +82,6 @@ __device__ __forceinline__ void dsm_add(uint32_t raddr, uint32_t v) {
 __device__ __forceinline__ void dsm_st(uint32_t raddr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(raddr), "r"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t dsm_ld(uint32_t raddr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(raddr) : "memory");
-  return v;
-}
 __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
