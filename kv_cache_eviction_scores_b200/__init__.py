@@ -10,6 +10,17 @@ and the Algorithm 1 paragraph): for the last ``window`` prompt queries,
 p = softmax(K q / sqrt d), a = sum_j p_j v_j, Delta_j = p_j/(1-p_j) (a - v_j),
 s_j = sum_t ||Delta_j||^2; scores are averaged over the query heads of each KV
 head, max-pooled, the window is set to +inf, and the lowest scores are evicted.
+
+Usage (CUDA tensors; q holds the last ``window`` query rows of each sequence)::
+
+    import kv_cache_eviction_scores_b200 as dk
+    # q [B, Hq, window, d], k / v [B, Hkv, n_max, d], bf16 or fp32
+    scores = dk.dropkv_scores(q, k, v, window, pool_kernel, lengths)   # [B, Hkv, n_max]
+    keep_idx, evict_idx = dk.dropkv_select(scores, keep_counts, lengths)
+    # or both at once:
+    scores, keep_idx, evict_idx = dk.evict(q, k, v, window, pool_kernel, keep_counts, lengths)
+    # the attention-only control score through the same pipeline:
+    control = dk.dropkv_scores(q, k, v, window, pool_kernel, lengths, score="attention")
 """
 
 from __future__ import annotations
@@ -25,7 +36,7 @@ __all__ = [
     "make_shape", "scores_workspace_bytes", "select_workspace_bytes", "dropkv_scores",
     "dropkv_select", "evict", "auto_path", "scores_launches", "select_launches",
     "OK", "ERR_ARG", "ERR_SINGULAR", "ERR_CUDA", "ERR_UNSUPPORTED", "ERR_WORKSPACE", "ERR_TIMEOUT",
-    "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR",
+    "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR", "SCORE_PERTURBATION", "SCORE_ATTENTION",
 ]
 
 OK, ERR_ARG, ERR_SINGULAR, ERR_CUDA, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_TIMEOUT = range(7)
