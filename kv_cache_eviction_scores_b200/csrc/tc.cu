@@ -809,9 +809,10 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       }
       // single thread: no warp vote needed.  Perturbation: K_j at i = 2j and
       // V_j at 2j + 1; attention-only: K_j at i = j.
+      // (slot, phase) of load i kept incrementally: R is a runtime ring size
       const int nload = kAttn ? T : 2 * T;
-      for (int i = 0; i < nload && !*abort_flag; ++i) {
-        const int r = i % R, ph = (i / R) & 1;
+      int r = 0, ph = 0;
+      for (int i = 0; i < nload && !*abort_flag; ++i, r = (r + 1 == R) ? 0 : r + 1, ph ^= (r == 0)) {
         if (!mbar_wait(EMPTY(r), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
         mbar_expect_tx(FULL(r), kTileBytes);
         const uint32_t dst = smem_u32(sRing + r * kTileBytes);
@@ -829,11 +830,20 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024), hd = sdesc_split(smem_u32(sAh), 16, 1024),
                 ld = sdesc_split(smem_u32(sAl), 16, 1024);
     const uint32_t nq = (uint32_t)nqc;
+    // ring (slot, phase) of K_j kept incrementally (R is a runtime ring size):
+    // V_j follows K_j, K_{j+1} follows V_j (or K_j for the attention score)
+    int pos = 0, pph = 0;
     for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
-      const int ik = kAttn ? j : 2 * j;  // ring position of K_j
-      const int rk = ik % R, pk = (ik / R) & 1;
-      const int rv = (2 * j + 1) % R, pv = ((2 * j + 1) / R) & 1;
+      const int rk = pos, pk = pph;
+      int rv = rk + 1, pv = pk;
+      if (rv == R) { rv = 0; pv ^= 1; }
+      if (kAttn) {
+        pos = rv; pph = pv;
+      } else {
+        pos = rv + 1; pph = pv;
+        if (pos == R) { pos = 0; pph ^= 1; }
+      }
       const uint32_t dS = tbase + (uint32_t)(s * 256), dD = dS + 128u;
       if (!warp_wait(TF(s), ph ^ 1) || !warp_wait(FULL(rk), pk)) {
         fail(a, abort_flag);
