@@ -221,6 +221,16 @@ DROPKV_API const char* dropkv_status_string(dropkv_status status);
 DROPKV_API int32_t dropkv_last_cuda_error(void);
 DROPKV_API const char* dropkv_last_cuda_error_string(void);
 
+/* Self-test of the bounded device waits that the kernels use: enqueues one
+ * CTA on `stream` that waits on an mbarrier nothing ever arrives on, gives up
+ * after limit_ns nanoseconds of %globaltimer and then writes
+ * DROPKV_ERR_TIMEOUT into *status_dev (device int32, 4-byte aligned, not
+ * cleared by the call).  The kernel returns normally: no fault or trap, the
+ * context stays usable.  0 < limit_ns <= 1e9, else DROPKV_ERR_ARG; no
+ * sm_100 device gives DROPKV_ERR_UNSUPPORTED. */
+DROPKV_API dropkv_status dropkv_selftest_wait_timeout(int32_t* status_dev, uint64_t limit_ns,
+                                                      void* stream);
+
 /* DROPKV_ABI_VERSION of the loaded library. */
 DROPKV_API int32_t dropkv_abi_version(void);
 

@@ -35,6 +35,7 @@ __all__ = [
     "DropKVError", "SingularError", "Shape", "Options", "lib", "lib_path",
     "make_shape", "scores_workspace_bytes", "select_workspace_bytes", "dropkv_scores",
     "dropkv_select", "evict", "auto_path", "scores_launches", "select_launches",
+    "selftest_wait_timeout",
     "OK", "ERR_ARG", "ERR_SINGULAR", "ERR_CUDA", "ERR_UNSUPPORTED", "ERR_WORKSPACE", "ERR_TIMEOUT",
     "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR", "SCORE_PERTURBATION", "SCORE_ATTENTION",
 ]
@@ -115,6 +116,8 @@ def lib():
     L.dropkv_status_string.restype = ctypes.c_char_p
     L.dropkv_abi_version.argtypes = []
     L.dropkv_abi_version.restype = i32
+    L.dropkv_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
+    L.dropkv_selftest_wait_timeout.restype = i32
     L.dropkv_last_cuda_error.argtypes = []
     L.dropkv_last_cuda_error.restype = i32
     L.dropkv_last_cuda_error_string.argtypes = []
@@ -257,6 +260,18 @@ def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int
     if return_attn:
         return out, attn, stats
     return out
+
+
+def selftest_wait_timeout(limit_ms: float = 20.0, device=None) -> int:
+    """Runs the bounded-wait self-test (a wait on an mbarrier nothing arrives
+    on) and returns the status word it leaves: ERR_TIMEOUT when the device-side
+    wait gave up as designed."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    _check(lib().dropkv_selftest_wait_timeout(_ptr(status), int(limit_ms * 1e6), _stream(dev)),
+           "dropkv_selftest_wait_timeout")
+    torch.cuda.synchronize(dev)
+    return int(status.item())
 
 
 def dropkv_select(scores: torch.Tensor, keep_counts: Sequence[int],

@@ -61,6 +61,8 @@ int resolve_path(const dropkv_shape& s, int requested) {
 
 }  // namespace
 
+dropkv_status device_ok() { return check_device(); }
+
 // Tensor path: bf16, d = 128, and the G*w query rows of a KV head split into
 // equal chunks of at most 128 rows whose size is a multiple of 16 (the N of
 // the token-major pass-2 MMA).

@@ -61,6 +61,8 @@ struct TcPlan {
 };
 
 bool tc_shape_ok(const dropkv_shape& s);
+// DROPKV_OK when the current device is an sm_100 part the kernels run on.
+dropkv_status device_ok();
 TcPlan tc_plan(const dropkv_shape& s);
 ScoresLayout scores_layout(const dropkv_shape& s, int B_slice);
 

@@ -167,3 +167,14 @@ def test_last_cuda_error_starts_clear():
     L = dk.lib()
     assert L.dropkv_last_cuda_error() == 0
     assert L.dropkv_last_cuda_error_string() == b"cudaSuccess"
+
+
+def test_wait_selftest_rejects_bad_arguments_on_the_host():
+    L = dk.lib()
+    fake = ctypes.c_void_p(0x100000)
+    assert L.dropkv_selftest_wait_timeout(None, 1000, None) == dk.ERR_ARG
+    assert L.dropkv_selftest_wait_timeout(ctypes.c_void_p(0x100002), 1000, None) == dk.ERR_ARG
+    assert L.dropkv_selftest_wait_timeout(fake, 0, None) == dk.ERR_ARG
+    assert L.dropkv_selftest_wait_timeout(fake, 2_000_000_000, None) == dk.ERR_ARG
+    if not torch.cuda.is_available():
+        assert L.dropkv_selftest_wait_timeout(fake, 1000, None) == dk.ERR_UNSUPPORTED
