@@ -49,7 +49,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_time_is_the_max_and_value_counts_all_ranks():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     assert set(out.keys()) == {0, 1}
