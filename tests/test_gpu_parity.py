@@ -125,6 +125,10 @@ EDGE = [
     # more batch rows than one launch slice holds
     W.Spec("batch70", B=70, Hq=2, Hkv=1, d=8, lengths=[10 + (b * 7) % 40 for b in range(70)],
            window=3, pool=3, keep=[5 + (b % 4) for b in range(70)], dtype="f32", n_max=60),
+    # more batch rows than one launch slice holds, on the tensor path
+    W.Spec("batch66_tc", B=66, Hq=4, Hkv=1, d=128,
+           lengths=[130 + (b * 37) % 170 for b in range(66)], window=8, pool=5,
+           keep=[20 + (b % 7) for b in range(66)], dtype="bf16", n_max=300),
     # NaN-poisoned padding with the tensor-path shape
     W.Spec("nan_pad_tc", B=2, Hq=8, Hkv=2, d=128, lengths=[140, 389], window=16, pool=7,
            keep=[16, 100], dtype="bf16", n_max=400, nan_pad=True),
