@@ -178,3 +178,25 @@ def test_wait_selftest_rejects_bad_arguments_on_the_host():
     assert L.dropkv_selftest_wait_timeout(fake, 2_000_000_000, None) == dk.ERR_ARG
     if not torch.cuda.is_available():
         assert L.dropkv_selftest_wait_timeout(fake, 1000, None) == dk.ERR_UNSUPPORTED
+
+
+def test_noalloc_select_rejects_bad_arguments_on_the_host():
+    L = dk.lib()
+    i32, vp = ctypes.c_int32, ctypes.c_void_p
+    ip = ctypes.POINTER(ctypes.c_int32)
+    fn = L.dropkv_select_noalloc
+    fn.argtypes = [i32, i32, i32, vp, ip, ip, vp, i32, vp, i32, vp]
+    fn.restype = i32
+    fake = ctypes.c_void_p(0x100000)
+    lens = (ctypes.c_int32 * 2)(100, 50)
+    keep_ok = (ctypes.c_int32 * 2)(10, 5)
+    keep_bad = (ctypes.c_int32 * 2)(10, 51)
+    assert fn(0, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, None) == dk.ERR_ARG
+    assert fn(2, 4, 100, None, lens, keep_ok, fake, 10, fake, 90, None) == dk.ERR_ARG
+    assert fn(2, 4, 100, fake, lens, keep_bad, fake, 64, fake, 90, None) == dk.ERR_ARG
+    assert fn(2, 4, 100, fake, lens, keep_ok, fake, 5, fake, 90, None) == dk.ERR_ARG   # max_keep
+    assert fn(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 80, None) == dk.ERR_ARG  # max_evict
+    odd = ctypes.c_void_p(0x100004)  # scores not 16-byte aligned
+    assert fn(2, 4, 100, odd, lens, keep_ok, fake, 10, fake, 90, None) == dk.ERR_ARG
+    if not torch.cuda.is_available():
+        assert fn(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, None) == dk.ERR_UNSUPPORTED
