@@ -78,3 +78,26 @@ def test_sequence_override_keeps_the_shape_and_budget_fraction():
     assert spec.outlier_channels == full.outlier_channels
     assert bench.bench_spec(argparse.Namespace(config=3, seq=None)) == full
     assert bench.NOMINAL_HBM_GBS == 8000.0
+
+
+def test_visible_elements_counts_the_causal_window():
+    # brute force: query t of a head sees keys 0 .. L - w + t
+    spec = W.small_spec(4)
+    brute = sum(sum(L - spec.window + t + 1 for t in range(spec.window)) for L in spec.lengths)
+    assert bench.visible_elements(spec) == brute * spec.Hq
+
+
+def test_roofline_arithmetic_of_the_passes():
+    spec = W.config_spec(3)
+    us = 200.0
+    kv = sum(spec.lengths) * spec.Hkv * spec.d * 2  # one read of K (or V), bf16
+    r = bench.roofline("k_tc_pass2", spec, us, 6554.6, 1657.0, 1965.0)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(2 * kv / (us * 1e-6) / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6554.6)
+    flops = 4 * spec.d * bench.visible_elements(spec)
+    assert r["tensor"]["achieved"] == pytest.approx(flops / (us * 1e-6) / 1e12)
+    # the attention-only second pass streams K alone and runs one contraction
+    ra = bench.roofline("k_tc_pass2", spec, us, 6554.6, 1657.0, 1965.0, "attention")
+    assert ra["achieved"] == pytest.approx(kv / (us * 1e-6) / 1e9)
+    assert ra["tensor"]["achieved"] == pytest.approx(flops / 2 / (us * 1e-6) / 1e12)
