@@ -13,9 +13,8 @@ flush is needed between steps.  With N GPUs (torchrun) every rank scores its
 own independent input set (seed 42 + rank): weak scaling, no data-path
 collective; the time is the max over ranks.
 
---impl reference times the fp64 CPU oracle on a bounded sample of the same
-workload (one query head of 32: its 64 window queries over all 131072 keys,
-scaled by 32) on the host cores.
+--impl reference times the fp64 CPU oracle on the same whole workload on the
+host cores (one OpenMP thread per batch row and query head).
 """
 
 import argparse
@@ -188,27 +187,22 @@ class ClockSampler:
 # ------------------------------------------------------------ reference ----
 
 def oracle_sample(wl):
-    """fp64 oracle on the first KV heads of batch row 0 (all their query heads,
-    window queries over every key), then merge/pool/protect/select of them.
-    The oracle runs one OpenMP thread per query head, so the sample takes as
-    many KV heads as keep the host cores busy.  Returns (seconds, share of the
-    whole workload, threads used, description)."""
+    """fp64 oracle on the whole workload: every KV head of every batch row (all
+    query heads, window queries over every key), then merge / pool / protect
+    and the selection.  The oracle runs one OpenMP thread per (batch row, query
+    head).  Returns (seconds, share of the workload = 1, threads used,
+    description)."""
     import oracle
     spec = wl.spec
-    L = wl.lengths[0]
-    G = spec.G
-    nkv = max(1, min(spec.Hkv, oracle.num_threads() // G))
     t0 = time.perf_counter()
-    s = oracle.scores(wl.q[0:1, 0:nkv * G], wl.k[0:1, 0:nkv, :L], wl.v[0:1, 0:nkv, :L], [L],
-                      spec.window, spec.pool)
-    oracle.select(s, [L], [wl.keep[0]])
+    s = oracle.scores(wl.q, wl.k, wl.v, wl.lengths, spec.window, spec.pool)
+    oracle.select(s, wl.lengths, wl.keep)
     dt = time.perf_counter() - t0
-    frac = (nkv * G * L) / (spec.Hq * sum(wl.lengths))
-    threads = min(oracle.num_threads(), nkv * G)
-    desc = (f"{nkv} of {spec.Hkv} KV heads of batch row 0 ({nkv * G} query heads x "
-            f"{spec.window} window queries over all {L} keys), fp64, {dt:.2f} s, "
-            f"scaled by {1 / frac:.3g}")
-    return dt, frac, threads, desc
+    threads = min(oracle.num_threads(), spec.B * spec.Hq)
+    desc = (f"the whole workload ({spec.B} x {spec.Hq} query heads x {spec.window} window "
+            f"queries over all {sum(wl.lengths)} keys, then merge / pool / select), fp64, "
+            f"{dt:.2f} s")
+    return dt, 1.0, threads, desc
 
 
 def run_reference(args):

@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define DROPKV_ABI_VERSION 1
+#define DROPKV_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define DROPKV_API __attribute__((visibility("default")))
@@ -110,7 +110,13 @@ typedef struct dropkv_options {
                           2i and 2i+1 are recorded on `stream` right before and after
                           the i-th kernel this call launches (for live timing)        */
   int32_t n_events;
-  int32_t reserved2;
+  int32_t tc_ctas;     /* tensor path only: the most CTAs one scoring pass launches
+                          per batch slice (0 = one per SM, at most 160).  Each CTA
+                          walks a contiguous run of 128-token tiles of one (b, h,
+                          query chunk), so fewer CTAs mean longer runs.  Values
+                          below the slice's (b, h, chunk) unit count act as that
+                          count, values above 160 as 160; < 0 is DROPKV_ERR_ARG.
+                          Any value gives the same scores up to fp32 rounding.      */
 } dropkv_options;
 
 /* Bytes of device workspace dropkv_scores* needs for this shape (any lengths).
@@ -169,13 +175,30 @@ DROPKV_API size_t dropkv_select_workspace_bytes(int32_t B, int32_t Hkv, int32_t 
  *   evict_idx    device int32 [B, Hkv, max_evict]: evicted positions ascending,
  *                then -1;  max_evict >= every lengths[b] - keep_counts[b].
  *                (keep_idx / evict_idx may be NULL when max_keep / max_evict is 0.)
- * Asynchronous on `stream`; integer results are exact.
+ * Asynchronous on `stream`; integer results are exact.  The kernels' waits on
+ * one another are bounded; if one gives up, that (b, h)'s lists are filled
+ * with -1 (every slot, once the other CTAs of the segment have finished) and
+ * DROPKV_ERR_TIMEOUT is recorded in the workspace, which only
+ * dropkv_select_ex reports.
  */
 DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
                             const int32_t* lengths, const int32_t* keep_counts,
                             int32_t* keep_idx, int32_t max_keep, int32_t* evict_idx,
                             int32_t max_evict, void* workspace, size_t workspace_bytes,
                             void* stream);
+
+/* dropkv_select that reports the device-side status.  status_dev NULL: the
+ * call synchronises `stream` and returns DROPKV_ERR_TIMEOUT if a bounded wait
+ * of the kernels gave up, else DROPKV_OK.  status_dev non-NULL (device int32,
+ * 4-byte aligned, caller-owned): asynchronous; the call zeroes *status_dev on
+ * the stream and the kernels raise it to DROPKV_ERR_TIMEOUT on a timeout.
+ * Host-side errors are returned directly and nothing is enqueued. */
+DROPKV_API dropkv_status dropkv_select_ex(int32_t B, int32_t Hkv, int32_t n_max,
+                                          const float* scores, const int32_t* lengths,
+                                          const int32_t* keep_counts, int32_t* keep_idx,
+                                          int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
+                                          void* workspace, size_t workspace_bytes, void* stream,
+                                          int32_t* status_dev);
 
 /*
  * dropkv_select without a workspace, for callers that cannot allocate device
@@ -192,9 +215,14 @@ DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, co
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
  *   before any stream capture.  No call allocates or frees memory.
- *   All calls share the array and it keeps the last call's contents (every
- *   call resets what must start at zero): calls whose work overlaps on the GPU,
- *   e.g. on two streams at once, race and must be serialised by the caller.
+ *   All calls share the array and it keeps the last call's contents: each
+ *   call enqueues one memset of the array's 4-byte status word on `stream`
+ *   before its kernels.  Calls whose work overlaps on the GPU, e.g. on
+ *   two streams at once, race and must be serialised by the caller.
+ *   A device-side timeout of the kernels' bounded waits is not reported by
+ *   this entry point (its status word sits in the shared array); the lists of
+ *   the affected (b, h) are then filled with -1.  Use dropkv_select_ex where a
+ *   timeout must be detected.
  */
 DROPKV_API dropkv_status dropkv_select_noalloc(int32_t B, int32_t Hkv, int32_t n_max,
                                                const float* scores, const int32_t* lengths,
@@ -230,6 +258,24 @@ DROPKV_API const char* dropkv_last_cuda_error_string(void);
  * sm_100 device gives DROPKV_ERR_UNSUPPORTED. */
 DROPKV_API dropkv_status dropkv_selftest_wait_timeout(int32_t* status_dev, uint64_t limit_ns,
                                                       void* stream);
+
+/* Self-test of the select kernel's failure path: runs the select of
+ * dropkv_select on the given arguments (B <= 64) with one CTA of every
+ * segment's cluster withholding its first arrival and every bounded wait
+ * limited to limit_ns nanoseconds (0 < limit_ns <= 1e9).  Every segment with
+ * at least one eviction then ends with DROPKV_ERR_TIMEOUT in *status_dev
+ * (device int32, zeroed by the call) and all its keep and evict slots set to
+ * -1.  Asynchronous on `stream`; no fault or trap is involved and the context
+ * stays usable.  Errors as for dropkv_select, plus DROPKV_ERR_ARG for B > 64
+ * or a bad status_dev / limit. */
+DROPKV_API dropkv_status dropkv_selftest_select_timeout(int32_t B, int32_t Hkv, int32_t n_max,
+                                                        const float* scores,
+                                                        const int32_t* lengths,
+                                                        const int32_t* keep_counts,
+                                                        int32_t* keep_idx, int32_t max_keep,
+                                                        int32_t* evict_idx, int32_t max_evict,
+                                                        int32_t* status_dev, uint64_t limit_ns,
+                                                        void* stream);
 
 /* DROPKV_ABI_VERSION of the loaded library. */
 DROPKV_API int32_t dropkv_abi_version(void);

@@ -35,7 +35,7 @@ __all__ = [
     "DropKVError", "SingularError", "Shape", "Options", "lib", "lib_path",
     "make_shape", "scores_workspace_bytes", "select_workspace_bytes", "dropkv_scores",
     "dropkv_select", "evict", "auto_path", "scores_launches", "select_launches",
-    "selftest_wait_timeout",
+    "selftest_wait_timeout", "selftest_select_timeout",
     "OK", "ERR_ARG", "ERR_SINGULAR", "ERR_CUDA", "ERR_UNSUPPORTED", "ERR_WORKSPACE", "ERR_TIMEOUT",
     "PATH_AUTO", "PATH_SIMT", "PATH_TENSOR", "SCORE_PERTURBATION", "SCORE_ATTENTION",
 ]
@@ -74,7 +74,7 @@ class Options(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("score", ctypes.c_int32),
                 ("attn_out", ctypes.c_void_p), ("stats_out", ctypes.c_void_p),
                 ("events", ctypes.c_void_p), ("n_events", ctypes.c_int32),
-                ("reserved2", ctypes.c_int32)]
+                ("tc_ctas", ctypes.c_int32)]
 
 
 _lib = None
@@ -106,6 +106,8 @@ def lib():
     L.dropkv_select_workspace_bytes.restype = sz
     L.dropkv_select.argtypes = [i32, i32, i32, vp, ip, ip, vp, i32, vp, i32, vp, sz, vp]
     L.dropkv_select.restype = i32
+    L.dropkv_select_ex.argtypes = [i32, i32, i32, vp, ip, ip, vp, i32, vp, i32, vp, sz, vp, vp]
+    L.dropkv_select_ex.restype = i32
     L.dropkv_auto_path.argtypes = [sp]
     L.dropkv_auto_path.restype = i32
     L.dropkv_scores_launches.argtypes = [sp, ip, i32]
@@ -118,6 +120,9 @@ def lib():
     L.dropkv_abi_version.restype = i32
     L.dropkv_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
     L.dropkv_selftest_wait_timeout.restype = i32
+    L.dropkv_selftest_select_timeout.argtypes = [i32, i32, i32, vp, ip, ip, vp, i32, vp, i32, vp,
+                                                 ctypes.c_uint64, vp]
+    L.dropkv_selftest_select_timeout.restype = i32
     L.dropkv_last_cuda_error.argtypes = []
     L.dropkv_last_cuda_error.restype = i32
     L.dropkv_last_cuda_error_string.argtypes = []
@@ -212,7 +217,7 @@ def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int
                   path: str = "auto", out: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, return_attn: bool = False,
                   status: Optional[torch.Tensor] = None, kernel_events=None,
-                  score: str = "perturbation"):
+                  score: str = "perturbation", tc_ctas: int = 0):
     """fp32 scores [B, Hkv, n_max] (pooled, window = +inf, padding = NaN).
 
     q: [B, Hq, window, d] window queries; k, v: [B, Hkv, n_max, d]; lengths:
@@ -226,6 +231,8 @@ def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int
     ``score``: "perturbation" (DropKV's exact single-removal score) or
     "attention" (the accumulated window attention probability, the control
     score), same merge / pool / window handling.
+    ``tc_ctas``: on the tensor path, the most CTAs a scoring pass launches
+    (0 = one per SM); fewer CTAs walk longer runs of tiles each.
     """
     if score not in _SCORES:
         raise ValueError(f"score must be one of {sorted(_SCORES)}")
@@ -239,7 +246,7 @@ def dropkv_scores(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int
         raise DropKVError(ERR_ARG, "dropkv_scores_workspace_bytes")
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    opts = Options(_PATHS[path], _SCORES[score], None, None, None, 0, 0)
+    opts = Options(_PATHS[path], _SCORES[score], None, None, None, 0, int(tc_ctas))
     ev_arr = None
     if kernel_events:
         # raw cudaEvent_t handles of (already recorded once) torch.cuda.Event objects
@@ -274,11 +281,41 @@ def selftest_wait_timeout(limit_ms: float = 20.0, device=None) -> int:
     return int(status.item())
 
 
+def selftest_select_timeout(scores: torch.Tensor, keep_counts: Sequence[int],
+                            lengths: Optional[Sequence[int]] = None, limit_ms: float = 20.0):
+    """Runs the select kernel with one CTA of every segment withholding an
+    arrival and waits limited to ``limit_ms``; returns (status word, keep_idx,
+    evict_idx).  Segments with evictions report ERR_TIMEOUT and lists of -1."""
+    B, Hkv, n_max = scores.shape
+    lens = list(lengths) if lengths is not None else [n_max] * B
+    keep = [int(x) for x in keep_counts]
+    max_keep = max(keep)
+    max_evict = max(L - kc for L, kc in zip(lens, keep))
+    dev = scores.device
+    keep_idx = torch.full((B, Hkv, max_keep), 7, dtype=torch.int32, device=dev)
+    evict_idx = torch.full((B, Hkv, max_evict), 7, dtype=torch.int32, device=dev)
+    status = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    _check(lib().dropkv_selftest_select_timeout(
+        B, Hkv, n_max, _ptr(scores), _i32_array(lengths), _i32_array(keep), _ptr(keep_idx),
+        max_keep, _ptr(evict_idx), max_evict, _ptr(status), int(limit_ms * 1e6), _stream(dev)),
+        "dropkv_selftest_select_timeout")
+    torch.cuda.synchronize(dev)
+    return int(status.item()), keep_idx, evict_idx
+
+
 def dropkv_select(scores: torch.Tensor, keep_counts: Sequence[int],
                   lengths: Optional[Sequence[int]] = None, *, max_keep: Optional[int] = None,
                   max_evict: Optional[int] = None,
-                  workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Keep / evict positions per (b, h), ascending, padded with -1 (int32)."""
+                  workspace: Optional[torch.Tensor] = None,
+                  status: Optional[torch.Tensor] = None,
+                  sync: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Keep / evict positions per (b, h), ascending, padded with -1 (int32).
+
+    Asynchronous by default.  With ``status`` (a CUDA int32 tensor of one
+    element) the device-side status of the kernels (OK, or ERR_TIMEOUT if a
+    bounded wait gave up) lands there; with ``sync=True`` the call waits for
+    the stream and raises on a device-side error.
+    """
     if not scores.is_cuda or scores.dtype != torch.float32 or not scores.is_contiguous():
         raise TypeError("scores must be a contiguous CUDA float32 tensor")
     B, Hkv, n_max = scores.shape
@@ -296,10 +333,15 @@ def dropkv_select(scores: torch.Tensor, keep_counts: Sequence[int],
     need = select_workspace_bytes(B, Hkv, n_max)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    st = lib().dropkv_select(B, Hkv, n_max, _ptr(scores), _i32_array(lengths),
-                             _i32_array(keep), _ptr(keep_idx), max_keep, _ptr(evict_idx),
-                             max_evict, _ptr(workspace),
-                             workspace.numel() * workspace.element_size(), _stream(dev))
+    args = (B, Hkv, n_max, _ptr(scores), _i32_array(lengths), _i32_array(keep), _ptr(keep_idx),
+            max_keep, _ptr(evict_idx), max_evict, _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(dev))
+    if status is not None or sync:
+        if status is not None and (not status.is_cuda or status.dtype != torch.int32):
+            raise TypeError("status must be a CUDA int32 tensor")
+        st = lib().dropkv_select_ex(*args, _ptr(status))
+    else:
+        st = lib().dropkv_select(*args)
     _check(st, "dropkv_select")
     return keep_idx, evict_idx
 

@@ -125,9 +125,50 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
 
 // The CUDA error behind the last DROPKV_ERR_CUDA returned to this thread.
 static thread_local cudaError_t g_last_cuda = cudaSuccess;
-static dropkv_status cuda_fail(cudaError_t e) {
+dropkv_status cuda_fail(cudaError_t e) {
   g_last_cuda = e == cudaSuccess ? cudaErrorUnknown : e;
   return DROPKV_ERR_CUDA;
+}
+
+dropkv_status check_select_args(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
+                                const int32_t* lengths, const int32_t* keep_counts,
+                                const int32_t* keep_idx, int32_t max_keep,
+                                const int32_t* evict_idx, int32_t max_evict) {
+  if (B < 1 || Hkv < 1 || n_max < 1 || !scores || !keep_counts) return DROPKV_ERR_ARG;
+  if ((!keep_idx && max_keep > 0) || (!evict_idx && max_evict > 0)) return DROPKV_ERR_ARG;
+  if (max_keep < 0 || max_evict < 0) return DROPKV_ERR_ARG;
+  if (!aligned16(scores) || ((uintptr_t)keep_idx & 3u) || ((uintptr_t)evict_idx & 3u))
+    return DROPKV_ERR_ARG;
+  if ((double)B * Hkv * (double)n_max > 4.0e18) return DROPKV_ERR_ARG;
+  for (int b = 0; b < B; ++b) {
+    const int L = lengths ? lengths[b] : n_max;
+    if (L < 0 || L > n_max) return DROPKV_ERR_ARG;
+    if (keep_counts[b] < 0 || keep_counts[b] > L) return DROPKV_ERR_ARG;
+    if (keep_counts[b] > max_keep || L - keep_counts[b] > max_evict) return DROPKV_ERR_ARG;
+  }
+  return DROPKV_OK;
+}
+
+dropkv_status run_select(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
+                         const int32_t* lengths, const int32_t* keep_counts, int32_t* keep_idx,
+                         int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
+                         int32_t* status_word, cudaStream_t st) {
+  // one reset per call: a timeout in one launch slice stays visible after the next
+  if (cudaError_t e = cudaMemsetAsync(status_word, 0, sizeof(int32_t), st)) return cuda_fail(e);
+  for (int b0 = 0; b0 < B; b0 += kMaxB) {
+    const int Bs = (B - b0) < kMaxB ? (B - b0) : kMaxB;
+    int32_t L[kMaxB], K[kMaxB];
+    for (int i = 0; i < Bs; ++i) {
+      L[i] = lengths ? lengths[b0 + i] : n_max;
+      K[i] = keep_counts[b0 + i];
+    }
+    const size_t seg0 = (size_t)b0 * Hkv;
+    cudaError_t e = launch_select(Bs, Hkv, n_max, scores + seg0 * n_max, L, K,
+                                  keep_idx + seg0 * max_keep, max_keep,
+                                  evict_idx + seg0 * max_evict, max_evict, status_word, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return DROPKV_OK;
 }
 
 // Runs the scoring pipeline; `sync` selects the synchronous contract.
@@ -145,6 +186,8 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
   if (opt && opt->stats_out && !aligned16(opt->stats_out)) return DROPKV_ERR_ARG;
   const int score = opt ? opt->score : DROPKV_SCORE_PERTURBATION;
   if (score != DROPKV_SCORE_PERTURBATION && score != DROPKV_SCORE_ATTENTION) return DROPKV_ERR_ARG;
+  const int tc_ctas = opt ? opt->tc_ctas : 0;
+  if (tc_ctas < 0) return DROPKV_ERR_ARG;
   const int path = resolve_path(s, opt ? opt->path : DROPKV_PATH_AUTO);
   if (path == -2) return DROPKV_ERR_ARG;
   if (path == -1) return DROPKV_ERR_UNSUPPORTED;
@@ -202,7 +245,7 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
       }
     } else {
       e = launch_tc_scores(s, qs, ks, vs, lens, lay, ws, attn_user, stats_user, status_word, score,
-                           st, kev);
+                           tc_ctas, st, kev);
       if (e == cudaSuccess) {
         kev.begin(st);
         e = launch_epilogue(s, lens, parts, lay.nparts, part_stride, sc, st);
@@ -263,42 +306,49 @@ size_t dropkv_select_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_max) {
   return select_workspace_bytes(Bs, Hkv, n_max);
 }
 
+static dropkv_status select_entry(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
+                                  const int32_t* lengths, const int32_t* keep_counts,
+                                  int32_t* keep_idx, int32_t max_keep, int32_t* evict_idx,
+                                  int32_t max_evict, void* workspace, size_t workspace_bytes,
+                                  void* stream, int32_t* status_dev, bool sync) {
+  dropkv_status r = check_select_args(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx,
+                                      max_keep, evict_idx, max_evict);
+  if (r != DROPKV_OK) return r;
+  if (status_dev && ((uintptr_t)status_dev & 3u)) return DROPKV_ERR_ARG;
+  const size_t need = dropkv_select_workspace_bytes(B, Hkv, n_max);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DROPKV_ERR_WORKSPACE;
+  r = check_device();
+  if (r != DROPKV_OK) return r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* status_word = status_dev ? status_dev : reinterpret_cast<int32_t*>(workspace);
+  r = run_select(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx, max_keep, evict_idx,
+                 max_evict, status_word, st);
+  if (r != DROPKV_OK || !sync) return r;
+  int32_t host_status = 0;
+  if (cudaError_t e1 =
+          cudaMemcpyAsync(&host_status, status_word, sizeof(int32_t), cudaMemcpyDeviceToHost, st))
+    return cuda_fail(e1);
+  if (cudaError_t e2 = cudaStreamSynchronize(st)) return cuda_fail(e2);
+  return host_status != 0 ? static_cast<dropkv_status>(host_status) : DROPKV_OK;
+}
+
 dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
                             const int32_t* lengths, const int32_t* keep_counts,
                             int32_t* keep_idx, int32_t max_keep, int32_t* evict_idx,
                             int32_t max_evict, void* workspace, size_t workspace_bytes,
                             void* stream) {
-  if (B < 1 || Hkv < 1 || n_max < 1 || !scores || !keep_counts) return DROPKV_ERR_ARG;
-  if ((!keep_idx && max_keep > 0) || (!evict_idx && max_evict > 0)) return DROPKV_ERR_ARG;
-  if (max_keep < 0 || max_evict < 0) return DROPKV_ERR_ARG;
-  if (!aligned16(scores) || ((uintptr_t)keep_idx & 3u) || ((uintptr_t)evict_idx & 3u))
-    return DROPKV_ERR_ARG;
-  if ((double)B * Hkv * (double)n_max > 4.0e18) return DROPKV_ERR_ARG;
-  for (int b = 0; b < B; ++b) {
-    const int L = lengths ? lengths[b] : n_max;
-    if (L < 0 || L > n_max) return DROPKV_ERR_ARG;
-    if (keep_counts[b] < 0 || keep_counts[b] > L) return DROPKV_ERR_ARG;
-    if (keep_counts[b] > max_keep || L - keep_counts[b] > max_evict) return DROPKV_ERR_ARG;
-  }
-  const size_t need = dropkv_select_workspace_bytes(B, Hkv, n_max);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DROPKV_ERR_WORKSPACE;
-  dropkv_status r = check_device();
-  if (r != DROPKV_OK) return r;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  for (int b0 = 0; b0 < B; b0 += kMaxB) {
-    const int Bs = (B - b0) < kMaxB ? (B - b0) : kMaxB;
-    int32_t L[kMaxB], K[kMaxB];
-    for (int i = 0; i < Bs; ++i) {
-      L[i] = lengths ? lengths[b0 + i] : n_max;
-      K[i] = keep_counts[b0 + i];
-    }
-    const size_t seg0 = (size_t)b0 * Hkv;
-    cudaError_t e = launch_select(Bs, Hkv, n_max, scores + seg0 * n_max, L, K,
-                                  keep_idx + seg0 * max_keep, max_keep,
-                                  evict_idx + seg0 * max_evict, max_evict, workspace, st);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  return DROPKV_OK;
+  return select_entry(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx, max_keep, evict_idx,
+                      max_evict, workspace, workspace_bytes, stream, nullptr, false);
+}
+
+dropkv_status dropkv_select_ex(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
+                               const int32_t* lengths, const int32_t* keep_counts,
+                               int32_t* keep_idx, int32_t max_keep, int32_t* evict_idx,
+                               int32_t max_evict, void* workspace, size_t workspace_bytes,
+                               void* stream, int32_t* status_dev) {
+  return select_entry(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx, max_keep, evict_idx,
+                      max_evict, workspace, workspace_bytes, stream, status_dev,
+                      status_dev == nullptr);
 }
 
 int32_t dropkv_auto_path(const dropkv_shape* shape) {

@@ -82,10 +82,11 @@ cudaError_t launch_epilogue(const dropkv_shape& s, const Lens& lens, const float
 
 // Tensor-core path (tcgen05 + TMA); returns cudaErrorNotSupported when the
 // tensor maps cannot be encoded.
+// cta_budget: most CTAs per pass (0 = one per SM).
 cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k,
                              const void* v, const Lens& lens, const ScoresLayout& lay,
                              char* ws, float* attn_out, float* stats_out, int32_t* status,
-                             int score, cudaStream_t st, KernelEvents& kev);
+                             int score, int cta_budget, cudaStream_t st, KernelEvents& kev);
 int tc_launch_count();
 int tc_split_target();
 bool tc_available();
@@ -93,8 +94,33 @@ bool tc_available();
 // ---- selection --------------------------------------------------------------
 size_t select_workspace_bytes(int B, int Hkv, int n_max);
 int select_launch_count();
+// One launch slice (B <= kMaxB rows).  `status` (device int32) receives
+// DROPKV_ERR_TIMEOUT by atomicMax if a bounded wait gives up; the caller
+// zeroes it once per call.
 cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const int32_t* L,
                           const int32_t* keep, int32_t* keep_idx, int32_t max_keep,
-                          int32_t* evict_idx, int32_t max_evict, void* ws, cudaStream_t st);
+                          int32_t* evict_idx, int32_t max_evict, int32_t* status,
+                          cudaStream_t st);
+
+// The same launch for the select self-test: CTA rank 1 of every segment's
+// cluster withholds its first arrival and every bounded wait gives up after
+// wait_ns, so the segments with evictions end in DROPKV_ERR_TIMEOUT.
+cudaError_t launch_select_stalled(int B, int Hkv, int n_max, const float* scores,
+                                  const int32_t* L, const int32_t* keep, int32_t* keep_idx,
+                                  int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
+                                  int32_t* status, uint64_t wait_ns, cudaStream_t st);
+
+// Shared by the select entry points: host-side argument checks, and the
+// slice loop with one status reset per call (returns DROPKV_ERR_CUDA through
+// cuda_fail, which records the CUDA error for dropkv_last_cuda_error).
+dropkv_status check_select_args(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
+                                const int32_t* lengths, const int32_t* keep_counts,
+                                const int32_t* keep_idx, int32_t max_keep,
+                                const int32_t* evict_idx, int32_t max_evict);
+dropkv_status run_select(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
+                         const int32_t* lengths, const int32_t* keep_counts, int32_t* keep_idx,
+                         int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
+                         int32_t* status_word, cudaStream_t st);
+dropkv_status cuda_fail(cudaError_t e);
 
 }  // namespace dropkv

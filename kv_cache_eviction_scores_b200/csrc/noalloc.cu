@@ -14,8 +14,11 @@
 // current) and caches it; because that lookup is a runtime call, the first call
 // on each device should happen before any stream capture.  All calls share the
 // one array, so calls whose work overlaps on the GPU (on different streams)
-// race; the kernels themselves reset every part of the scratch that must start
-// at zero at the beginning of each call.
+// race.  The only part of the scratch that must start at zero is the 4-byte
+// status word of the select kernels: each call enqueues one cudaMemsetAsync of
+// it on the caller's stream before its kernels.  That word is not returned to
+// the caller: a select kernel whose bounded wait gives up fills the lists of
+// its (b, h) with -1 instead.
 #include <mutex>
 
 #include "internal.h"
@@ -61,43 +64,17 @@ extern "C" dropkv_status dropkv_select_noalloc(int32_t B, int32_t Hkv, int32_t n
                                                const int32_t* keep_counts, int32_t* keep_idx,
                                                int32_t max_keep, int32_t* evict_idx,
                                                int32_t max_evict, void* stream) {
-  if (B < 1 || Hkv < 1 || n_max < 1 || !scores || !keep_counts) return DROPKV_ERR_ARG;
-  if ((!keep_idx && max_keep > 0) || (!evict_idx && max_evict > 0)) return DROPKV_ERR_ARG;
-  if (max_keep < 0 || max_evict < 0) return DROPKV_ERR_ARG;
-  if ((reinterpret_cast<uintptr_t>(scores) & 15u) || (reinterpret_cast<uintptr_t>(keep_idx) & 3u) ||
-      (reinterpret_cast<uintptr_t>(evict_idx) & 3u))
-    return DROPKV_ERR_ARG;
-  if ((double)B * Hkv * (double)n_max > 4.0e18) return DROPKV_ERR_ARG;
-  for (int b = 0; b < B; ++b) {
-    const int L = lengths ? lengths[b] : n_max;
-    if (L < 0 || L > n_max) return DROPKV_ERR_ARG;
-    if (keep_counts[b] < 0 || keep_counts[b] > L) return DROPKV_ERR_ARG;
-    if (keep_counts[b] > max_keep || L - keep_counts[b] > max_evict) return DROPKV_ERR_ARG;
-  }
+  dropkv_status r = check_select_args(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx,
+                                      max_keep, evict_idx, max_evict);
+  if (r != DROPKV_OK) return r;
   // the scratch a launch slice needs must fit the static array
   const int Bs = B < kMaxB ? B : kMaxB;
   if (select_workspace_bytes(Bs, Hkv, n_max) > kNoAllocScratchBytes) return DROPKV_ERR_WORKSPACE;
-  int dev = -1, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return DROPKV_ERR_UNSUPPORTED;
-  }
-  if (major != 10) return DROPKV_ERR_UNSUPPORTED;
+  r = device_ok();
+  if (r != DROPKV_OK) return r;
   void* ws = nullptr;
-  if (scratch_ptr(&ws) != cudaSuccess) return DROPKV_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  for (int b0 = 0; b0 < B; b0 += kMaxB) {
-    const int n = (B - b0) < kMaxB ? (B - b0) : kMaxB;
-    int32_t L[kMaxB], K[kMaxB];
-    for (int i = 0; i < n; ++i) {
-      L[i] = lengths ? lengths[b0 + i] : n_max;
-      K[i] = keep_counts[b0 + i];
-    }
-    const size_t seg0 = (size_t)b0 * Hkv;
-    if (launch_select(n, Hkv, n_max, scores + seg0 * n_max, L, K, keep_idx + seg0 * max_keep,
-                      max_keep, evict_idx + seg0 * max_evict, max_evict, ws, st) != cudaSuccess)
-      return DROPKV_ERR_CUDA;
-  }
-  return DROPKV_OK;
+  if (cudaError_t e = scratch_ptr(&ws)) return cuda_fail(e);
+  return run_select(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx, max_keep, evict_idx,
+                    max_evict, reinterpret_cast<int32_t*>(ws),
+                    reinterpret_cast<cudaStream_t>(stream));
 }

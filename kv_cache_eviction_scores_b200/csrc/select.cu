@@ -27,9 +27,13 @@
 //       keys; two block scans give every thread its kept / evicted ranks, the
 //       positions are staged in shared memory and copied out coalesced.
 // The phases are separated by cluster-wide mbarrier phases with bounded waits;
-// a wait that gives up records DROPKV_ERR_TIMEOUT in the workspace status word
-// and the CTA keeps taking the remaining phase barriers (without the work), so
-// no CTA leaves while another may still address its shared memory.
+// a wait that gives up records DROPKV_ERR_TIMEOUT in the status word and the
+// CTA keeps taking the remaining phase barriers (without the work).  The kernel
+// ends on the hardware cluster barrier, so no CTA leaves while another may
+// still address its shared memory.  Before that barrier every CTA stores
+// whether it gave up into every CTA; after it, if any CTA of the segment gave
+// up, each CTA writes -1 over its share of the segment's keep and evict slots.
+// Every data write precedes the barrier, so no stale index survives a timeout.
 #include "common.cuh"
 #include "internal.h"
 
@@ -53,6 +57,9 @@ struct SelParams {
   int32_t E[kMaxB];                  // evictions per row
   int32_t* status;                   // device status word (0 = OK)
   int32_t cache;                     // 1: every CTA's range fits one cached sub-range
+  int32_t stall_rank;                // self-test only: this rank withholds its first
+                                     // gather arrival (-1: none, the product path)
+  uint64_t wait_ns;                  // limit of every bounded wait
 };
 
 __device__ __forceinline__ uint32_t key_of(float s) {
@@ -119,7 +126,8 @@ __device__ __forceinline__ void arrive_at(uint32_t bar, uint32_t rank) {
 }
 // Thread 0 only: bounded wait (acquire, cluster scope) for the phase of
 // parity `parity` of this CTA's mbarrier `bar`.  On expiry records the timeout.
-__device__ bool wait_at(uint32_t bar, uint32_t parity, volatile int* fail, int32_t* status) {
+__device__ bool wait_at(uint32_t bar, uint32_t parity, volatile int* fail, int32_t* status,
+                        uint64_t limit_ns) {
   const uint64_t t0 = gtimer();
   for (;;) {
     uint32_t done;
@@ -131,7 +139,7 @@ __device__ bool wait_at(uint32_t bar, uint32_t parity, volatile int* fail, int32
         : "r"(bar), "r"(parity)
         : "memory");
     if (done) return true;
-    if (gtimer() - t0 > kWaitNs) {
+    if (gtimer() - t0 > limit_ns) {
       *fail = 1;
       atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
       return false;
@@ -145,7 +153,8 @@ __device__ bool wait_at(uint32_t bar, uint32_t parity, volatile int* fail, int32
 // cluster, then waits (bounded, acquire at cluster scope) for all kC arrivals
 // on its own; a second block barrier releases the other threads.  Returns
 // false once any wait of this CTA has given up.
-__device__ bool cluster_phase(uint32_t bar, int& phase, volatile int* fail, int32_t* status) {
+__device__ bool cluster_phase(uint32_t bar, int& phase, volatile int* fail, int32_t* status,
+                              uint64_t limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) {
     asm volatile("fence.acq_rel.cluster;" ::: "memory");
@@ -164,7 +173,7 @@ __device__ bool cluster_phase(uint32_t bar, int& phase, volatile int* fail, int3
           : "r"(bar), "r"(parity)
           : "memory");
       if (done) break;
-      if (gtimer() - t0 > kWaitNs) {
+      if (gtimer() - t0 > limit_ns) {
         *fail = 1;
         atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
         break;
@@ -195,6 +204,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   __shared__ __align__(8) uint64_t bar;     // all-to-all phases (count, final): kC arrivals
   __shared__ __align__(8) uint64_t gbar;    // rank 0: a round's histogram adds landed (kC)
   __shared__ __align__(8) uint64_t bbar;    // every CTA: rank 0 broadcast the round's digit (1)
+  __shared__ uint32_t fails[kC];             // per rank: 1 if a wait of that CTA gave up
   __shared__ int fail;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const uint32_t rank = cluster_rank();
@@ -218,6 +228,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   }
   for (int i = tid; i < 3 * kBins; i += kThreads) (&H[0][0])[i] = 0;
   if (tid < 2 * kC) cnt[tid >> 1][tid & 1] = 0;
+  if (tid < kC) fails[tid] = 0;
   // cache layout: key r of the range at r ^ ((r >> 5) & 31), so that both the
   // coalesced fill (32 consecutive r per warp) and the per-thread runs (lane t
   // reads r = 32 t + u) touch 32 distinct banks
@@ -281,10 +292,10 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
       __syncthreads();
       if (tid == 0) {
         asm volatile("fence.acq_rel.cluster;" ::: "memory");
-        arrive_at(gbarA, 0);
+        if (!(round == 0 && (int)rank == p.stall_rank)) arrive_at(gbarA, 0);
       }
       if (rank == 0) {
-        if (tid == 0) wait_at(gbarA, (uint32_t)(round & 1), &fail, p.status);
+        if (tid == 0) wait_at(gbarA, (uint32_t)(round & 1), &fail, p.status, p.wait_ns);
         __syncthreads();
         if (fail == 0) {
           // the digit holding rank `rem` (1-based) of the keys with this prefix
@@ -322,7 +333,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
         }
       }
       // broadcast: the round's (prefix, rem) is in this CTA's ctl
-      if (tid == 0) wait_at(bbarA, (uint32_t)(round & 1), &fail, p.status);
+      if (tid == 0) wait_at(bbarA, (uint32_t)(round & 1), &fail, p.status, p.wait_ns);
       __syncthreads();
       ok = fail == 0;
       prefix = ctl[0];
@@ -366,7 +377,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
     dsm_st(dst, (uint32_t)a);
     dsm_st(dst + 4u, (uint32_t)e);
   }
-  ok = cluster_phase(barA, phase, &fail, p.status) && ok;
+  ok = cluster_phase(barA, phase, &fail, p.status, p.wait_ns) && ok;
   if (tid == 0) {
     int a = 0, e = 0;
     if (ok)
@@ -427,10 +438,11 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
       for (int i = tid; i < n_sub; i += kThreads) {
         if (i < ev_tot) {
           const int r = ev_base + i;
-          if (r < p.max_evict) eout[r] = staging[i];  // guards: only inconsistent ranks
+          // the guards only matter after a wait gave up (inconsistent counts)
+          if (r >= 0 && r < p.max_evict) eout[r] = staging[i];
         } else {
           const int r = (sub0 - ev_base) + (i - ev_tot);  // kept before + local kept rank
-          if (r < p.max_keep) kout[r] = staging[i];
+          if (r >= 0 && r < p.max_keep) kout[r] = staging[i];
         }
       }
       __syncthreads();
@@ -443,13 +455,34 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
       for (int i = E + tid; i < p.max_evict; i += kThreads) eout[i] = -1;
     }
   }
-  // rank 0's histograms and every CTA's counters outlive every remote access
-  cluster_phase(barA, phase, &fail, p.status);
+  // every CTA learns whether any CTA of the segment gave up a wait
+  __syncthreads();
+  if (tid < kC) dsm_st(mapa(smem_addr(&fails[rank]), (uint32_t)tid), fail != 0 ? 1u : 0u);
+  // The hardware cluster barrier, not a bounded phase: no CTA may exit while
+  // another can still address its shared memory, even after a wait gave up
+  // (the waits' limits can expire at different times).  Every thread of every
+  // CTA reaches it after finitely many bounded waits.
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+  bool any = fail != 0;
+  for (int r = 0; r < kC; ++r) any = any || fails[r] != 0;
+  if (any) {
+    // this CTA's share of the slots; the shares of the kC CTAs cover them all
+    int32_t* kout = keep_idx + (size_t)seg * p.max_keep;
+    int32_t* eout = evict_idx + (size_t)seg * p.max_evict;
+    const int kc = (p.max_keep + kC - 1) / kC, ec = (p.max_evict + kC - 1) / kC;
+    const int k0 = min(p.max_keep, (int)rank * kc), k1 = min(p.max_keep, k0 + kc);
+    const int e0 = min(p.max_evict, (int)rank * ec), e1 = min(p.max_evict, e0 + ec);
+    for (int i = k0 + tid; i < k1; i += kThreads) kout[i] = -1;
+    for (int i = e0 + tid; i < e1; i += kThreads) eout[i] = -1;
+  }
 }
 
 SelParams make_params(int B, int Hkv, int n_max, const int32_t* L, const int32_t* keep,
                       int max_keep, int max_evict, int32_t* status) {
   SelParams p;
+  p.stall_rank = -1;
+  p.wait_ns = kWaitNs;
   p.B = B;
   p.Hkv = Hkv;
   p.n_max = n_max;
@@ -471,12 +504,14 @@ size_t select_workspace_bytes(int, int, int) { return 256; }
 
 int select_launch_count() { return 1; }
 
-// L, keep: host arrays of B <= kMaxB rows.
-cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const int32_t* L,
-                          const int32_t* keep, int32_t* keep_idx, int32_t max_keep,
-                          int32_t* evict_idx, int32_t max_evict, void* ws, cudaStream_t st) {
-  int32_t* status = reinterpret_cast<int32_t*>(ws);
+namespace {
+cudaError_t launch_impl(int B, int Hkv, int n_max, const float* scores, const int32_t* L,
+                        const int32_t* keep, int32_t* keep_idx, int32_t max_keep,
+                        int32_t* evict_idx, int32_t max_evict, int32_t* status, int stall_rank,
+                        uint64_t wait_ns, cudaStream_t st) {
   SelParams p = make_params(B, Hkv, n_max, L, keep, max_keep, max_evict, status);
+  p.stall_rank = stall_rank;
+  p.wait_ns = wait_ns;
   int max_L = 0;
   for (int b = 0; b < B; ++b) max_L = L[b] > max_L ? L[b] : max_L;
   const long long span = (((long long)max_L + kC - 1) / kC + 31) & ~31ll;
@@ -487,9 +522,29 @@ cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const 
   auto kern = p.cache ? k_select<true> : k_select<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(status, 0, sizeof(int32_t), st)) != cudaSuccess) return e;
   kern<<<B * Hkv * kC, kThreads, smem, st>>>(p, scores, keep_idx, evict_idx);
   return cudaGetLastError();
+}
+}  // namespace
+
+// L, keep: host arrays of B <= kMaxB rows.
+cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const int32_t* L,
+                          const int32_t* keep, int32_t* keep_idx, int32_t max_keep,
+                          int32_t* evict_idx, int32_t max_evict, int32_t* status,
+                          cudaStream_t st) {
+  return launch_impl(B, Hkv, n_max, scores, L, keep, keep_idx, max_keep, evict_idx, max_evict,
+                     status, -1, kWaitNs, st);
+}
+
+// Self-test: CTA rank 1 of every cluster withholds its first gather arrival,
+// so rank 0's wait for it runs out after wait_ns (and later waits of the
+// segment may too); the kernel then reports the timeout and fills -1.
+cudaError_t launch_select_stalled(int B, int Hkv, int n_max, const float* scores,
+                                  const int32_t* L, const int32_t* keep, int32_t* keep_idx,
+                                  int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
+                                  int32_t* status, uint64_t wait_ns, cudaStream_t st) {
+  return launch_impl(B, Hkv, n_max, scores, L, keep, keep_idx, max_keep, evict_idx, max_evict,
+                     status, 1, wait_ns, st);
 }
 
 }  // namespace dropkv

@@ -199,7 +199,10 @@ k_simt_pass2(const T* __restrict__ q, const T* __restrict__ k, const T* __restri
           continue;
         }
         const A den = l - e;  // (1 - p_j) * l
-        if (!(den > A(0))) {  // p_j rounds to 1: removal is singular
+        // p_j rounds to 1 (in fp32, the precision of the stored inputs, also
+        // when the arithmetic is fp64) or its complement is not positive:
+        // removal is singular
+        if (!(den > A(0)) || (float)(e / l) == 1.0f) {
           atomicMax(status, kStatusSingular);
           continue;
         }

@@ -1069,8 +1069,8 @@ void tc_splits(const Lens& lens, int units_per_row, int budget, int32_t* splits)
 
 cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k, const void* v,
                              const Lens& lens, const ScoresLayout& lay, char* ws, float* attn_out,
-                             float* stats_out, int32_t* status, int score, cudaStream_t st,
-                             KernelEvents& kev) {
+                             float* stats_out, int32_t* status, int score, int cta_budget,
+                             cudaStream_t st, KernelEvents& kev) {
   const bool attn_only = score == DROPKV_SCORE_ATTENTION;
   auto pass2 = attn_only ? k_tc_pass2<true> : k_tc_pass2<false>;
   const TcPlan plan = tc_plan(s);
@@ -1086,7 +1086,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   a.chunks = plan.chunks;
   for (int i = 0; i < lens.B; ++i) a.L[i] = lens.L[i];
   const int units = s.Hkv * plan.chunks;
-  const int budget = std::min(num_sms(), kMaxCtas);
+  const int budget = std::min(cta_budget > 0 ? cta_budget : num_sms(), kMaxCtas);
   tc_splits(lens, units, std::max(budget, units * lens.B), a.splits);
   a.cta_base[0] = 0;
   for (int i = 0; i < lens.B; ++i) a.cta_base[i + 1] = a.cta_base[i] + units * a.splits[i];

@@ -59,3 +59,26 @@ def assert_select_exact(gpu_scores, lengths, keep, gpu_keep, gpu_evict, what="")
                                      max_keep=gpu_keep.shape[2], max_evict=gpu_evict.shape[2])
     assert np.array_equal(ref_keep, gpu_keep), f"{what}: keep lists differ"
     assert np.array_equal(ref_ev, gpu_evict), f"{what}: evict lists differ"
+
+
+def dominant_key_case(tau, *, dtype, d, L, Hq, Hkv=1, w=1, seed=9):
+    """One dominant key at position 0 whose probability misses 1 by about tau
+    for every window query: q rows are the unit vector e_0, key 0 is
+    x0 sqrt(d) e_0 with x0 = ln((L - 1)(1 - tau) / tau), every other key is 0
+    (logit 0), values are N(0, 1).  Returns (q, k, v, tau_exact) where
+    tau_exact = 1 - p_0 of the first window query, computed in fp64 from the
+    stored tensors (the later window queries see more zero keys, so their
+    1 - p_0 is a little larger)."""
+    import torch
+    P = L - w  # position of the first window query: it sees keys 0..P
+    x0 = np.log(P * (1.0 - tau) / tau)
+    q = torch.zeros(1, Hq, w, d, dtype=torch.float64)
+    q[..., 0] = 1.0
+    k = torch.zeros(1, Hkv, L, d, dtype=torch.float64)
+    k[:, :, 0, 0] = x0 * np.sqrt(d)
+    g = torch.Generator().manual_seed(seed)
+    v = torch.randn(1, Hkv, L, d, generator=g, dtype=torch.float64)
+    q, k, v = q.to(dtype), k.to(dtype), v.to(dtype)
+    logit0 = float(k[0, 0, 0, 0].double()) * float(q[0, 0, 0, 0].double()) / np.sqrt(d)
+    s = P * np.exp(-logit0)  # the other P visible keys have logit 0
+    return q, k, v, s / (1.0 + s)

@@ -26,7 +26,7 @@ def _declared():
 def test_header_declares_the_entry_points():
     names = set(_declared())
     assert {"dropkv_scores", "dropkv_scores_async", "dropkv_scores_ex", "dropkv_select",
-            "dropkv_scores_workspace_bytes", "dropkv_select_workspace_bytes",
+            "dropkv_select_ex", "dropkv_scores_workspace_bytes", "dropkv_select_workspace_bytes",
             "dropkv_status_string", "dropkv_abi_version"} <= names
 
 
@@ -200,3 +200,49 @@ def test_noalloc_select_rejects_bad_arguments_on_the_host():
     assert fn(2, 4, 100, odd, lens, keep_ok, fake, 10, fake, 90, None) == dk.ERR_ARG
     if not torch.cuda.is_available():
         assert fn(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, None) == dk.ERR_UNSUPPORTED
+
+
+def test_negative_cta_budget_is_rejected_on_the_host():
+    s = _shape()
+    fake = ctypes.c_void_p(0x100000)
+    opts = dk.Options(dk.PATH_AUTO, dk.SCORE_PERTURBATION, None, None, None, 0, -1)
+    assert dk.lib().dropkv_scores_ex(ctypes.byref(s), fake, fake, fake, None, fake, fake,
+                                     1 << 30, None, None, ctypes.byref(opts)) == dk.ERR_ARG
+
+
+def test_select_ex_rejects_bad_arguments_on_the_host():
+    L = dk.lib()
+    fake = ctypes.c_void_p(0x100000)
+    lens = (ctypes.c_int32 * 2)(100, 50)
+    keep_ok = (ctypes.c_int32 * 2)(10, 5)
+    keep_bad = (ctypes.c_int32 * 2)(10, 51)
+    ws = dk.select_workspace_bytes(2, 4, 100)
+    assert L.dropkv_select_ex(2, 4, 100, fake, lens, keep_bad, fake, 64, fake, 90, fake, ws,
+                              None, fake) == dk.ERR_ARG
+    assert L.dropkv_select_ex(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, fake, ws,
+                              None, ctypes.c_void_p(0x100002)) == dk.ERR_ARG  # status misaligned
+    assert L.dropkv_select_ex(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, fake, ws - 1,
+                              None, fake) == dk.ERR_WORKSPACE
+    if not torch.cuda.is_available():
+        for status in (None, fake):
+            assert L.dropkv_select_ex(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, fake,
+                                      ws, None, status) == dk.ERR_UNSUPPORTED
+
+
+def test_select_selftest_rejects_bad_arguments_on_the_host():
+    L = dk.lib()
+    fake = ctypes.c_void_p(0x100000)
+    lens = (ctypes.c_int32 * 2)(100, 50)
+    keep_ok = (ctypes.c_int32 * 2)(10, 5)
+    fn = L.dropkv_selftest_select_timeout
+    assert fn(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, None, 1000, None) == dk.ERR_ARG
+    assert fn(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, fake, 0, None) == dk.ERR_ARG
+    assert fn(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, fake, 2_000_000_000,
+              None) == dk.ERR_ARG
+    lens65 = (ctypes.c_int32 * 65)(*([100] * 65))
+    keep65 = (ctypes.c_int32 * 65)(*([10] * 65))
+    assert fn(65, 1, 100, fake, lens65, keep65, fake, 10, fake, 90, fake, 1000,
+              None) == dk.ERR_ARG  # one launch slice at most
+    if not torch.cuda.is_available():
+        assert fn(2, 4, 100, fake, lens, keep_ok, fake, 10, fake, 90, fake, 1000,
+                  None) == dk.ERR_UNSUPPORTED

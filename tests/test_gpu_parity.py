@@ -15,7 +15,8 @@ import oracle
 import kv_cache_eviction_scores_b200 as dk
 from kv_cache_eviction_scores_b200 import workloads as W
 
-from parity import assert_evict_sets_match, assert_scores_close, assert_select_exact
+from parity import (assert_evict_sets_match, assert_scores_close, assert_select_exact,
+                    dominant_key_case)
 
 pytestmark = pytest.mark.gpu
 
@@ -73,39 +74,8 @@ def test_small_configs(idx):
         _check_whole(wl, TOL_BF16, path, f"{spec.name} {path}")
 
 
-# ---- full-size configurations, sampled against the oracle -----------------
-
-def _sample_positions(spec, wl, b, h, rng):
-    L, w = wl.lengths[b], spec.window
-    pos = set(range(0, 6)) | set(range(L - w - 6, L)) | {127, 128, 129, L // 2}
-    pos |= set(int(x) for x in rng.integers(0, L, size=24))
-    if "heavy_positions" in wl.extras:
-        pos |= set(int(x) for x in wl.extras["heavy_positions"][b, h])
-    return sorted(p for p in pos if 0 <= p < L)
-
-
-@pytest.mark.parametrize("idx", [1, 2, 3, 4])
-def test_full_configs_sampled(idx):
-    spec = W.config_spec(idx)
-    wl = W.generate(spec, 42)
-    rng = np.random.default_rng(idx)
-    G = spec.G
-    heads = [(0, 0), (spec.B - 1, spec.Hkv - 1)]
-    for path in _paths(spec):
-        s, keep_idx, ev_idx = _run(wl, path)
-        for b in range(spec.B):
-            L = wl.lengths[b]
-            assert np.all(np.isnan(s[b, :, L:])), "padding must be NaN"
-            assert np.all(np.isposinf(s[b, :, L - spec.window: L])), "window must be +inf"
-            assert np.all(np.isfinite(s[b, :, : L - spec.window]))
-        for (b, h) in heads:
-            L = wl.lengths[b]
-            pos = _sample_positions(spec, wl, b, h, rng)
-            ref = oracle.scores_at(wl.q[b, h * G:(h + 1) * G], wl.k[b, h, :L], wl.v[b, h, :L],
-                                   spec.window, spec.pool, pos)
-            assert_scores_close(s[b, h, pos], ref, TOL_BF16, f"{spec.name} {path} ({b},{h})")
-        assert_select_exact(s, wl.lengths, wl.keep, keep_idx, ev_idx, f"{spec.name} {path}")
-
+# The full-size configurations are compared whole, with the oracle's evict
+# sets, in tests/test_gpu_full.py.
 
 # ---- edge cases -------------------------------------------------------------
 
@@ -171,6 +141,56 @@ def test_singular_input_is_rejected(dtype):
         torch.cuda.synchronize()
         assert int(status.item()) == dk.ERR_SINGULAR
     assert dk.auto_path(shape) in (dk.PATH_SIMT, dk.PATH_TENSOR)
+
+
+# The rule at its boundary (write-up, Algorithm 1 paragraph: rejected, no
+# epsilon).  fp32 inputs run in fp64 on the SIMT path, which applies the
+# oracle's reading exactly: p_j rounding to 1 in fp32 (1 - p <= 2^-25) is
+# singular, 1 - p = 4e-8 (rounds to 1 - 2^-24) is scored, at 1e-6.
+@pytest.mark.parametrize("tau,singular", [(1e-6, False), (4e-8, False), (2.5e-8, True),
+                                          (1e-9, True)])
+def test_singular_boundary_fp32_simt(tau, singular):
+    L, w = 40, 1
+    q, k, v, t = dominant_key_case(tau, dtype=torch.float32, d=1, L=L, Hq=1, w=w)
+    assert (np.float32(1.0 - t) == np.float32(1.0)) == singular
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    if singular:
+        with pytest.raises(oracle.SingularError):
+            oracle.scores(q, k, v, [L], w, 1)
+        with pytest.raises(dk.SingularError):
+            dk.dropkv_scores(qd, kd, vd, w, 1, [L], path="simt")
+        return
+    ref = oracle.scores(q, k, v, [L], w, 1)
+    s = dk.dropkv_scores(qd, kd, vd, w, 1, [L], path="simt")
+    torch.cuda.synchronize()
+    assert_scores_close(s.cpu().numpy(), ref, TOL_F32, f"tau {tau}")
+
+
+# On the fp32-arithmetic paths (bf16 inputs: SIMT and tensor core) the rule is
+# the fp32 complement L - e not > 0.  Where it can differ from the oracle's
+# (1 - p within a few fp32 ulps of 2^-25) the fp32 paths cannot score to 1e-3
+# anyway, so the margins are: 1 - p ~ 1e-9 must be rejected, and p ~ 0.9
+# (1 - p ~ 0.1) must be scored to the bf16 tolerance.
+@pytest.mark.parametrize("tau,singular", [(0.1, False), (1e-9, True)])
+def test_singular_boundary_bf16(tau, singular):
+    L, w, Hq = 200, 1, 16  # G * w = 16: the tensor-core shape
+    q, k, v, t = dominant_key_case(tau, dtype=torch.bfloat16, d=128, L=L, Hq=Hq, w=w)
+    spec = W.Spec("dominant", 1, Hq, 1, 128, [L], w, 1, [10], "bf16")
+    paths = _paths(spec)
+    assert "tensor" in paths
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    if singular:
+        with pytest.raises(oracle.SingularError):
+            oracle.scores(q, k, v, [L], w, 1)
+        for path in paths:
+            with pytest.raises(dk.SingularError):
+                dk.dropkv_scores(qd, kd, vd, w, 1, [L], path=path)
+        return
+    ref = oracle.scores(q, k, v, [L], w, 1)
+    for path in paths:
+        s = dk.dropkv_scores(qd, kd, vd, w, 1, [L], path=path)
+        torch.cuda.synchronize()
+        assert_scores_close(s.cpu().numpy(), ref, TOL_BF16, f"tau {tau} {path}")
 
 
 def test_nonsingular_async_status_is_ok():

@@ -1,5 +1,5 @@
 """Joint-removal objective on tiny inputs: DropKV's evicted set against the
-brute-force optimum (CPU only).
+brute-force optimum, from the oracle (CPU) and from the GPU path.
 
 The write-up ("DropKV：精确单项输出扰动评分组件", sections 核心公式 and
 结果与独立对照) scores every token by the exact output change its removal
@@ -15,7 +15,11 @@ deleted.  Here:
   the oracle's eviction must be the brute-force optimum (exact pin);
 * for |S| = 2, 3 the ratio J(S_dropkv) / min_S J(S) is >= 1; the pages quote a
   median ratio on real models, which synthetic inputs do not reproduce, so
-  the ratio itself is only reported.
+  the ratio itself is only reported;
+* on the GPU (``-m gpu``), the evicted set that the CUDA path selects from its
+  own scores is the oracle's evicted set, and for |S| = 1 the brute-force
+  optimum (fp32 inputs on the fp64 SIMT path; bf16 inputs on the tensor-core
+  path, where the set may differ only by a tie within the bf16 tolerance).
 """
 
 import itertools
@@ -24,6 +28,8 @@ import numpy as np
 import pytest
 
 import oracle
+
+from parity import assert_evict_sets_match
 
 G, HKV, D, L, W = 2, 1, 4, 11, 2          # history tokens [0, L - W) are evictable
 HIST = L - W
@@ -105,3 +111,63 @@ def test_multi_eviction_ratio_against_brute_force(n_evict):
         ratios.append(J_drop / J_opt)
     print(f"|S| = {n_evict}: J(DropKV) / J(optimum) over 6 seeds: "
           f"median {np.median(ratios):.3f}, max {max(ratios):.3f}")
+
+
+# ---- the GPU path's evicted set ------------------------------------------------
+
+def _dev_evicted(q, k, v, n_evict, L, w, path):
+    import torch
+    import kv_cache_eviction_scores_b200 as dk
+    qd, kd, vd = (torch.as_tensor(x).cuda() for x in (q, k, v))
+    s, _, ev = dk.evict(qd, kd, vd, w, 1, [L - n_evict], [L], path=path)
+    torch.cuda.synchronize()
+    return ev.cpu().numpy()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("path", ["auto", "simt"])
+@pytest.mark.parametrize("seed", range(6))
+def test_gpu_evicted_set_is_the_oracles_and_the_single_optimum(path, seed):
+    q, k, v = (x.astype(np.float32) for x in _inputs(seed))  # the stored fp32 inputs
+    q64, k64, v64 = (x.astype(np.float64) for x in (q, k, v))
+    J = np.array([joint_objective(q64, k64, v64, (j,)) for j in range(HIST)])
+    for n_evict in (1, 2, 3):
+        ev = _dev_evicted(q, k, v, n_evict, L, W, path)
+        assert tuple(int(j) for j in ev[0, 0]) == dropkv_evicted(q64, k64, v64, n_evict)
+        if n_evict == 1:
+            assert int(ev[0, 0, 0]) == int(np.argmin(J))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(3))
+def test_gpu_tensor_path_single_eviction_is_the_optimum(seed):
+    import torch
+    # tensor-core shape: bf16, d = 128, G * w = 16, 140 tokens (two tiles)
+    Gt, wt, Lt, d = 8, 2, 140, 128
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(1, Gt, wt, d, generator=g).to(torch.bfloat16)
+    k = (torch.randn(1, 1, Lt, d, generator=g) * 1.3).to(torch.bfloat16)
+    v = torch.randn(1, 1, Lt, d, generator=g).to(torch.bfloat16)
+    q64, k64, v64 = (x.double().numpy() for x in (q, k, v))
+    hist = Lt - wt
+    J = np.empty(hist)
+    for j in range(hist):
+        keep = np.ones(Lt, dtype=bool)
+        keep[j] = False
+        tot = 0.0
+        for hq in range(Gt):
+            for t in range(wt):
+                P = Lt - wt + t
+                a, _ = _softmax_out(q64[0, hq, t], k64[0, 0, : P + 1], v64[0, 0, : P + 1])
+                a_s, _ = _softmax_out(q64[0, hq, t], k64[0, 0, : P + 1][keep[: P + 1]],
+                                      v64[0, 0, : P + 1][keep[: P + 1]])
+                tot += float(np.sum((a_s - a) ** 2))
+        J[j] = tot
+    ref = oracle.scores(q, k, v, [Lt], wt, 1)
+    np.testing.assert_allclose(ref[0, 0, :hist], J / Gt, rtol=1e-9)  # score = J({j}) / G
+    ev = _dev_evicted(q, k, v, 1, Lt, wt, "tensor")
+    # the GPU's choice is the optimum unless the two best are a bf16-tolerance tie
+    assert_evict_sets_match(ev, ref, [Lt], [Lt - 1], 1e-3, "tensor single eviction")
+    order = np.argsort(J)
+    if J[order[1]] > J[order[0]] * (1 + 2e-3):
+        assert int(ev[0, 0, 0]) == int(order[0])

@@ -234,6 +234,48 @@ def test_peaked_but_nonsingular_input_is_accepted():
     assert np.all(np.isfinite(s[0, 0, : L - w]))
 
 
+# The rule at its boundary: "rounds to 1" is the fp32 rounding of the exact
+# p_j (the inputs' precision), with no epsilon.  fp32 has 1 - 2^-24 as its
+# largest value below 1, so p rounds to 1 exactly when 1 - p <= 2^-25 (the
+# midpoint rounds to even, i.e. to 1).  A threshold rule such as
+# p > 1 - 1e-5 or p > 1 - 1e-7 fails the accepted cases below, and a rule
+# that only catches exact cancellation (1 - p == 0 in fp64) fails the
+# rejected ones.
+BOUNDARY = [
+    (1e-6, False),      # far below the boundary in fp32 terms: scored
+    (4e-8, False),      # between 2^-25 and 2^-24: rounds to 1 - 2^-24, scored
+    (2.5e-8, True),     # just above 1 - 2^-25: rounds to 1, rejected
+    (1e-9, True),       # rounds to 1, rejected
+]
+
+
+@pytest.mark.parametrize("tau,singular", BOUNDARY)
+def test_singular_rule_at_the_fp32_boundary(tau, singular):
+    from parity import dominant_key_case
+    L, w = 40, 1
+    q, k, v, t = dominant_key_case(tau, dtype=torch.float32, d=1, L=L, Hq=1, w=w)
+    assert (np.float32(1.0 - t) == np.float32(1.0)) == singular  # the construction
+    assert abs(t - tau) <= 0.01 * tau
+    if singular:
+        with pytest.raises(oracle.SingularError):
+            oracle.scores(q, k, v, [L], w, 1)
+        _, _, _, st, where = oracle.raw_scores(q, k, v, [L], raise_singular=False)
+        assert st == oracle.ERR_SINGULAR and where[3] == 0
+        return
+    raw, _, _, st, _ = oracle.raw_scores(q, k, v, [L])
+    assert st == oracle.OK
+    # the accepted case is scored exactly: closed form against deletion.  For
+    # the dominant token both sides lose about 1e-16 / tau of relative
+    # precision in 1 - p (squared in the score); for the others deletion
+    # subtracts two O(1) outputs that differ by about p_j, so it carries a
+    # relative error of order 1e-16 / p_j (p_j about tau / 39 here)
+    bf = bruteforce.raw_scores(q.double().numpy(), k.double().numpy(), v.double().numpy(), [L])
+    np.testing.assert_allclose(raw[0, 0, 0], bf[0, 0, 0], rtol=1e-7)
+    np.testing.assert_allclose(raw[0, 0, 1:L], bf[0, 0, 1:L], rtol=1e-4)
+    # the dominant token's perturbation is about ||mean of the others - v_0||^2
+    assert raw[0, 0, 0] > 1e-3
+
+
 def test_argument_errors():
     wl = W.generate(W.config_spec(0), 42)
     with pytest.raises(ValueError):

@@ -5,8 +5,9 @@ its own pool (or a path that cannot afford cudaMalloc's implicit device
 synchronisation) cannot hand dropkv_select a workspace.  dropkv_select_noalloc
 takes none and uses a 4 KiB scratch array compiled into the library.  This
 test calls it through the C ABI twice in a row and checks that both calls give
-exactly the keep / evict lists of dropkv_select (integer outputs: exact), also
-for a launch of more than 64 batch rows (sliced on the host).
+exactly the keep / evict lists of dropkv_select and of the oracle's selection
+on the same scores (integer outputs: exact), also for a launch of more than 64
+batch rows (sliced on the host).
 
 The file is named so that pytest collects it last.
 """
@@ -18,6 +19,7 @@ import pytest
 import torch
 
 import kv_cache_eviction_scores_b200 as dk
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +57,7 @@ def test_noalloc_select_matches_select_on_two_calls_in_a_row():
     ref_keep, ref_ev = dk.dropkv_select(scores, keep, lengths)
     torch.cuda.synchronize()
     max_keep, max_evict = ref_keep.shape[2], ref_ev.shape[2]
+    o_keep, o_ev = oracle.select(scores.cpu().numpy(), lengths, keep, max_keep, max_evict)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for call in range(2):
         keep_idx = torch.full((B, Hkv, max_keep), 7, dtype=torch.int32, device=DEV)
@@ -66,6 +69,8 @@ def test_noalloc_select_matches_select_on_two_calls_in_a_row():
         torch.cuda.synchronize()
         assert torch.equal(keep_idx, ref_keep), f"call {call}: keep lists differ"
         assert torch.equal(ev_idx, ref_ev), f"call {call}: evict lists differ"
+        assert np.array_equal(keep_idx.cpu().numpy(), o_keep), f"call {call}: keep vs oracle"
+        assert np.array_equal(ev_idx.cpu().numpy(), o_ev), f"call {call}: evict vs oracle"
 
 
 def test_noalloc_select_many_rows_matches_select():
@@ -86,3 +91,6 @@ def test_noalloc_select_many_rows_matches_select():
     assert st == dk.OK
     torch.cuda.synchronize()
     assert torch.equal(keep_idx, ref_keep) and torch.equal(ev_idx, ref_ev)
+    o_keep, o_ev = oracle.select(scores.cpu().numpy(), lengths, keep, max_keep, max_evict)
+    assert np.array_equal(keep_idx.cpu().numpy(), o_keep)
+    assert np.array_equal(ev_idx.cpu().numpy(), o_ev)
