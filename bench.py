@@ -46,11 +46,15 @@ CSRC = os.path.join(ROOT, "kv_cache_eviction_scores_b200", "csrc")
 # kernel order per scoring call (must match the library's launch sequence)
 KERNELS = {
     "simt": ["k_simt_pass1", "k_simt_pass2", "k_epilogue"],
-    "tensor": ["k_tc_pass1", "k_tc_combine", "k_tc_pass2", "k_epilogue"],
+    # the DropKV score's second pass runs on CTA pairs; the attention-only
+    # control keeps the single-CTA second pass (K streamed alone)
+    "tensor": ["k_tc_pass1", "k_tc_combine", "k_tc_pass2_pair", "k_epilogue"],
+    "tensor_attention": ["k_tc_pass1", "k_tc_combine", "k_tc_pass2", "k_epilogue"],
 }
 KERNEL_SRC = {
     "k_simt_pass1": "simt.cu", "k_simt_pass2": "simt.cu", "k_epilogue": "epilogue.cu",
     "k_tc_pass1": "tc.cu", "k_tc_combine": "tc.cu", "k_tc_pass2": "tc.cu",
+    "k_tc_pass2_pair": "tc_pair.cu",
 }
 
 
@@ -105,6 +109,43 @@ def visible_elements(spec):
     w = spec.window
     per_query_head = sum(w * (L - w) + w * (w + 1) // 2 for L in spec.lengths)
     return per_query_head * spec.Hq
+
+
+def split_runs(lengths, units, budget, tile=128):
+    """Tile runs of the CTAs of one tensor-path pass: the library's split rule
+    (one more split to the batch row whose runs are longest while the CTA
+    budget allows), restated here to report the load balance."""
+    nts = [(L + tile - 1) // tile for L in lengths]
+    splits = [1] * len(lengths)
+    total = units * len(lengths)
+    budget = max(budget, total)
+    while True:
+        best, worst = -1, 0.0
+        for b, nt in enumerate(nts):
+            per = nt / splits[b]
+            if splits[b] < nt and per > worst:
+                best, worst = b, per
+        if best < 0 or total + units > budget:
+            break
+        splits[best] += 1
+        total += units
+    return [(sp + 1) * nt // splits[b] - sp * nt // splits[b]
+            for b, nt in enumerate(nts) for sp in range(splits[b])]
+
+
+def tensor_plan(spec, sms):
+    """CTA counts and per-CTA tile runs (min, max) of the two tensor-core
+    passes: pass 1 one CTA per (b, h, query chunk, split), the DropKV second
+    pass one CTA pair per (b, h, query chunk, split), each CTA of a pair
+    taking half of the pair's run."""
+    nq = spec.G * spec.window
+    units = spec.Hkv * ((nq + 255) // 256)
+    budget = min(sms, 160)
+    r1 = split_runs(spec.lengths, units, budget)
+    r2 = split_runs(spec.lengths, units, budget // 2)
+    h2 = [(x + 1) // 2 for x in r2]
+    return {"pass1_ctas": len(r1) * units, "pass1_tiles_per_cta": [min(r1), max(r1)],
+            "pass2_ctas": 2 * len(r2) * units, "pass2_tiles_per_cta": [min(h2), max(h2)]}
 
 
 # ----------------------------------------------------------- multi-rank ----
@@ -286,7 +327,7 @@ def roofline(kernel, spec, us, hbm_peak, tc_peak, sm_mhz, score="perturbation"):
                 "tensor": {"achieved": tach, "peak": tc_peak, "unit": "TFLOP/s",
                            "frac": tach / tc_peak,
                            "work": f"{flops:.4g} flop (2*d per visible element)"}}
-    if kernel in ("k_tc_pass1", "k_tc_pass2"):
+    if kernel in ("k_tc_pass1", "k_tc_pass2", "k_tc_pass2_pair"):
         # each pass streams K and V once: one read of the valid K and V rows is
         # the algorithmic traffic of a launch (2 tensors x d x 2 bytes per
         # (token, KV head)); the two contractions (4 d flop per visible element)
@@ -380,7 +421,7 @@ def run_ours(args):
                          dtype=torch.uint8, device=dev)
     scores = torch.empty(spec.B, spec.Hkv, spec.n_max, dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    names = KERNELS[path]
+    names = KERNELS["tensor_attention" if path == "tensor" and args.score == "attention" else path]
     nk = len(names)
 
     def step(events=None):
@@ -409,17 +450,32 @@ def run_ours(args):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
+    # the timed region: K whole steps back to back, only the two bracketing
+    # events on the stream (the kernels of a step may overlap one another's
+    # tails through programmatic dependent launch)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
     for i in range(K):
-        step(ev[i])
+        step()
     t1.record()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    clk = clocks.stop()
     ms = max_over_ranks(t0.elapsed_time(t1), dist, dev) / K
+    # the per-kernel breakdown: the same K steps again, with events recorded
+    # on the launching stream right before and after every kernel
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    b0.record()
+    for i in range(K):
+        step(ev[i])
+    b1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    ms_events = max_over_ranks(b0.elapsed_time(b1), dist, dev) / K
     kern_us = {}
     for j, name in enumerate(names):
         kern_us[name] = statistics.mean(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1])
@@ -465,6 +521,9 @@ def run_ours(args):
                 "nominal_gbs": NOMINAL_HBM_GBS},
         "phases_us": {"scores": sum(kern_us[n] for n in names),
                       "select": kern_us["select (all launches)"]},
+        "ms_per_step_with_kernel_events": ms_events,
+        "plan": (tensor_plan(spec, torch.cuda.get_device_properties(dev).multi_processor_count)
+                 if path == "tensor" else None),
         "roofline": roof,
         "kernels_us": kern_us,
         "e2e": e2e,

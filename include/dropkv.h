@@ -176,10 +176,10 @@ DROPKV_API size_t dropkv_select_workspace_bytes(int32_t B, int32_t Hkv, int32_t 
  *                then -1;  max_evict >= every lengths[b] - keep_counts[b].
  *                (keep_idx / evict_idx may be NULL when max_keep / max_evict is 0.)
  * Asynchronous on `stream`; integer results are exact.  The kernels' waits on
- * one another are bounded; if one gives up, that (b, h)'s lists are filled
- * with -1 (every slot, once the other CTAs of the segment have finished) and
- * DROPKV_ERR_TIMEOUT is recorded in the workspace, which only
- * dropkv_select_ex reports.
+ * one another are bounded; if one gives up, that (b, h)'s keep and evict
+ * slots are all filled with -1.  Only dropkv_select_ex reports the timeout
+ * itself (DROPKV_ERR_TIMEOUT); this entry point enqueues nothing but the
+ * selection kernel and leaves the workspace untouched.
  */
 DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
                             const int32_t* lengths, const int32_t* keep_counts,

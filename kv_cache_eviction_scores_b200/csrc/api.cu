@@ -70,8 +70,8 @@ bool tc_shape_ok(const dropkv_shape& s) {
   if (!tc_available()) return false;
   if (s.dtype != DROPKV_BF16 || s.d != 128 || s.n_max < 128) return false;
   const int nq = (s.Hq / s.Hkv) * s.window;
-  const int chunks = (nq + 127) / 128;
-  if (nq % (16 * chunks) != 0) return false;
+  const int chunks = (nq + 127) / 128, chunks2 = (nq + 255) / 256;
+  if (nq % (16 * chunks) != 0 || nq % (16 * chunks2) != 0) return false;
   return true;
 }
 
@@ -80,7 +80,10 @@ TcPlan tc_plan(const dropkv_shape& s) {
   const int nq = (s.Hq / s.Hkv) * s.window;
   p.chunks = (nq + 127) / 128;
   p.nqc = nq / p.chunks;
-  p.max_ctas = 0;
+  p.chunks1 = (nq + 255) / 256;
+  p.rows1 = (nq + p.chunks1 - 1) / p.chunks1;
+  p.chunks2 = (nq + 255) / 256;
+  p.nqc2 = nq / p.chunks2;
   return p;
 }
 
@@ -88,7 +91,8 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   ScoresLayout l;
   const size_t rows = (size_t)Bs * s.Hq * s.window;
   const bool tc = tc_shape_ok(s);
-  l.nparts = tc ? 4 * tc_plan(s).chunks : 1;  // tensor path: four column groups per chunk
+  // tensor path: four column groups per query chunk of either second pass
+  l.nparts = tc ? 4 * tc_plan(s).chunks : 1;
   size_t o = 0;
   l.status = o;
   o += kAlign;
@@ -102,10 +106,10 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
   if (tc) {
     const TcPlan p = tc_plan(s);
     // pass-1 partials: at most (split target + one per (b, h, chunk)) CTAs,
-    // two warpgroups each, 128 rows of (a[128], max, normaliser, pad).
-    const size_t ctas = (size_t)tc_split_target() + (size_t)Bs * s.Hkv * p.chunks;
+    // rows1 rows each of (a[128], max, normaliser, pad).
+    const size_t ctas = (size_t)tc_split_target() + (size_t)Bs * s.Hkv * p.chunks1;
     l.tc_partial = o;
-    o = align_up(o + ctas * 128 * 136 * sizeof(float), kAlign);
+    o = align_up(o + ctas * p.rows1 * kTcPartStride * sizeof(float), kAlign);
     l.tc_ahi = o;
     o = align_up(o + rows * s.d * 2, kAlign);
     l.tc_alo = o;
@@ -116,7 +120,7 @@ ScoresLayout scores_layout(const dropkv_shape& s, int Bs) {
     o = align_up(o + (size_t)Bs * s.Hkv * (size_t)((s.n_max + 127) / 128) * 128 * sizeof(float),
                  kAlign);
     l.tc_tmin = o;
-    o = align_up(o + (size_t)Bs * s.Hkv * (size_t)((s.n_max + 127) / 128) * p.chunks * sizeof(float),
+    o = align_up(o + (size_t)Bs * s.Hkv * (size_t)((s.n_max + 127) / 128) * p.chunks1 * sizeof(float),
                  kAlign);
   }
   l.total = o;
@@ -153,8 +157,10 @@ dropkv_status run_select(int32_t B, int32_t Hkv, int32_t n_max, const float* sco
                          const int32_t* lengths, const int32_t* keep_counts, int32_t* keep_idx,
                          int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
                          int32_t* status_word, cudaStream_t st) {
-  // one reset per call: a timeout in one launch slice stays visible after the next
-  if (cudaError_t e = cudaMemsetAsync(status_word, 0, sizeof(int32_t), st)) return cuda_fail(e);
+  // one reset per call: a timeout in one launch slice stays visible after the
+  // next (status_word NULL: the caller does not ask for the device status)
+  if (status_word)
+    if (cudaError_t e = cudaMemsetAsync(status_word, 0, sizeof(int32_t), st)) return cuda_fail(e);
   for (int b0 = 0; b0 < B; b0 += kMaxB) {
     const int Bs = (B - b0) < kMaxB ? (B - b0) : kMaxB;
     int32_t L[kMaxB], K[kMaxB];
@@ -244,11 +250,12 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
         kev.end(st);
       }
     } else {
+      int nparts = lay.nparts;
       e = launch_tc_scores(s, qs, ks, vs, lens, lay, ws, attn_user, stats_user, status_word, score,
-                           tc_ctas, st, kev);
+                           tc_ctas, st, kev, &nparts);
       if (e == cudaSuccess) {
         kev.begin(st);
-        e = launch_epilogue(s, lens, parts, lay.nparts, part_stride, sc, st);
+        e = launch_epilogue(s, lens, parts, nparts, part_stride, sc, st);
         kev.end(st);
       }
     }
@@ -320,7 +327,9 @@ static dropkv_status select_entry(int32_t B, int32_t Hkv, int32_t n_max, const f
   r = check_device();
   if (r != DROPKV_OK) return r;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int32_t* status_word = status_dev ? status_dev : reinterpret_cast<int32_t*>(workspace);
+  // the plain entry point reports no device status: nothing to reset or record
+  int32_t* status_word =
+      status_dev ? status_dev : (sync ? reinterpret_cast<int32_t*>(workspace) : nullptr);
   r = run_select(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx, max_keep, evict_idx,
                  max_evict, status_word, st);
   if (r != DROPKV_OK || !sync) return r;

@@ -11,6 +11,17 @@ namespace dropkv {
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may begin while its predecessor in the
+// stream is still running: pdl_wait() returns once the predecessor grid has
+// completed and its memory writes are visible (at once when there is no such
+// predecessor).  pdl_trigger() lets the successor grid begin launching early;
+// the successor still waits in its own pdl_wait() for this grid to finish.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Warp reductions over all 32 lanes.
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll

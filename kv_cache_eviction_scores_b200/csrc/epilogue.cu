@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(kThreads)
 k_epilogue(const float* __restrict__ parts, int nparts, size_t part_stride, Lens lens, int Hkv,
            int n_max, int w, int radius, float G, float* __restrict__ scores) {
   extern __shared__ float merged[];  // radius + kTile + radius
+  pdl_trigger();
+  pdl_wait();  // the partial planes come from the previous kernel
   const int bh = blockIdx.y, b = bh / Hkv;
   const int L = lens.L[b];
   const int j0 = blockIdx.x * kTile;
@@ -94,9 +96,8 @@ cudaError_t launch_epilogue(const dropkv_shape& s, const Lens& lens, const float
     if (e != cudaSuccess) return e;
   }
   dim3 grid((s.n_max + kTile - 1) / kTile, lens.B * s.Hkv);
-  k_epilogue<<<grid, kThreads, smem, st>>>(parts, nparts, part_stride, lens, s.Hkv, s.n_max,
-                                        s.window, radius, (float)(s.Hq / s.Hkv), scores);
-  return cudaGetLastError();
+  return launch_ex(k_epilogue, grid, dim3(kThreads), smem, st, true, 1, parts, nparts, part_stride,
+                   lens, s.Hkv, s.n_max, s.window, radius, (float)(s.Hq / s.Hkv), scores);
 }
 
 }  // namespace dropkv

@@ -37,6 +37,37 @@ struct KernelEvents {
   }
 };
 
+// Launches `kern` on `st`; with pdl = true the launch carries the programmatic
+// stream-serialization attribute, so that it may overlap the tail of the
+// previous kernel in the stream (the kernel must call pdl_wait() before it
+// reads that kernel's results).  cluster_x > 1 launches clusters of that size.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, bool pdl, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = n ? attr : nullptr;
+  cfg.numAttrs = (unsigned)n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // ---- scoring: workspace carve-up ------------------------------------------
 struct ScoresLayout {
   size_t status;     // int32 status word (sync variant)
@@ -48,17 +79,22 @@ struct ScoresLayout {
   size_t tc_alo;     // bf16 [B, Hq, w, d] low part of a (tensor path)
   size_t tc_qstat;   // fp32 [B, Hq, w, 4] per-query pass-2 constants (tensor path)
   size_t tc_nv;      // fp32 [B, Hkv, ceil(n_max/128)*128] ||v_j||^2 (tensor path, pass 1 -> pass 2)
-  size_t tc_tmin;    // fp32 [B, Hkv, ceil(n_max/128), chunks] min ||v_j||^2 per tile share
+  size_t tc_tmin;    // fp32 [B, Hkv, ceil(n_max/128), chunks1] min ||v_j||^2 per tile share
   size_t total;
   int nparts;
 };
 
 // Tensor-path plan for one batch slice.
 struct TcPlan {
-  int chunks;        // query chunks per KV head (G*w split into chunks of nqc rows)
-  int nqc;           // rows per chunk (multiple of 16, <= 128)
-  int max_ctas;      // upper bound of pass-1 CTAs (sizes the partial buffer)
+  int chunks;        // pass-2 query chunks per KV head (G*w split into chunks of nqc rows)
+  int nqc;           // rows per pass-2 chunk (multiple of 16, <= 128)
+  int chunks1;       // pass-1 query chunks per KV head (two 128-row query tiles each)
+  int rows1;         // rows per pass-1 chunk (<= 256; the last chunk may be shorter)
+  int chunks2;       // CTA-pair pass-2 query chunks per KV head
+  int nqc2;          // rows per pair chunk (multiple of 16, <= 256)
 };
+// floats per pass-1 partial row: O[128], max, normaliser, padding
+constexpr int kTcPartStride = 132;
 
 bool tc_shape_ok(const dropkv_shape& s);
 // DROPKV_OK when the current device is an sm_100 part the kernels run on.
@@ -81,12 +117,14 @@ cudaError_t launch_epilogue(const dropkv_shape& s, const Lens& lens, const float
                             int nparts, size_t part_stride, float* scores, cudaStream_t st);
 
 // Tensor-core path (tcgen05 + TMA); returns cudaErrorNotSupported when the
-// tensor maps cannot be encoded.
+// tensor maps cannot be encoded.  *nparts_used receives how many partial-score
+// planes per (b, h) the second pass wrote (the epilogue sums them).
 // cta_budget: most CTAs per pass (0 = one per SM).
 cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k,
                              const void* v, const Lens& lens, const ScoresLayout& lay,
                              char* ws, float* attn_out, float* stats_out, int32_t* status,
-                             int score, int cta_budget, cudaStream_t st, KernelEvents& kev);
+                             int score, int cta_budget, cudaStream_t st, KernelEvents& kev,
+                             int* nparts_used);
 int tc_launch_count();
 int tc_split_target();
 bool tc_available();

@@ -55,7 +55,7 @@ struct SelParams {
   int32_t max_keep, max_evict;
   int32_t L[kMaxB];
   int32_t E[kMaxB];                  // evictions per row
-  int32_t* status;                   // device status word (0 = OK)
+  int32_t* status;                   // device status word (0 = OK), or NULL: not reported
   int32_t cache;                     // 1: every CTA's range fits one cached sub-range
   int32_t stall_rank;                // self-test only: this rank withholds its first
                                      // gather arrival (-1: none, the product path)
@@ -141,7 +141,7 @@ __device__ bool wait_at(uint32_t bar, uint32_t parity, volatile int* fail, int32
     if (done) return true;
     if (gtimer() - t0 > limit_ns) {
       *fail = 1;
-      atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
+      if (status) atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
       return false;
     }
   }
@@ -175,7 +175,7 @@ __device__ bool cluster_phase(uint32_t bar, int& phase, volatile int* fail, int3
       if (done) break;
       if (gtimer() - t0 > limit_ns) {
         *fail = 1;
-        atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
+        if (status) atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
         break;
       }
     }
@@ -206,6 +206,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   __shared__ __align__(8) uint64_t bbar;    // every CTA: rank 0 broadcast the round's digit (1)
   __shared__ uint32_t fails[kC];             // per rank: 1 if a wait of that CTA gave up
   __shared__ int fail;
+  pdl_wait();  // the scores may come from the previous kernel in the stream
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const uint32_t rank = cluster_rank();
   const int seg = blockIdx.x / kC;
@@ -522,8 +523,8 @@ cudaError_t launch_impl(int B, int Hkv, int n_max, const float* scores, const in
   auto kern = p.cache ? k_select<true> : k_select<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<B * Hkv * kC, kThreads, smem, st>>>(p, scores, keep_idx, evict_idx);
-  return cudaGetLastError();
+  return launch_ex(kern, dim3(B * Hkv * kC), dim3(kThreads), smem, st, true, 1, p, scores,
+                   keep_idx, evict_idx);
 }
 }  // namespace
 

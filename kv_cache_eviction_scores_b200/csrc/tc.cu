@@ -52,110 +52,16 @@
 
 #include <algorithm>
 
-#include "common.cuh"
-#include "internal.h"
-#include "tc_ptx.cuh"
+#include "tc_common.cuh"
 
 namespace dropkv {
 
 namespace {
 
-using namespace tc;
-
-constexpr int kTok = 128;          // tokens per tile
-constexpr int kHd = 128;           // head dim
-constexpr int kBox = 128 * 128;    // bytes of a 128-row x 64-col bf16 box (SW128)
-constexpr int kTileBytes = 2 * kBox;
-constexpr int kSimtWarps = 16;     // softmax / score warps: 4 per TMEM lane quarter
-constexpr int kWarpTma = kSimtWarps, kWarpMma = kSimtWarps + 1, kWarpNv = kSimtWarps + 2;
-constexpr int kThreads2 = (kSimtWarps + 2) * 32;  // pass 2: + TMA warp, MMA warp
-constexpr int kThreads1 = (kSimtWarps + 3) * 32;  // pass 1: + the ||v||^2 warp
-constexpr int kMaxRegs = 96;       // pass 1: 19 warps share the SM's 64K registers
-constexpr int kMaxRegs2 = 96;      // pass 2: 18 warps, 5 on a sub-partition (16K registers)
-constexpr uint32_t kColO = 384;    // pass-1 TMEM columns: three S/P buffers [0, 384), then O
-constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr int kPartStride = 136;   // floats per partial row: O[128], m, l (4 parts), pad
-constexpr int kMaxCtas = 160;      // split target ceiling (one CTA per SM)
-constexpr int kSt1 = 3;            // pass-1 V stages (HBM latency needs > 1 tile in flight)
-constexpr int kStK = 2;            // pass-1 K stages (S runs two tiles ahead of P V)
-constexpr int kBars1 = 1 + 2 * kStK + 2 * kSt1 + 13;  // pass-1 mbarriers
-constexpr int kRing2 = 5;          // pass-2 ring of 32 KB K/V slots (the last one doubles as A_lo)
-constexpr float kLoSkip = 8e-4f;   // pass 2 drops A_lo when ||A||^2 <= kLoSkip ||v||^2 throughout
-
-struct TcArgs {
-  int32_t B, Hq, Hkv, n_max, w, G, nqc, chunks;
-  int32_t qbox_rows;     // rows of the pass-1 Q box: min(128, all query rows)
-  int32_t L[kMaxB];
-  int32_t splits[kMaxB];
-  int32_t cta_base[kMaxB + 1];
-  float c_log2;          // log2(e) / sqrt(d)
-  const __nv_bfloat16* q;  // [rows][128] window queries
-  float* partial;        // [ctas][128][kPartStride]
-  int32_t* status;
-  __nv_bfloat16* ahi;    // [rows][128]
-  __nv_bfloat16* alo;    // [rows][128]
-  float4* qstat;         // [rows]: (M, 1/L, L, ||A||^2)
-  float* attn_user;      // optional [rows][128]
-  float* stats_user;     // optional [rows][2]
-  float* parts;          // [chunks][B*Hkv*n_max]
-  size_t part_stride;
-  float* attn_f32;       // [rows][128] fp32 window outputs a (read back by pass 2)
-  const __nv_bfloat16* v;  // [B*Hkv][n_max][128] values (rare direct-distance path)
-  float* nvbuf;          // [B*Hkv][ntmax*128] ||v_j||^2 (pass 1 -> pass 2), tile-padded rows
-  float* tmin;           // [B*Hkv][ntmax][chunks] min ||v_j||^2 over a chunk's share of a tile
-  int32_t ntmax;         // ceil(n_max / 128)
-};
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
-__device__ __forceinline__ uint32_t u32(float f) { return __float_as_uint(f); }
-__device__ __forceinline__ uint32_t pack_bf16_rn(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ void decode_cta(const TcArgs& a, int cta, int& b, int& h, int& chunk,
-                                           int& t0, int& t1) {
-  b = 0;
-  while (b + 1 < a.B && cta >= a.cta_base[b + 1]) ++b;
-  const int local = cta - a.cta_base[b];
-  const int sp = local % a.splits[b];
-  const int hc = local / a.splits[b];
-  h = hc / a.chunks;
-  chunk = hc % a.chunks;
-  const int nt = (a.L[b] + kTok - 1) / kTok;
-  t0 = (int)((long long)sp * nt / a.splits[b]);
-  t1 = (int)((long long)(sp + 1) * nt / a.splits[b]);
-}
-
-// Records a timeout once and raises the CTA-wide abort flag.
-__device__ __forceinline__ void fail(const TcArgs& a, volatile int* abort_flag) {
-  *abort_flag = 1;
-  atomicMax(a.status, (int)DROPKV_ERR_TIMEOUT);
-}
-// Bounded wait whose outcome is the same for every lane of the warp, so the
-// warp stays converged for the .sync.aligned tcgen05 instructions after it.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
-  const bool ok = mbar_wait(bar, parity, kWaitNs);
-  return __all_sync(0xffffffffu, ok);
-}
-__device__ __forceinline__ bool warp_aborted(volatile int* f) {
-  return __any_sync(0xffffffffu, *f != 0);
-}
-
-// Descriptor-word offset of the 16-wide K slice kk of a K-major SW128 operand
-// with `rows` rows (kmajor_desc's address offset >> 4).
-__device__ __forceinline__ uint32_t kslice(int kk, uint32_t rows) {
-  return (uint32_t)(kk >> 2) * rows * 8u + (uint32_t)(kk & 3) * 2u;
-}
 // =========================== pass 1 =========================================
-// Writes P = exp2(S c - mu) for one warp's 32 tokens of a query row (S already
-// in registers, masked keys at -inf) as hi/lo bf16 planes over the same 32
-// TMEM columns: tokens 16k..16k+15 keep hi in columns [16k, 16k+8) and lo in
+// Writes P = exp2(S c - mu) for 32 tokens of one query row (S already in
+// registers, masked keys at -inf) as hi/lo bf16 planes over the same 32 TMEM
+// columns: tokens 16k..16k+15 keep hi in columns [16k, 16k+8) and lo in
 // [16k+8, 16k+16).  Returns the row's sum of P over the 32 tokens.
 // Warp-collective.
 __device__ __forceinline__ float p1_exp32(const uint32_t (&sr)[32], uint32_t tS, uint64_t c2,
@@ -187,74 +93,88 @@ __device__ __forceinline__ float p1_exp32(const uint32_t (&sr)[32], uint32_t tS,
   return la + lb;
 }
 
-// Rare path of pass 1, out of line: the reference max moved for some lanes
-// (factor fac <= 1 for them, 1 for the others), so this warp's 32 columns of O
-// are rescaled once the P V that last accumulated into O has landed (waited on
-// through that P V's buffer barrier and parity).  Warp-collective.  Returns
-// false on a timeout.
+// Causal mask of 32 tokens starting at tok0 for a query at position prow.
+__device__ __forceinline__ void p1_mask32(uint32_t (&sr)[32], int tok0, int prow) {
+#pragma unroll
+  for (int u = 0; u < 32; ++u)
+    if (tok0 + u > prow) sr[u] = 0xFF800000u;  // -inf
+}
+
+// Rare path of pass 1, out of line: the reference max of some rows moved
+// (factor fac < 1 for them, 1 for the others), so the warp's 32 rows of O
+// (128 columns) are rescaled once the P V that last accumulated into O has
+// landed (waited on through that P V's barrier and parity).  Warp-collective.
+// Returns false on a timeout.
 __device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, uint32_t pd_bar,
                                           uint32_t parity) {
   if (!warp_wait(pd_bar, parity)) return false;
   tc_fence_after();
-  uint32_t o[32];
-  tmem_ld32(tO, o);
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[32];
+    tmem_ld32(tO + 32u * c, o);
 #pragma unroll
-  for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
-  tmem_st32(tO, o);
+    for (int u = 0; u < 32; ++u) o[u] = u32(f32(o[u]) * fac);
+    tmem_st32(tO + 32u * c, o);
+  }
+  tmem_st_wait();
   return true;
 }
 
-__global__ void __maxnreg__(kMaxRegs)
+// One CTA per (b, h, query chunk, token split).  The chunk's rows (<= 256)
+// are two query tiles of 128 rows; a K/V tile in shared memory serves both.
+// Tensor-pipe order per tile j: P V of tile 0, S of tile 0 for j + 1, P V of
+// tile 1, S of tile 1 for j + 1 -- each query tile's S overwrites its own P,
+// so it waits for that P V; the other tile's work keeps the pipe busy while
+// one tile's softmax runs.
+__global__ void __launch_bounds__(kThreads1, 1)
 k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* sQ = smem;                              // 128 rows x 2 boxes
-  uint8_t* sK = smem + kTileBytes;                 // kStK stages
+  uint8_t* sQ = smem;                              // two query tiles
+  uint8_t* sK = smem + 2 * kTileBytes;             // kStK stages
   uint8_t* sV = sK + kStK * kTileBytes;            // kSt1 stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kSt1 * kTileBytes);  // kBars1 barriers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBars1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xmax = reinterpret_cast<float*>(tmem_slot + 2);  // [3 buffers][4 groups][128]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1 KB alignment
     if (threadIdx.x == 0) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
     return;
   }
+  pdl_trigger();  // the combine may launch now; it waits for this grid to finish
   int b, h, chunk, t0, t1;
-  decode_cta(a, blockIdx.x, b, h, chunk, t0, t1);
+  decode_plan(a, a.splits1, a.cta_base1, a.chunks1, blockIdx.x, b, h, chunk, t0, t1);
   const int T = t1 - t0;
   const int L = a.L[b];
+  const int R = min(a.rows1, a.nq - chunk * a.rows1);  // this chunk's query rows
+  const int nt = R > 128 ? 2 : 1;                       // query tiles
   // barriers: Q; K full/empty (kStK stages); V full/empty (kSt1 stages); per
-  // TMEM S/P buffer: S ready, P written, tile max exchanged, P V done; O final
+  // query tile: S ready, P written, P V done
   const uint32_t BQ = smem_u32(&bars[0]);
   auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto KE = [&](int s) { return smem_u32(&bars[1 + kStK + s]); };
   auto VF = [&](int s) { return smem_u32(&bars[1 + 2 * kStK + s]); };
   auto VE = [&](int s) { return smem_u32(&bars[1 + 2 * kStK + kSt1 + s]); };
   constexpr int kB0 = 1 + 2 * kStK + 2 * kSt1;
-  auto SF = [&](int s) { return smem_u32(&bars[kB0 + s]); };
-  auto PF = [&](int s) { return smem_u32(&bars[kB0 + 3 + s]); };
-  auto XB = [&](int s) { return smem_u32(&bars[kB0 + 6 + s]); };
-  auto PD = [&](int s) { return smem_u32(&bars[kB0 + 9 + s]); };
-  const uint32_t OF = smem_u32(&bars[kB0 + 12]);  // committed once, after the last P V
+  auto SF = [&](int t) { return smem_u32(&bars[kB0 + t]); };
+  auto PF = [&](int t) { return smem_u32(&bars[kB0 + 2 + t]); };
+  auto PD = [&](int t) { return smem_u32(&bars[kB0 + 4 + t]); };
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
-    mbar_init(OF, 1);
     for (int s = 0; s < kStK; ++s) {
       mbar_init(KF(s), 1); mbar_init(KE(s), 1);
     }
     for (int s = 0; s < kSt1; ++s) {
       mbar_init(VF(s), 1);
-      mbar_init(VE(s), 2);  // P V commit + the ||v||^2 warp's reads
+      mbar_init(VE(s), 2);  // the last P V's commit + the ||v||^2 warp's reads
     }
-    for (int s = 0; s < 3; ++s) {
-      mbar_init(SF(s), 1); mbar_init(PF(s), kSimtWarps); mbar_init(XB(s), kSimtWarps);
-      mbar_init(PD(s), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(SF(t), 1); mbar_init(PF(t), 4); mbar_init(PD(t), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpMma) {
+  if (warp == kW1Mma) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
     tc_fence_before();
@@ -263,72 +183,76 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const int z = b * a.Hkv + h;
-  const int qrow0 = (b * a.Hkv + h) * a.G * a.w + chunk * a.nqc;
+  const int qrow0 = (b * a.Hkv + h) * a.nq + chunk * a.rows1;
 
-  if (warp == kWarpTma) {
-    // ---------------- TMA producer ----------------
-    // order: Q, K_0, K_1, then K_{j+2} and V_j for each tile j (S runs two
-    // tiles ahead of P V)
+  if (warp == kW1Tma || warp == kW1TmaV) {
+    // ---------------- TMA producers ----------------
+    // warp kW1Tma: the query tiles, then K_0, K_1, ... (K_{i+2} once both
+    // query tiles' S have read K_i); warp kW1TmaV: V_0, V_1, ... (kSt1 ahead).
     if (lane == 0) {
-      prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
-      mbar_expect_tx(BQ, 2u * 128u * (uint32_t)a.qbox_rows);
-      tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
-      tma_load_2d(smem_u32(sQ) + kBox, &tmQ, BQ, 64, qrow0);
-      auto load = [&](uint8_t* buf, int nst, const CUtensorMap* m, int i, uint32_t full,
-                      uint32_t empty) {
-        const int ph = (i / nst) & 1;
-        if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); return false; }
+      const bool kq = warp == kW1Tma;
+      if (kq) {
+        prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
+        mbar_expect_tx(BQ, (uint32_t)nt * 2u * 128u * (uint32_t)a.qbox_rows);
+        for (int t = 0; t < nt; ++t) {  // rows past the tensor read as zeros
+          tma_load_2d(smem_u32(sQ) + t * kTileBytes, &tmQ, BQ, 0, qrow0 + 128 * t);
+          tma_load_2d(smem_u32(sQ) + t * kTileBytes + kBox, &tmQ, BQ, 64, qrow0 + 128 * t);
+        }
+      } else {
+        prefetch_tmap(&tmV);
+      }
+      uint8_t* buf = kq ? sK : sV;
+      const int nst = kq ? kStK : kSt1;
+      const CUtensorMap* m = kq ? &tmK : &tmV;
+      for (int i = 0; i < T && !*abort_flag; ++i) {
+        const int st = i % nst, ph = (i / nst) & 1;
+        const uint32_t full = kq ? KF(st) : VF(st), empty = kq ? KE(st) : VE(st);
+        if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
         mbar_expect_tx(full, kTileBytes);
-        const uint32_t dst = smem_u32(buf + (i % nst) * kTileBytes);
+        const uint32_t dst = smem_u32(buf + st * kTileBytes);
         tma_load_3d(dst, m, full, 0, (t0 + i) * kTok, z);
         tma_load_3d(dst + kBox, m, full, 64, (t0 + i) * kTok, z);
-        return true;
-      };
-      bool ok = true;
-      for (int i = 0; i < 2 && i < T && ok; ++i)
-        ok = load(sK, kStK, &tmK, i, KF(i % kStK), KE(i % kStK));
-      for (int j = 0; j < T && ok && !*abort_flag; ++j) {
-        if (j + 2 < T) ok = load(sK, kStK, &tmK, j + 2, KF((j + 2) % kStK), KE((j + 2) % kStK));
-        if (ok) ok = load(sV, kSt1, &tmV, j, VF(j % kSt1), VE(j % kSt1));
       }
     }
-  } else if (warp == kWarpMma) {
+  } else if (warp == kW1Mma) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T
     constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);    // O += P V (V MN-major)
     bool ok = warp_wait(BQ, 0);
     if (!ok) fail(a, abort_flag);
-    // operand descriptors of stage 0; a stage or K slice only moves the start
-    // address, i.e. adds to the low word
+    // operand descriptors of stage 0; a stage, tile or K slice only moves the
+    // start address, i.e. adds to the low word
     const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024);
     const SDesc kd0 = sdesc_split(smem_u32(sK), 16, 1024);
     const SDesc vd0 = sdesc_split(smem_u32(sV), kBox, 1024);
-    auto issue_S = [&](int i) {
-      const int s = i % kStK, ph = (i / kStK) & 1, bf = i % 3;
+    // S_t(i) = Q_t K_i^T into tile t's S/P columns, which hold P_t(i - 1)
+    // until P V_t(i - 1) has read it
+    auto issue_S = [&](int t, int i) {
+      const int s = i % kStK, ph = (i / kStK) & 1;
       if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
-      // S(i) overwrites the buffer whose P the (i-3)-th P V reads from TMEM
-      if (i >= 3 && !warp_wait(PD(bf), ((i - 3) / 3) & 1)) { fail(a, abort_flag); return false; }
+      if (i >= 1 && !warp_wait(PD(t), (uint32_t)((i - 1) & 1))) { fail(a, abort_flag); return false; }
       tc_fence_after();
       if (lane == 0) {
+        const uint32_t qlo = qd.lo + (uint32_t)t * (kTileBytes >> 4);
         const uint32_t klo = kd0.lo + (uint32_t)s * (kTileBytes >> 4);
-        const uint32_t dS = tbase + (uint32_t)(bf * 128);
+        const uint32_t dS = tbase + (uint32_t)(128 * t);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss_w(dS, qd.lo + kslice(kk, 128), qd.hi, klo + kslice(kk, 128), kd0.hi, IDS,
+          mma_ss_w(dS, qlo + kslice(kk, 128), qd.hi, klo + kslice(kk, 128), kd0.hi, IDS,
                    kk > 0 ? 1u : 0u);
-        mma_commit(KE(s));
-        mma_commit(SF(bf));
+        mma_commit(SF(t));
+        if (t == nt - 1) mma_commit(KE(s));  // the last reader of this K stage
       }
       __syncwarp();
       return true;
     };
-    auto issue_PV = [&](int i) {
-      const int s = i % kSt1, ph = (i / kSt1) & 1, bf = i % 3, bph = (i / 3) & 1;
-      if (!warp_wait(PF(bf), bph)) { fail(a, abort_flag); return false; }
+    auto issue_PV = [&](int t, int i) {
+      const int s = i % kSt1, ph = (i / kSt1) & 1;
+      if (!warp_wait(PF(t), (uint32_t)(i & 1))) { fail(a, abort_flag); return false; }
       if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
       uint8_t* vb = sV + s * kTileBytes;
       const int tile0 = (t0 + i) * kTok;
-      if (tile0 + kTok > L) {
+      if (t == 0 && tile0 + kTok > L) {
         // rows at or beyond L hold no data (possibly NaN): zero them so that the
         // P = 0 weights of those rows contribute exactly 0 to O
         const int r0 = L - tile0;
@@ -343,8 +267,8 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       if (lane == 0) {
         const uint32_t vlo = vd0.lo + (uint32_t)s * (kTileBytes >> 4);
-        const uint32_t dO = tbase + kColO;
-        const uint32_t pS = tbase + (uint32_t)(bf * 128);
+        const uint32_t dO = tbase + kColO1 + (uint32_t)(128 * t);
+        const uint32_t pS = tbase + (uint32_t)(128 * t);
         // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16);
         // V slice kk starts 16 rows (2048 bytes) further
 #pragma unroll
@@ -354,22 +278,19 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
-        mma_commit(VE(s));
-        mma_commit(PD(bf));
-        if (i == T - 1) mma_commit(OF);
+        mma_commit(PD(t));
+        if (t == nt - 1) mma_commit(VE(s));  // the last reader of this V stage
       }
       __syncwarp();
       return true;
     };
-    // tensor-pipe order: S(0), S(1), then S(j + 2), P V(j) for each j.  S(j + 2)
-    // needs only P V(j - 1) done (its buffer) and goes ahead of P V(j), which
-    // waits for the softmax warps, so S is ready when they reach tile j + 2.
-    for (int i = 0; i < 2 && i < T && ok; ++i) ok = issue_S(i);
-    for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
-      if (j + 2 < T) ok = issue_S(j + 2);
-      if (ok) ok = issue_PV(j);
-    }
-  } else if (warp == kWarpNv) {
+    for (int t = 0; t < nt && t < 2 && ok && T > 0; ++t) ok = issue_S(t, 0);
+    for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j)
+      for (int t = 0; t < nt && ok; ++t) {
+        ok = issue_PV(t, j);
+        if (ok && j + 1 < T) ok = issue_S(t, j + 1);
+      }
+  } else if (warp == kW1Nv) {
     // ---------------- ||v_j||^2 ----------------
     // This CTA's share of every V tile's rows (the query chunks of a KV head
     // cover the same tokens and split the rows), 4 rows per lane; the order of
@@ -385,7 +306,7 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       float vmin = INFINITY;
       for (int rr = 0; rr < 4; ++rr) {
         const int row = rr * 32 + lane;
-        if ((row * a.chunks) / 128 != chunk || tile0 + row >= L) continue;
+        if ((row * a.chunks1) / 128 != chunk || tile0 + row >= L) continue;
         uint64_t acc2 = pk2(0.f, 0.f);
 #pragma unroll
         for (int bx = 0; bx < 2; ++bx)
@@ -408,123 +329,116 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       __syncwarp();
       if (lane == 0) mbar_arrive(VE(s));
       vmin = warp_min(vmin);  // pass 2 decides from it whether A needs its low part
-      if (lane == 0) a.tmin[((size_t)z * a.ntmax + t0 + j) * a.chunks + chunk] = vmin;
+      if (lane == 0) a.tmin[((size_t)z * a.ntmax + t0 + j) * a.chunks1 + chunk] = vmin;
     }
-  } else if (warp < kSimtWarps) {
+  } else if (warp < kSmWarps1) {
     // ---------------- softmax warps ----------------
-    // Sixteen warps work on every tile: warp (g, quarter) owns the query rows
-    // [32 quarter, +32) (its TMEM lanes), the tile's tokens [32 g, 32 g + 32)
-    // (its S/P columns) and O's head-dim columns [32 g, 32 g + 32).
-    // Software pipelined by one tile: step j posts tile j's max for the other
-    // three warps of its rows, then writes P of tile j - 1, whose maxes were
-    // posted a full step earlier, so the exchange rarely waits.
-    const int g = warp >> 2, ql = warp & 3;
-    const int row = ql * 32 + lane;  // query row within the chunk
-    const bool valid_row = row < a.nqc;
-    const int Prow = valid_row ? L - a.w + (chunk * a.nqc + row) % a.w : L - 1;
+    // Warpgroup t owns query tile t; thread = one query row (its TMEM lane),
+    // all 128 tokens of a tile: a max pass over S, then P = 2^(S c - m)
+    // written back over S as hi/lo planes.  The reference max moves only when
+    // a tile exceeds it by more than 8 (so 2^(.) <= 256); then l and the row
+    // of O are rescaled, after the P V that last accumulated into O.
+    const int t = warp >> 2, ql = warp & 3;
+    const int row = ql * 32 + lane;       // row within the query tile
+    const int crow = 128 * t + row;       // row within the chunk
+    const bool valid_row = crow < R;
+    const int Prow = L - a.w + (chunk * a.rows1 + crow) % a.w;
     const uint32_t lane_off = (uint32_t)(ql * 32) << 16;
-    const int c0 = g * 32;
-    const uint32_t tO = tbase + kColO + (uint32_t)c0 + lane_off;
+    const uint32_t tS = tbase + (uint32_t)(128 * t) + lane_off;
+    const uint32_t tO = tbase + kColO1 + (uint32_t)(128 * t) + lane_off;
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
     float m_ref = -INFINITY, l = 0.f;
-    for (int j = 0; j <= T; ++j) {
+    bool live = t < nt;  // a second warpgroup without a second tile only idles
+    for (int j = 0; j < T && live; ++j) {
+      if (!warp_wait(SF(t), (uint32_t)(j & 1))) { fail(a, abort_flag); live = false; break; }
+      if (warp_aborted(abort_flag)) { live = false; break; }
+      tc_fence_after();
+      const int tok0 = (t0 + j) * kTok;
+      const bool masked = tok0 + kTok - 1 > L - a.w;  // only the last tiles hide keys past P_t
       uint32_t sr[32];
-      if (j < T) {
-        // ---- tile j: row max of this warp's 32 keys, posted to the exchange
-        const int bf = j % 3;
-        if (!warp_wait(SF(bf), (j / 3) & 1)) { fail(a, abort_flag); break; }
-        if (warp_aborted(abort_flag)) break;
-        tc_fence_after();
-        const int tok0 = (t0 + j) * kTok + c0;
-        tmem_ld32(tbase + (uint32_t)(bf * 128) + lane_off + (uint32_t)c0, sr);
-        if (tok0 + 31 > L - a.w) {  // only the last tiles: hide keys past P_t
-#pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
-        }
-        float ya = -INFINITY, yb = -INFINITY;
+      float ya = -INFINITY, yb = -INFINITY;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        tmem_ld32(tS + 32u * cc, sr);
+        if (masked) p1_mask32(sr, tok0 + 32 * cc, Prow);
 #pragma unroll
         for (int u = 0; u < 32; u += 4) {
           ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
           yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
         }
-        xmax[bf * 512 + g * 128 + row] = fmaxf(ya, yb) * c;  // c > 0: commutes with the max
-        __syncwarp();
-        if (lane == 0) mbar_arrive(XB(bf));
       }
-      if (j >= 1) {
-        // ---- tile i = j - 1: the row's reference, then P = 2^(S c - m) over S
-        const int i = j - 1, bf = i % 3;
-        if (!warp_wait(XB(bf), (i / 3) & 1)) { fail(a, abort_flag); break; }
-        const float* xm = xmax + bf * 512;
-        const float mt = fmaxf(fmaxf(xm[row], xm[128 + row]), fmaxf(xm[256 + row], xm[384 + row]));
-        // the reference max moves only when a tile exceeds it by more than 8
-        // (so 2^(S c - m) <= 256); then l and O are rescaled
-        float fac = 1.f;
-        bool resc = false;
-        if (mt > m_ref + 8.f) {
-          if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
-          resc = m_ref != -INFINITY && i > 0;
-          m_ref = mt;
-          l *= fac;
-        }
-        // warp-uniform: every lane votes, and all or none call the rescale; O
-        // holds P V up to tile i - 1, which has landed once PD of its buffer
-        // completes that tile's phase
-        if (__any_sync(0xffffffffu, resc) &&
-            !p1_rescale_o(tO, fac, PD((i - 1) % 3), (uint32_t)(((i - 1) / 3) & 1))) {
-          fail(a, abort_flag);
-          break;
-        }
-        const uint32_t tS = tbase + (uint32_t)(bf * 128) + lane_off + (uint32_t)c0;
-        const int tok0 = (t0 + i) * kTok + c0;
-        tmem_ld32(tS, sr);
-        if (tok0 + 31 > L - a.w) {
-#pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (tok0 + u > Prow) sr[u] = 0xFF800000u;
-        }
-        l += p1_exp32(sr, tS, c2, m_ref == -INFINITY ? 0.f : m_ref);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(PF(bf));
+      const float mt = fmaxf(ya, yb) * c;  // c > 0: commutes with the max
+      float fac = 1.f;
+      bool resc = false;
+      if (mt > m_ref + 8.f) {
+        if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
+        resc = m_ref != -INFINITY && j > 0;
+        m_ref = mt;
+        l *= fac;
       }
-    }
-    // partial row: this warp's 32 columns of O, the shared max, its normaliser part
-    float* out = a.partial + ((size_t)blockIdx.x * 128 + row) * kPartStride;
-    bool have = T > 0 && !warp_aborted(abort_flag);
-    if (have) {
-      if (!warp_wait(OF, 0)) {
+      // warp-uniform: every lane votes, and all or none call the rescale; O
+      // holds P V up to tile j - 1, which has landed once PD completes its phase
+      if (__any_sync(0xffffffffu, resc) &&
+          !p1_rescale_o(tO, fac, PD(t), (uint32_t)((j - 1) & 1))) {
         fail(a, abort_flag);
-        have = false;
+        live = false;
+        break;
       }
-      tc_fence_after();
+      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        tmem_ld32(tS + 32u * cc, sr);
+        if (masked) p1_mask32(sr, tok0 + 32 * cc, Prow);
+        l += p1_exp32(sr, tS + 32u * cc, c2, mu);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(PF(t));
     }
-    uint32_t o[32];
-    if (have) tmem_ld32(tO, o);
-    if (valid_row) {
+    // partial row: O, the reference max, the normaliser
+    if (t < nt) {
+      bool have = live && T > 0 && !warp_aborted(abort_flag);
+      if (have) {
+        if (!warp_wait(PD(t), (uint32_t)((T - 1) & 1))) {
+          fail(a, abort_flag);
+          have = false;
+        }
+        tc_fence_after();
+      }
+      float* out = a.partial + ((size_t)blockIdx.x * a.rows1 + crow) * kPartStride;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t o[32];
+        if (have) tmem_ld32(tO + 32u * cc, o);
+        if (valid_row) {
 #pragma unroll
-      for (int u = 0; u < 32; u += 4)
-        *reinterpret_cast<float4*>(out + c0 + u) =
-            have ? make_float4(f32(o[u]), f32(o[u + 1]), f32(o[u + 2]), f32(o[u + 3]))
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
-      if (g == 0) out[128] = have ? m_ref : -INFINITY;
-      out[129 + g] = have ? l : 0.f;
+          for (int u = 0; u < 32; u += 4)
+            *reinterpret_cast<float4*>(out + 32 * cc + u) =
+                have ? make_float4(f32(o[u]), f32(o[u + 1]), f32(o[u + 2]), f32(o[u + 3]))
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      if (valid_row) {
+        out[128] = have ? m_ref : -INFINITY;
+        out[129] = have ? l : 0.f;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == kW1Mma) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
 }
 
 // =========================== combine ========================================
-// One warp per query row: merge the 2 * splits partials of its (b, h, chunk).
+// One warp per query row: merge the split partials of its pass-1 (b, h, chunk).
 __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
+  pdl_trigger();
+  pdl_wait();  // the partials come from pass 1
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows = a.B * a.Hq * a.w;
   const int r = blockIdx.x * 4 + warp;
@@ -534,42 +448,47 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
   const int t = r % a.w;
   const int h = hq / a.G;
   const int gr = (hq % a.G) * a.w + t;
-  const int chunk = gr / a.nqc, rr = gr % a.nqc;
-  const int cta0 = a.cta_base[b] + (h * a.chunks + chunk) * a.splits[b];
-  const int np = a.splits[b];
-  auto P = [&](int i) { return a.partial + ((size_t)(cta0 + i) * 128 + rr) * kPartStride; };
-  // lanes take the partials' (max, normaliser) in parallel: M, then the
-  // weights 2^(m_i - M) and L = sum_i w_i l_i
-  float M = -INFINITY;
-  for (int i = lane; i < np; i += 32) M = fmaxf(M, P(i)[128]);
-  M = warp_max(M);
-  float lpart = 0.f;
+  const int chunk = gr / a.rows1, rr = gr % a.rows1;
+  const int cta0 = a.cta_base1[b] + (h * a.chunks1 + chunk) * a.splits1[b];
+  const int np = a.splits1[b];
+  auto P = [&](int i) { return a.partial + ((size_t)(cta0 + i) * a.rows1 + rr) * kPartStride; };
+  // lanes take the partials' (max, normaliser) pairs in parallel, 32 at a
+  // time: M, then the weights 2^(m_i - M) and L = sum_i w_i l_i; the weights
+  // of the first 32 partials stay in the lanes that loaded them
+  float M = -INFINITY, m_own = -INFINITY, l_own = 0.f;
   for (int i = lane; i < np; i += 32) {
-    const float* p = P(i);
-    const float mi = p[128];
-    const float wgt = (mi == -INFINITY) ? 0.f : ex2(mi - M);
-    lpart = fmaf(wgt, (p[129] + p[130]) + (p[131] + p[132]), lpart);  // four normaliser parts
+    const float2 ml = *reinterpret_cast<const float2*>(P(i) + 128);
+    if (i == lane) { m_own = ml.x; l_own = ml.y; }
+    M = fmaxf(M, ml.x);
+  }
+  M = warp_max(M);
+  const float w_own = (m_own == -INFINITY) ? 0.f : ex2(m_own - M);
+  float lpart = w_own * l_own;
+  for (int i = lane + 32; i < np; i += 32) {
+    const float2 ml = *reinterpret_cast<const float2*>(P(i) + 128);
+    lpart = fmaf((ml.x == -INFINITY) ? 0.f : ex2(ml.x - M), ml.y, lpart);
   }
   const float Lsum = warp_sum(lpart);
-  // O = sum_i w_i O_i, four partial rows in flight per step
+  // O = sum_i w_i O_i, eight partial rows in flight per step
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < np; i0 += 4) {
-    float4 o[4];
-    float wg[4];
+  for (int i0 = 0; i0 < np; i0 += 8) {
+    float4 o[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int i = min(i0 + k, np - 1);
-      const float* p = P(i);
-      o[k] = *reinterpret_cast<const float4*>(p + lane * 4);
-      const float mi = p[128];
-      wg[k] = (i0 + k >= np || mi == -INFINITY) ? 0.f : ex2(mi - M);
-    }
+    for (int k = 0; k < 8; ++k)
+      o[k] = *reinterpret_cast<const float4*>(P(min(i0 + k, np - 1)) + lane * 4);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      acc.x = fmaf(wg[k], o[k].x, acc.x);
-      acc.y = fmaf(wg[k], o[k].y, acc.y);
-      acc.z = fmaf(wg[k], o[k].z, acc.z);
-      acc.w = fmaf(wg[k], o[k].w, acc.w);
+    for (int k = 0; k < 8; ++k) {
+      const int i = i0 + k;
+      float wg = __shfl_sync(0xffffffffu, w_own, i & 31);
+      if (i >= 32) {  // past the first 32 partials: recompute the weight
+        const float mi = P(min(i, np - 1))[128];
+        wg = (mi == -INFINITY) ? 0.f : ex2(mi - M);
+      }
+      if (i >= np) wg = 0.f;
+      acc.x = fmaf(wg, o[k].x, acc.x);
+      acc.y = fmaf(wg, o[k].y, acc.y);
+      acc.z = fmaf(wg, o[k].z, acc.z);
+      acc.w = fmaf(wg, o[k].w, acc.w);
     }
   }
   const float inv = 1.f / Lsum;
@@ -753,6 +672,8 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     *abort_flag = 0;
     fence_mbar_init();
   }
+  pdl_trigger();
+  pdl_wait();  // qstat, A and ||v||^2 come from the combine and pass 1
   if (threadIdx.x < nqc) {
     const int i = threadIdx.x;
     const float4 q = a.qstat[qrow0 + i];  // (M, 1/L, L, ||A||^2)
@@ -782,8 +703,8 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     float namx = 0.f;
     for (int i = 0; i < (nqc + 15) / 16; ++i) namx = fmaxf(namx, nAmax[i]);
     bool need = false;
-    for (int i = threadIdx.x; i < T * a.chunks; i += blockDim.x) {
-      const float tm = a.tmin[((size_t)z * a.ntmax + t0) * a.chunks + i];
+    for (int i = threadIdx.x; i < T * a.chunks1; i += blockDim.x) {
+      const float tm = a.tmin[((size_t)z * a.ntmax + t0) * a.chunks1 + i];
       if (!(namx <= kLoSkip * tm)) need = true;  // NaN-safe
     }
     lo = __syncthreads_or(need) != 0;
@@ -1021,9 +942,7 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t pass1_smem() {
-  return (1 + kStK + kSt1) * (size_t)kTileBytes + kBars1 * 8 + 8 + 3 * 4 * 128 * 4;
-}
+size_t pass1_smem() { return (2 + kStK + kSt1) * (size_t)kTileBytes + kBars1 * 8 + 8; }
 size_t pass2_smem(int nqc) {
   return kRing2 * (size_t)kTileBytes + 2 * (size_t)nqc * 256 + (size_t)nqc / 2 * 16 + 8 * 4 +
          (5 + 2 * kRing2) * 8 + 8;
@@ -1037,6 +956,11 @@ int num_sms() {
 }
 
 }  // namespace
+
+// tc_pair.cu
+cudaError_t launch_tc_pass2_pair(const TcArgs& a, const CUtensorMap& mQ, const CUtensorMap& mAh,
+                                 const CUtensorMap& mAl, const CUtensorMap& mK,
+                                 const CUtensorMap& mV, int pairs, cudaStream_t st);
 
 bool tc_available() { return true; }
 int tc_split_target() { return kMaxCtas; }
@@ -1070,9 +994,9 @@ void tc_splits(const Lens& lens, int units_per_row, int budget, int32_t* splits)
 cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k, const void* v,
                              const Lens& lens, const ScoresLayout& lay, char* ws, float* attn_out,
                              float* stats_out, int32_t* status, int score, int cta_budget,
-                             cudaStream_t st, KernelEvents& kev) {
+                             cudaStream_t st, KernelEvents& kev, int* nparts_used) {
   const bool attn_only = score == DROPKV_SCORE_ATTENTION;
-  auto pass2 = attn_only ? k_tc_pass2<true> : k_tc_pass2<false>;
+  auto pass2 = k_tc_pass2<true>;  // the attention-only control; DropKV runs the pair kernel
   const TcPlan plan = tc_plan(s);
   TcArgs a;
   memset(&a, 0, sizeof(a));
@@ -1084,13 +1008,28 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   a.G = s.Hq / s.Hkv;
   a.nqc = plan.nqc;
   a.chunks = plan.chunks;
+  a.nq = a.G * a.w;
+  a.chunks1 = plan.chunks1;
+  a.rows1 = plan.rows1;
   for (int i = 0; i < lens.B; ++i) a.L[i] = lens.L[i];
-  const int units = s.Hkv * plan.chunks;
   const int budget = std::min(cta_budget > 0 ? cta_budget : num_sms(), kMaxCtas);
+  const int units = s.Hkv * plan.chunks;    // pass 2
   tc_splits(lens, units, std::max(budget, units * lens.B), a.splits);
   a.cta_base[0] = 0;
   for (int i = 0; i < lens.B; ++i) a.cta_base[i + 1] = a.cta_base[i] + units * a.splits[i];
   const int ctas = a.cta_base[lens.B];
+  const int units1 = s.Hkv * plan.chunks1;  // pass 1
+  tc_splits(lens, units1, std::max(budget, units1 * lens.B), a.splits1);
+  a.cta_base1[0] = 0;
+  for (int i = 0; i < lens.B; ++i) a.cta_base1[i + 1] = a.cta_base1[i] + units1 * a.splits1[i];
+  const int ctas1 = a.cta_base1[lens.B];
+  a.chunks2 = plan.chunks2;
+  a.nqc2 = plan.nqc2;
+  const int units2 = s.Hkv * plan.chunks2;  // pair pass 2, in CTA pairs
+  tc_splits(lens, units2, std::max(budget / 2, units2 * lens.B), a.splits2);
+  a.cta_base2[0] = 0;
+  for (int i = 0; i < lens.B; ++i) a.cta_base2[i + 1] = a.cta_base2[i] + units2 * a.splits2[i];
+  const int pairs = a.cta_base2[lens.B];
   a.c_log2 = (float)(1.4426950408889634 / sqrt((double)s.d));
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
   a.partial = reinterpret_cast<float*>(ws + lay.tc_partial);
@@ -1111,32 +1050,37 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   const uint64_t rows = (uint64_t)lens.B * s.Hq * s.window;
   a.qbox_rows = (int32_t)std::min<uint64_t>(128, rows);
   CUtensorMap mQ1, mQ2, mK, mV, mAh, mAl;
-  if (!map_2d(&mQ1, q, rows, (uint32_t)a.qbox_rows) || !map_2d(&mQ2, q, rows, (uint32_t)plan.nqc) ||
+  const uint32_t box2 = attn_only ? (uint32_t)plan.nqc : (uint32_t)(plan.nqc2 / 2);
+  if (!map_2d(&mQ1, q, rows, (uint32_t)a.qbox_rows) || !map_2d(&mQ2, q, rows, box2) ||
       !map_3d(&mK, k, (uint64_t)lens.B * s.Hkv, (uint64_t)s.n_max) ||
       !map_3d(&mV, v, (uint64_t)lens.B * s.Hkv, (uint64_t)s.n_max) ||
-      !map_2d(&mAh, a.ahi, rows, (uint32_t)plan.nqc) ||
-      !map_2d(&mAl, a.alo, rows, (uint32_t)plan.nqc))
+      !map_2d(&mAh, a.ahi, rows, box2) || !map_2d(&mAl, a.alo, rows, box2))
     return cudaErrorNotSupported;
 
   const size_t sm1 = pass1_smem(), sm2 = pass2_smem(plan.nqc);
   cudaError_t e = cudaFuncSetAttribute(k_tc_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sm1);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && attn_only)
     e = cudaFuncSetAttribute(pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
   if (e != cudaSuccess) return e;
+  *nparts_used = 4 * (attn_only ? plan.chunks : plan.chunks2);
 
   kev.begin(st);
-  k_tc_pass1<<<ctas, kThreads1, sm1, st>>>(mQ1, mK, mV, a);
+  k_tc_pass1<<<ctas1, kThreads1, sm1, st>>>(mQ1, mK, mV, a);
   kev.end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kev.begin(st);
-  k_tc_combine<<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(a);
+  e = launch_ex(k_tc_combine, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st, true, 1, a);
   kev.end(st);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (e != cudaSuccess) return e;
   kev.begin(st);
-  pass2<<<ctas, kThreads2, sm2, st>>>(mQ2, mAh, mAl, mK, mV, a);
+  if (attn_only) {
+    e = launch_ex(pass2, dim3(ctas), dim3(kThreads2), sm2, st, true, 1, mQ2, mAh, mAl, mK, mV, a);
+  } else {
+    e = launch_tc_pass2_pair(a, mQ2, mAh, mAl, mK, mV, pairs, st);
+  }
   kev.end(st);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace dropkv

@@ -9,7 +9,7 @@ oracle on:
   heavy keys, 128K with outlier channels, and the batched mixed-length case
   with NaN-poisoned padding), on every path the shape allows;
 * "deep pipeline" cases in which every tensor-path CTA walks a long run of
-  tiles (16 to 128), so the steady state of both passes -- every TMEM buffer
+  tiles (16 to 64), so the steady state of both passes -- every TMEM buffer
   and shared-memory ring slot reused many times, the deferred O rescale, the
   barriers' parity flips -- is compared element by element, including a
   ragged-length case and one with planted heavy keys (p up to about 0.97);
@@ -66,19 +66,13 @@ def _compare(wl, ref, got, what):
     return worst
 
 
-def tiles_per_cta(spec, tc_ctas=0, sms=148):
-    """Tile runs the tensor path gives its CTAs: the same greedy split rule
-    as the library (one more split to the row whose CTAs are longest while
-    the CTA budget allows), returned as the (min, max) tiles per CTA."""
-    G = spec.Hq // spec.Hkv
-    nq = G * spec.window
-    chunks = (nq + 127) // 128
-    units = spec.Hkv * chunks
-    budget = min(tc_ctas if tc_ctas > 0 else sms, 160)
-    budget = max(budget, units * spec.B)
-    nts = [(L + TILE - 1) // TILE for L in spec.lengths]
-    splits = [1] * spec.B
-    total = units * spec.B
+def _split_runs(lengths, units, budget):
+    """The library's split rule: one more split to the row whose runs are
+    longest while the budget allows; returns every run's tile count."""
+    nts = [(L + TILE - 1) // TILE for L in lengths]
+    splits = [1] * len(lengths)
+    total = units * len(lengths)
+    budget = max(budget, total)
     while True:
         best, worst = -1, 0.0
         for b, nt in enumerate(nts):
@@ -89,11 +83,21 @@ def tiles_per_cta(spec, tc_ctas=0, sms=148):
             break
         splits[best] += 1
         total += units
-    runs = []
-    for b, nt in enumerate(nts):
-        for sp in range(splits[b]):
-            runs.append((sp + 1) * nt // splits[b] - sp * nt // splits[b])
-    return min(runs), max(runs)
+    return [(sp + 1) * nt // splits[b] - sp * nt // splits[b]
+            for b, nt in enumerate(nts) for sp in range(splits[b])]
+
+
+def tiles_per_cta(spec, tc_ctas=0, sms=148):
+    """Tile runs of the tensor path's CTAs, (min, max) over both passes: pass 1
+    runs one CTA per (b, h, chunk of <= 256 query rows, split) within the CTA
+    budget; the DropKV second pass runs CTA pairs (half the budget) and each
+    CTA of a pair takes half of the pair's run."""
+    nq = (spec.Hq // spec.Hkv) * spec.window
+    units = spec.Hkv * ((nq + 255) // 256)
+    budget = min(tc_ctas if tc_ctas > 0 else sms, 160)
+    r1 = _split_runs(spec.lengths, units, budget)
+    r2 = [x // 2 for x in _split_runs(spec.lengths, units, budget // 2)]
+    return min(r1 + r2), max(r1 + r2)
 
 
 # ---- the four full-size configurations, whole arrays -------------------------
@@ -112,31 +116,30 @@ def test_full_config_whole(idx):
 
 # ---- deep pipelines: long tile runs per CTA ----------------------------------
 
+# A CTA budget of 64 gives every (b, h) unit one pass-1 CTA walking all 32
+# tiles of its 4096 tokens, and one CTA pair in the second pass (16 tiles each).
 DEEP = [
-    # 8 rows x 8 KV heads x 2 query chunks = 128 units: one split per row
-    # (one row gets two), so CTAs walk 32 (16) tiles of 128 tokens
     W.Spec("deep_b8_w64_outlier", B=8, Hq=32, Hkv=8, d=128, lengths=[4096] * 8, window=64,
            pool=7, keep=[W.budget(0.05, 4096)] * 8, outlier_channels=4),
-    # ragged lengths with NaN-poisoned padding: runs of 14 to 32 tiles, each
-    # ending in a partial tile at a different offset
+    # ragged lengths with NaN-poisoned padding: runs ending in a partial tile
+    # at a different offset
     W.Spec("deep_b8_ragged_nan", B=8, Hq=32, Hkv=8, d=128,
            lengths=[4096, 3001, 4000, 2500, 3333, 4095, 1800, 3900], window=64, pool=7,
            keep=[W.budget(0.05, L) for L in (4096, 3001, 4000, 2500, 3333, 4095, 1800, 3900)],
            n_max=4096, nan_pad=True, outlier_channels=4),
     # planted heavy keys (p up to about 0.97): the careful path and the moving
-    # reference max fire in the middle of long runs; G*w = 128 is one query
-    # chunk, so 64 units: a budget of 64 CTAs gives each a run of 32 tiles
+    # reference max fire in the middle of long runs
     W.Spec("deep_b8_heavy", B=8, Hq=32, Hkv=8, d=128, lengths=[4096] * 8, window=32, pool=7,
            keep=[W.budget(0.05, 4096)] * 8, heavy_per_head=16),
 ]
-DEEP_CTAS = {"deep_b8_heavy": 64}
+DEEP_CTAS = 64
 
 
 @pytest.mark.parametrize("spec", DEEP, ids=[s.name for s in DEEP])
 def test_deep_pipeline_whole(spec):
-    tc_ctas = DEEP_CTAS.get(spec.name, 0)
+    tc_ctas = DEEP_CTAS
     lo, hi = tiles_per_cta(spec, tc_ctas)
-    assert lo >= 14, (lo, hi)  # every CTA's run is long: the steady state is compared
+    assert lo >= 7, (lo, hi)  # every CTA's run is long: the steady state is compared
     wl = W.generate(spec, 7)
     ref = oracle.scores(wl.q, wl.k, wl.v, wl.lengths, spec.window, spec.pool)
     for path in _paths(spec):
@@ -145,8 +148,9 @@ def test_deep_pipeline_whole(spec):
 
 @pytest.mark.parametrize("tc_ctas", [16, 48, 0])
 def test_cta_budget_gives_the_same_scores(tc_ctas):
-    # 128K-token workload shape at n = 16384: with 16 CTAs each (b, h, chunk)
-    # unit is one CTA walking all 128 tiles; 48 gives uneven runs of 42/43
+    # 128K-token workload shape at n = 16384: with 16 CTAs, pass-1 CTAs walk 64
+    # tiles and each second-pass CTA 64 (one pair per KV head); 48 gives
+    # uneven runs of 21/22
     spec = W.Spec("cfg3_shape_16k", B=1, Hq=32, Hkv=8, d=128, lengths=[16384], window=64,
                   pool=7, keep=[W.budget(0.05, 16384)], outlier_channels=4)
     lo, hi = tiles_per_cta(spec, tc_ctas)
@@ -155,7 +159,7 @@ def test_cta_budget_gives_the_same_scores(tc_ctas):
     got = _gpu(wl, "tensor", tc_ctas=tc_ctas)
     _compare(wl, ref, got, f"tc_ctas={tc_ctas} (tiles per CTA {lo}..{hi})")
     if tc_ctas == 16:
-        assert lo == hi == 128
+        assert lo == hi == 64
 
 
 def test_window_attention_outputs_deep():
