@@ -64,14 +64,18 @@ int resolve_path(const dropkv_shape& s, int requested) {
 dropkv_status device_ok() { return check_device(); }
 
 // Tensor path: bf16, d = 128, and the G*w query rows of a KV head split into
-// equal chunks of at most 128 rows whose size is a multiple of 16 (the N of
-// the token-major pass-2 MMA).
+// equal chunks whose widths suit the token-major second passes' MMAs.
 bool tc_shape_ok(const dropkv_shape& s) {
   if (!tc_available()) return false;
   if (s.dtype != DROPKV_BF16 || s.d != 128 || s.n_max < 128) return false;
   const int nq = (s.Hq / s.Hkv) * s.window;
+  // the single-CTA second pass: chunks of <= 128 rows, multiples of 16; the
+  // pair second pass: chunks of <= 256 rows taken as one or two halves whose
+  // width (the MMA's N) is a multiple of 16
   const int chunks = (nq + 127) / 128, chunks2 = (nq + 255) / 256;
-  if (nq % (16 * chunks) != 0 || nq % (16 * chunks2) != 0) return false;
+  if (nq % (16 * chunks) != 0 || nq % chunks2 != 0) return false;
+  const int nqc2 = nq / chunks2;
+  if (nqc2 % (nqc2 > 128 ? 32 : 16) != 0) return false;
   return true;
 }
 

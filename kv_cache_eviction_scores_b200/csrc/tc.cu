@@ -521,81 +521,6 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
 }
 
 // =========================== pass 2 =========================================
-// ||a - v||^2 taken directly (fp32 a, bf16 v, both from global memory).  Used
-// only where the expansion ||a||^2 + ||v||^2 - 2 a.v cancels by more than 32x,
-// i.e. a is close to v (a dominant token, p_j near 1).
-__device__ __noinline__ float direct_sqdist(const float* A, const __nv_bfloat16* v) {
-  float s = 0.f;
-  for (int c = 0; c < kHd; c += 4) {
-    const float4 a4 = *reinterpret_cast<const float4*>(A + c);
-    const uint2 v4 = *reinterpret_cast<const uint2*>(v + c);
-    const float d0 = a4.x - __uint_as_float(v4.x << 16);
-    const float d1 = a4.y - __uint_as_float(v4.x & 0xFFFF0000u);
-    const float d2 = a4.z - __uint_as_float(v4.y << 16);
-    const float d3 = a4.w - __uint_as_float(v4.y & 0xFFFF0000u);
-    s = fmaf(d0, d0, s);
-    s = fmaf(d1, d1, s);
-    s = fmaf(d2, d2, s);
-    s = fmaf(d3, d3, s);
-  }
-  return s;
-}
-
-// Fast path for 16 query columns of one token (every p < 2^-4, no possible
-// cancellation, every key visible): packed fp32 pairs,
-//   p = 2^(x c - M'),  M' = M + log2 L,
-//   ratio = p / (1 - p) = p (1 + p (1 + p (1 + p (1 + p)))) + O(p^6)
-//   (relative truncation error p^5 / (1 - p) <= 1.0e-6 for p < 2^-4),
-//   s += ratio^2 (D' + ||A||^2 + ||v||^2)   with D' = -2 A.v from the MMA.
-// kf holds (-M'_t, -M'_t+1, ||A_t||^2, ||A_t+1||^2) per column pair.
-__device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf, uint64_t c2,
-                                       uint64_t nv2, uint64_t& acc2, float& pmax) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 k = kf[i];
-    float y0, y1;
-    upk2(ffma2(pk2(f32(r[2 * i]), f32(r[2 * i + 1])), c2, pk2(k.x, k.y)), y0, y1);
-    const float p0 = ex2(y0), p1 = ex2(y1);
-    pmax = fmax3(pmax, p0, p1);
-    const uint64_t P = pk2(p0, p1);
-    const uint64_t one = pk2(1.f, 1.f);
-    const uint64_t ratio = fmul2(P, ffma2(P, ffma2(P, ffma2(P, fadd2(P, one), one), one), one));
-    const uint64_t zt = fadd2(fadd2(pk2(f32(r[16 + 2 * i]), f32(r[16 + 2 * i + 1])),
-                                    pk2(k.z, k.w)), nv2);
-    acc2 = ffma2(fmul2(ratio, ratio), zt, acc2);
-  }
-}
-
-// Careful path for 16 query columns of one token (r[0..15] = S^T, r[16..31] =
-// D): the causal mask, ratio = e / (L - e) with the singular check when
-// p >= 2^-8, and the direct squared distance where the expansion cancels by
-// more than 32x.
-__device__ __noinline__ float careful16(const uint32_t* r, int col0, int tok, bool masked, int L,
-                                        int w, int crow0, const float4* qstat_rows, float c,
-                                        float nv, const float* arows, const __nv_bfloat16* vrow,
-                                        int* sing) {
-  float acc = 0.f;
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int col = col0 + u;
-    const float4 k = qstat_rows[col];  // (M, 1/L, L, ||A||^2)
-    const bool vis = !masked || tok <= L - w + (crow0 + col) % w;
-    const float e = ex2(fmaf(f32(r[u]), c, -k.x));
-    const float p = e * k.y;
-    float ratio = fmaf(p, fmaf(p, p, p), p);
-    const float base = k.w + nv;
-    float zt = base + f32(r[16 + u]);
-    if (vis && p >= 0.00390625f) {
-      const float den = k.z - e;  // (1 - p) L
-      if (!(den > 0.f)) *sing = 1;
-      ratio = __fdiv_rn(e, den);
-    }
-    if (vis && zt < 0.03125f * base) zt = direct_sqdist(arows + (size_t)col * kHd, vrow);
-    if (vis) acc += ratio * ratio * zt;
-  }
-  return acc;
-}
-
 // Attention-only score (the write-up's control, section 结果与独立对照) for 16
 // query columns of one token: sum of p = 2^(x c - M') over the columns that see
 // the token (all of them when `masked` is false).  r[0..15] holds S^T.
@@ -1050,7 +975,9 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   const uint64_t rows = (uint64_t)lens.B * s.Hq * s.window;
   a.qbox_rows = (int32_t)std::min<uint64_t>(128, rows);
   CUtensorMap mQ1, mQ2, mK, mV, mAh, mAl;
-  const uint32_t box2 = attn_only ? (uint32_t)plan.nqc : (uint32_t)(plan.nqc2 / 2);
+  // the pair pass loads, per query half of nqc2 / nh columns, half the rows per CTA
+  const int nh2 = plan.nqc2 > 128 ? 2 : 1;
+  const uint32_t box2 = attn_only ? (uint32_t)plan.nqc : (uint32_t)(plan.nqc2 / nh2 / 2);
   if (!map_2d(&mQ1, q, rows, (uint32_t)a.qbox_rows) || !map_2d(&mQ2, q, rows, box2) ||
       !map_3d(&mK, k, (uint64_t)lens.B * s.Hkv, (uint64_t)s.n_max) ||
       !map_3d(&mV, v, (uint64_t)lens.B * s.Hkv, (uint64_t)s.n_max) ||

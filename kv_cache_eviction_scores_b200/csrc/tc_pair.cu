@@ -9,22 +9,24 @@
 //
 // Layout.  Two CTAs of a cluster process 256 tokens per step: each CTA owns
 // one 128-token tile of its own contiguous token range, taken from its end
-// down (the M = 256 MMA takes 128 rows of A from each CTA), and the nqc <= 256 query columns of the chunk
-// are split between them (each CTA holds nqc / 2 rows of Q, -2A_hi and -2A_lo,
-// the B operand's halves).  Per step the even CTA issues
-//     S^T = K Q^T                     into TMEM columns [0, nqc)
-//     D   = V (-2A_hi)^T [+ V (-2A_lo)^T]   into TMEM columns [256, 256 + nqc)
-// and commits to barriers of both CTAs.  The score warps of each CTA turn S^T
-// into ratio^2 (kept in registers) and hand the S columns back, then read D
-// and accumulate, and hand the D columns back: S of step i + 1 overlaps the D
-// arithmetic of step i, and D of step i + 1 the S arithmetic of step i + 1.
-// Halving each CTA's operand reads (compared with one CTA per 128-row MMA)
-// keeps the tensor pipe's shared-memory traffic well under the SM's bandwidth.
+// down (the M = 256 MMA takes 128 rows of A from each CTA).  The chunk's
+// nqc <= 256 query columns are processed as nh halves of nqh <= 128 columns;
+// for each half both CTAs hold nqh / 2 rows of Q, -2A_hi and -2A_lo (the B
+// operand's halves).  Per (step, half) the even CTA issues
+//     S^T = K Q_h^T  and  D = V (-2A_hi,h)^T [+ V (-2A_lo,h)^T]
+// into one of two TMEM buffers of 256 columns and commits to barriers of both
+// CTAs; the score warps of each CTA read S^T and D of their 32 columns 16 at
+// a time and hand the buffer back after the last read, so the MMAs of the
+// next half overlap this half's arithmetic.  An M = 256, N = 128 pair MMA
+// reads 6 KB of shared memory per CTA per 64-cycle K step (4 KB of its own
+// tokens, 2 KB of its query rows), against 8 KB for a single-CTA M = 128,
+// N = 128 MMA, which alone is the SM's whole shared-memory bandwidth.
 //
 // Every wait is bounded (2 s of %globaltimer); on expiry the kernel records
-// DROPKV_ERR_TIMEOUT, every role leaves its loop, and the CTAs meet at the
-// hardware cluster barrier before freeing TMEM, so neither leaves while the
-// other may still address its shared memory or TMEM.
+// DROPKV_ERR_TIMEOUT, every role leaves its loop, the issued MMAs are waited
+// for, and the CTAs meet at the hardware cluster barrier before freeing TMEM,
+// so neither leaves while the other may still address its shared memory or
+// TMEM.
 #include <cuda.h>
 #include <string.h>
 
@@ -35,101 +37,23 @@ namespace {
 
 constexpr int kRingP = 4;          // 32 KB K/V slots per CTA
 constexpr int kThreadsP = (kSimtWarps + 2) * 32;
-constexpr uint32_t kColD = 256;    // D columns start here
 
-// Fast path of phase A for 16 query columns: ratio^2 for every p < 2^-4 with
-// the series p (1 + p (1 + p (1 + p (1 + p)))) of p / (1 - p) (truncation
-// error p^5 / (1 - p) <= 1.0e-6 relative).  kf holds (-M'_t, -M'_t+1,
-// ||A_t||^2, ||A_t+1||^2) per column pair.
-__device__ __forceinline__ void pairA_fast(const uint32_t (&r)[16], const float4* kf, uint64_t c2,
-                                           uint64_t (&r2)[8], float& pmax) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 k = kf[i];
-    float y0, y1;
-    upk2(ffma2(pk2(f32(r[2 * i]), f32(r[2 * i + 1])), c2, pk2(k.x, k.y)), y0, y1);
-    const float p0 = ex2(y0), p1 = ex2(y1);
-    pmax = fmax3(pmax, p0, p1);
-    const uint64_t P = pk2(p0, p1);
-    const uint64_t one = pk2(1.f, 1.f);
-    const uint64_t ratio = fmul2(P, ffma2(P, ffma2(P, ffma2(P, fadd2(P, one), one), one), one));
-    r2[i] = fmul2(ratio, ratio);
-  }
-}
-
-// Careful path of phase A, out of line: the causal mask (and tokens this CTA
-// does not own), ratio = e / (L - e) with the singular check when p >= 2^-8.
-// out[u] = ratio^2 of column col0 + u, 0 where the token is not visible.
-__device__ __noinline__ void pairA_careful(const uint32_t* r, int col0, int tok, bool valid,
-                                           bool masked, int L, int w, int crow0,
-                                           const float4* qstat_rows, float c, int* sing,
-                                           float* out) {
-#pragma unroll 1
-  for (int u = 0; u < 16; ++u) {
-    const int col = col0 + u;
-    const float4 k = qstat_rows[col];  // (M, 1/L, L, ||A||^2)
-    const bool vis = valid && (!masked || tok <= L - w + (crow0 + col) % w);
-    const float e = ex2(fmaf(f32(r[u]), c, -k.x));
-    const float p = e * k.y;
-    float ratio = fmaf(p, fmaf(p, p, p), p);
-    if (vis && p >= 0.00390625f) {
-      const float den = k.z - e;  // (1 - p) L
-      if (!(den > 0.f)) *sing = 1;
-      ratio = __fdiv_rn(e, den);
-    }
-    out[u] = vis ? ratio * ratio : 0.f;
-  }
-}
-
-// ||a - v||^2 taken directly (fp32 a, bf16 v, both from global memory).  Used
-// only where the expansion ||a||^2 + ||v||^2 - 2 a.v cancels by more than 32x.
-__device__ __noinline__ float pair_direct_sqdist(const float* A, const __nv_bfloat16* v) {
-  float s = 0.f;
-  for (int c = 0; c < kHd; c += 4) {
-    const float4 a4 = *reinterpret_cast<const float4*>(A + c);
-    const uint2 v4 = *reinterpret_cast<const uint2*>(v + c);
-    const float d0 = a4.x - __uint_as_float(v4.x << 16);
-    const float d1 = a4.y - __uint_as_float(v4.x & 0xFFFF0000u);
-    const float d2 = a4.z - __uint_as_float(v4.y << 16);
-    const float d3 = a4.w - __uint_as_float(v4.y & 0xFFFF0000u);
-    s = fmaf(d0, d0, s);
-    s = fmaf(d1, d1, s);
-    s = fmaf(d2, d2, s);
-    s = fmaf(d3, d3, s);
-  }
-  return s;
-}
-
-// Careful path of phase B, out of line: ratio^2 (r2, 0 where invisible) times
-// the squared distance, recomputed directly where the expansion cancels by
-// more than 32x.
-__device__ __noinline__ float pairB_careful(const uint32_t* d, const float* r2, int col0,
-                                            const float4* qstat_rows, float nv, const float* arows,
-                                            const __nv_bfloat16* vrow) {
-  float acc = 0.f;
-#pragma unroll 1
-  for (int u = 0; u < 16; ++u) {
-    if (!(r2[u] > 0.f)) continue;  // invisible (or an exact zero weight)
-    const float base = qstat_rows[col0 + u].w + nv;
-    float zt = base + f32(d[u]);
-    if (zt < 0.03125f * base) zt = pair_direct_sqdist(arows + (size_t)(col0 + u) * kHd, vrow);
-    acc = fmaf(r2[u], zt, acc);
-  }
-  return acc;
-}
-
-__global__ void __maxnreg__(112)
+__global__ void __maxnreg__(kMaxRegs2)
 k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmAhi,
                 const __grid_constant__ CUtensorMap tmAlo, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int nqc = a.nqc2, half = nqc / 2;
+  const int nqc = a.nqc2;
+  const int nh = nqc > 128 ? 2 : 1;       // query halves per step
+  const int nqh = nqc / nh;               // columns per half (multiple of 16, <= 128)
+  const int hr = nqh / 2;                 // rows of a half held by each CTA
+  const int rows = nqc / 2;               // query rows held by each CTA
   uint8_t* sRing = smem;                          // kRingP slots
-  uint8_t* sQ = smem + kRingP * kTileBytes;       // half rows x 2 boxes
-  uint8_t* sAh = sQ + half * 256;
-  uint8_t* sAl = sAh + half * 256;
-  float4* kf = reinterpret_cast<float4*>(sAl + half * 256);  // [nqc/2] fast-path constants
-  float* nAmax = reinterpret_cast<float*>(kf + half);           // [16] max ||A||^2 per 16 columns
+  uint8_t* sQ = smem + kRingP * kTileBytes;       // rows x 2 boxes; half h at rows [h hr, +hr)
+  uint8_t* sAh = sQ + rows * 256;
+  uint8_t* sAl = sAh + rows * 256;
+  float4* kf = reinterpret_cast<float4*>(sAl + rows * 256);  // [nqc/2] fast-path constants
+  float* nAmax = reinterpret_cast<float*>(kf + nqc / 2);       // [16] max ||A||^2 per 16 columns
   uint64_t* bars = reinterpret_cast<uint64_t*>(nAmax + 16);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * kRingP);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -151,19 +75,21 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int L = a.L[b];
   const int z = b * a.Hkv + h;
   const int qrow0 = z * a.nq + chunk * nqc;           // the chunk's first query row
-  // barriers (leader's copies gather both CTAs): BQ, FULL[r] -- arrivals of
-  // both producers; EMPTY[r], S_READY, D_READY -- the leader's commits,
-  // multicast to both CTAs; S_FREE, D_FREE -- the 32 score warps of the pair
+  // barriers (the leader's copies gather both CTAs): BQ, FULL[r] -- arrivals
+  // of both producers; TF[2] -- the 32 score warps of the pair hand a TMEM
+  // buffer back; EMPTY[r], MD[2] -- the leader's commits, multicast to both
+  // CTAs; FIN -- the leader's MMAs are all done
   const uint32_t BQ = smem_u32(&bars[0]);
-  const uint32_t SREADY = smem_u32(&bars[1]), DREADY = smem_u32(&bars[2]);
-  const uint32_t SFREE = smem_u32(&bars[3]), DFREE = smem_u32(&bars[4]);
+  auto MD = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto TF = [&](int s) { return smem_u32(&bars[3 + s]); };
   auto FULL = [&](int r) { return smem_u32(&bars[5 + r]); };
   auto EMPTY = [&](int r) { return smem_u32(&bars[5 + kRingP + r]); };
-  const uint32_t FIN = smem_u32(&bars[5 + 2 * kRingP]);  // the leader's MMAs are all done
+  const uint32_t FIN = smem_u32(&bars[5 + 2 * kRingP]);
   if (threadIdx.x == 0) {
     mbar_init(BQ, 2);
-    mbar_init(SREADY, 1); mbar_init(DREADY, 1);
-    mbar_init(SFREE, 2 * kSimtWarps); mbar_init(DFREE, 2 * kSimtWarps);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(MD(s), 1); mbar_init(TF(s), 2 * kSimtWarps);
+    }
     for (int r = 0; r < kRingP; ++r) {
       mbar_init(FULL(r), 2); mbar_init(EMPTY(r), 1);
     }
@@ -172,10 +98,14 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (!aligned) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
     fence_mbar_init();
   }
+  if (warp == kWarpMma) {
+    tmem_alloc2(smem_u32(tmem_slot), 512);
+    tmem_relinquish2();
+    tc_fence_before();
+  }
   pdl_trigger();
   pdl_wait();  // qstat, A and ||v||^2 come from the combine and pass 1
-  // per-column constants of the whole chunk (each CTA's score warps see all
-  // nqc columns of its tokens)
+  // per-column constants of the whole chunk
   for (int i = threadIdx.x; i < nqc; i += blockDim.x) {
     const float4 q = a.qstat[qrow0 + i];  // (M, 1/L, L, ||A||^2)
     float* kff = reinterpret_cast<float*>(kf);
@@ -183,11 +113,6 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     kff[(i >> 1) * 4 + 2 + (i & 1)] = q.w;
   }
   if (threadIdx.x < 16) nAmax[threadIdx.x] = 0.f;
-  if (warp == kWarpMma) {
-    tmem_alloc2(smem_u32(tmem_slot), 512);
-    tmem_relinquish2();
-    tc_fence_before();
-  }
   __syncthreads();
   for (int i = threadIdx.x; i < nqc; i += blockDim.x)  // ||A||^2 >= 0: float bits order as ints
     atomicMax(reinterpret_cast<int*>(nAmax) + i / 16, __float_as_int(a.qstat[qrow0 + i].w));
@@ -215,17 +140,21 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (lane == 0 && !*abort_flag) {
       prefetch_tmap(&tmQ); prefetch_tmap(&tmAhi); prefetch_tmap(&tmAlo);
       prefetch_tmap(&tmK); prefetch_tmap(&tmV);
-      // this CTA's half of the query-side operands; completion counted at the leader
+      // this CTA's rows of every half of the query-side operands; completion
+      // counted at the leader
       const uint32_t cBQ = mapa_u32(BQ, 0);
-      mbar_expect_tx_cluster(cBQ, (uint32_t)((lo ? 3 : 2) * half * 256));
-      const int hrow = qrow0 + (int)rank * half;
-      tma_load_2d_pair(smem_u32(sQ), &tmQ, cBQ, 0, hrow);
-      tma_load_2d_pair(smem_u32(sQ) + half * 128, &tmQ, cBQ, 64, hrow);
-      tma_load_2d_pair(smem_u32(sAh), &tmAhi, cBQ, 0, hrow);
-      tma_load_2d_pair(smem_u32(sAh) + half * 128, &tmAhi, cBQ, 64, hrow);
-      if (lo) {
-        tma_load_2d_pair(smem_u32(sAl), &tmAlo, cBQ, 0, hrow);
-        tma_load_2d_pair(smem_u32(sAl) + half * 128, &tmAlo, cBQ, 64, hrow);
+      mbar_expect_tx_cluster(cBQ, (uint32_t)((lo ? 3 : 2) * rows * 256));
+      for (int hh = 0; hh < nh; ++hh) {
+        const int grow = qrow0 + hh * nqh + (int)rank * hr;  // global query row
+        const uint32_t so = (uint32_t)(hh * hr * 128);       // smem row offset
+        tma_load_2d_pair(smem_u32(sQ) + so, &tmQ, cBQ, 0, grow);
+        tma_load_2d_pair(smem_u32(sQ) + rows * 128 + so, &tmQ, cBQ, 64, grow);
+        tma_load_2d_pair(smem_u32(sAh) + so, &tmAhi, cBQ, 0, grow);
+        tma_load_2d_pair(smem_u32(sAh) + rows * 128 + so, &tmAhi, cBQ, 64, grow);
+        if (lo) {
+          tma_load_2d_pair(smem_u32(sAl) + so, &tmAlo, cBQ, 0, grow);
+          tma_load_2d_pair(smem_u32(sAl) + rows * 128 + so, &tmAlo, cBQ, 64, grow);
+        }
       }
       // K_i at load 2i, V_i at 2i + 1; a step past this CTA's tiles only arrives
       for (int i = 0; i < 2 * steps && !*abort_flag; ++i) {
@@ -247,59 +176,61 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else if (warp == kWarpMma) {
     if (leader) {
-      const uint32_t IDT = idesc_bf16(256, nqc, false, false);
+      const uint32_t IDT = idesc_bf16(256, nqh, false, false);
       bool ok = !warp_aborted(abort_flag);
       if (ok && !(ok = __all_sync(0xffffffffu, mbar_wait_cluster(BQ, 0, kWaitNs))))
         fail(a, abort_flag);
       const SDesc rd0 = sdesc_split(smem_u32(sRing), 16, 1024);
       const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024), hd = sdesc_split(smem_u32(sAh), 16, 1024),
                   ld = sdesc_split(smem_u32(sAl), 16, 1024);
-      const uint32_t hq = (uint32_t)half;
+      const uint32_t rw = (uint32_t)rows;
+      int k = 0;  // (step, half) item: TMEM buffer k & 1
       for (int i = 0; i < steps && ok && !warp_aborted(abort_flag); ++i) {
         const int rk = (2 * i) % kRingP, pk = ((2 * i) / kRingP) & 1;
         const int rv = (2 * i + 1) % kRingP, pv = ((2 * i + 1) / kRingP) & 1;
-        const uint32_t pph = (uint32_t)((i - 1) & 1);
-        // S^T = K Q^T once both CTAs' K tiles are in and the S columns are free
+        // both CTAs' K and V tiles of this step
         if (!__all_sync(0xffffffffu, mbar_wait_cluster(FULL(rk), pk, kWaitNs)) ||
-            (i > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(SFREE, pph, kWaitNs)))) {
-          fail(a, abort_flag);
+            !__all_sync(0xffffffffu, mbar_wait_cluster(FULL(rv), pv, kWaitNs))) {
+          ok = false;
           break;
         }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t klo = rd0.lo + (uint32_t)rk * (kTileBytes >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma2_ss_w(tbase, klo + kslice(kk, 128), rd0.hi, qd.lo + kslice(kk, hq), qd.hi, IDT,
-                      kk > 0 ? 1u : 0u);
-          mma2_commit_mc(EMPTY(rk), 3);
-          mma2_commit_mc(SREADY, 3);
-        }
-        __syncwarp();
-        // D = V (-2A)^T once both V tiles are in and the D columns are free
-        if (!__all_sync(0xffffffffu, mbar_wait_cluster(FULL(rv), pv, kWaitNs)) ||
-            (i > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(DFREE, pph, kWaitNs)))) {
-          fail(a, abort_flag);
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t vlo = rd0.lo + (uint32_t)rv * (kTileBytes >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma2_ss_w(tbase + kColD, vlo + kslice(kk, 128), rd0.hi, hd.lo + kslice(kk, hq), hd.hi,
-                      IDT, kk > 0 ? 1u : 0u);
-          if (lo) {
+        for (int hh = 0; hh < nh; ++hh, ++k) {
+          const int s = k & 1;
+          // the buffer's previous item has been read by all 32 score warps
+          if (k >= 2 &&
+              !__all_sync(0xffffffffu, mbar_wait_cluster(TF(s), (uint32_t)(((k >> 1) - 1) & 1),
+                                                         kWaitNs))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t dS = tbase + (uint32_t)(s * 256), dD = dS + 128u;
+            const uint32_t klo = rd0.lo + (uint32_t)rk * (kTileBytes >> 4);
+            const uint32_t vlo = rd0.lo + (uint32_t)rv * (kTileBytes >> 4);
+            const uint32_t ho = (uint32_t)(hh * hr * 128) >> 4;  // half's row offset
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma2_ss_w(tbase + kColD, vlo + kslice(kk, 128), rd0.hi, ld.lo + kslice(kk, hq),
-                        ld.hi, IDT, 1u);
+              mma2_ss_w(dS, klo + kslice(kk, 128), rd0.hi, qd.lo + ho + kslice(kk, rw), qd.hi, IDT,
+                        kk > 0 ? 1u : 0u);
+            if (hh == nh - 1) mma2_commit_mc(EMPTY(rk), 3);  // the last reader of K_i
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma2_ss_w(dD, vlo + kslice(kk, 128), rd0.hi, hd.lo + ho + kslice(kk, rw), hd.hi, IDT,
+                        kk > 0 ? 1u : 0u);
+            if (lo) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma2_ss_w(dD, vlo + kslice(kk, 128), rd0.hi, ld.lo + ho + kslice(kk, rw), ld.hi,
+                          IDT, 1u);
+            }
+            if (hh == nh - 1) mma2_commit_mc(EMPTY(rv), 3);  // the last reader of V_i
+            mma2_commit_mc(MD(s), 3);
           }
-          mma2_commit_mc(EMPTY(rv), 3);
-          mma2_commit_mc(DREADY, 3);
+          __syncwarp();
         }
-        __syncwarp();
       }
+      if (!ok) fail(a, abort_flag);
       // whatever was issued (all of it, or less after a timeout) has completed
       // before either CTA frees its TMEM
       if (lane == 0) mma2_commit_mc(FIN, 1);
@@ -308,112 +239,94 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else if (warp < kSimtWarps) {
     // Sixteen warps per CTA: warp (g, quarter) owns the tokens [32 quarter,
-    // +32) of this CTA's tile (its TMEM lanes) and the 16-column chunks
-    // [ch0, ch0 + nch) of the query columns, and writes its own partial-score
-    // plane (the epilogue sums the four planes of a chunk).
+    // +32) of this CTA's tile (its TMEM lanes) and the query columns
+    // [32 g, min(nqh, 32 g + 32)) of every half, and writes its own
+    // partial-score plane (the epilogue sums the four planes of a chunk).
     const int g = warp >> 2, ql = warp & 3;
     const int row = ql * 32 + lane;
     const uint32_t lane_off = (uint32_t)(ql * 32) << 16;
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
-    const int ncht = nqc / 16;
-    const int ch0 = g * ncht / 4, nch = (g + 1) * ncht / 4 - ch0;  // 0..4, warp-uniform
+    const int ch0 = min(nqh / 16, 2 * g), ch1 = min(nqh / 16, 2 * g + 2);  // 16-column chunks
+    const int nch = ch1 - ch0;  // 0, 1 or 2 (warp-uniform)
     const float4* qrows = a.qstat + qrow0;
     const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
     float* plane = a.parts + (size_t)(chunk * 4 + g) * a.part_stride + (size_t)z * a.n_max;
-    const uint32_t cSFREE = mapa_u32(SFREE, 0), cDFREE = mapa_u32(DFREE, 0);
-    const uint32_t tS = tbase + lane_off + (uint32_t)(ch0 * 16);
-    const uint32_t tD = tS + kColD;
+    const uint32_t cTF0 = mapa_u32(TF(0), 0), cTF1 = mapa_u32(TF(1), 0);
     auto nv_at = [&](int st) -> float {
       const int tk = tile_at(st) * kTok + row;
       return (st < my_n && tk < L) ? a.nvbuf[(size_t)z * a.ntmax * kTok + tk] : 0.f;
     };
     float nv_next = nv_at(0);
     int sing = 0;
+    int k = 0;
     bool live = !warp_aborted(abort_flag);
     for (int i = 0; i < steps && live; ++i) {
-      const bool valid_tile = i < my_n;
+      const bool valid_tile = i < my_n;  // warp-uniform
       const int tile0 = (valid_tile ? tile_at(i) : my0) * kTok;
       const int tok = tile0 + row;
       const bool valid = valid_tile && tok < L;
-      const bool masked = !valid_tile || tile0 + kTok - 1 > L - a.w;  // warp-uniform
+      const bool masked = tile0 + kTok - 1 > L - a.w;  // warp-uniform
       const float nv = nv_next;
       nv_next = nv_at(i + 1);
       const __nv_bfloat16* vrow = a.v + ((size_t)z * a.n_max + (valid ? tok : 0)) * kHd;
-      // ---- phase A: ratio^2 of every owned column, then the S columns go back
-      if (!__all_sync(0xffffffffu, mbar_wait_cluster(SREADY, (uint32_t)(i & 1), kWaitNs))) {
-        fail(a, abort_flag);
-        break;
-      }
-      if (warp_aborted(abort_flag)) break;
-      tc_fence_after();
-      uint64_t r2[4][8];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        if (cc >= nch) break;
-        uint32_t r[16];
-        tmem_ld16(tS + 16u * cc, r);
-        bool redo = masked;
-        if (!masked) {
-          float pmax = 0.f;
-          pairA_fast(r, kf + (ch0 + cc) * 8, c2, r2[cc], pmax);
-          redo = pmax >= 0.0625f;  // a large p: the series would be short
-        }
-        if (__any_sync(0xffffffffu, redo)) {
-          float t16[16];
-          pairA_careful(r, (ch0 + cc) * 16, tok, valid, masked, L, a.w, chunk * nqc, qrows, c,
-                        &sing, t16);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) r2[cc][k] = pk2(t16[2 * k], t16[2 * k + 1]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(cSFREE);
-      // ---- phase B: D of the owned columns; the D columns go back once read
-      if (!__all_sync(0xffffffffu, mbar_wait_cluster(DREADY, (uint32_t)(i & 1), kWaitNs))) {
-        fail(a, abort_flag);
-        break;
-      }
-      tc_fence_after();
       float acc = 0.f;
-      if (nch == 0) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(cDFREE);
-      }
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        if (cc >= nch) break;
-        uint32_t d[16];
-        tmem_ld16(tD + 16u * cc, d);
-        if (cc == nch - 1) {
+      for (int hh = 0; hh < nh; ++hh, ++k) {
+        const int s = k & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait_cluster(MD(s), (uint32_t)((k >> 1) & 1), kWaitNs))) {
+          fail(a, abort_flag);
+          live = false;
+          break;
+        }
+        if (warp_aborted(abort_flag)) { live = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tbase + (uint32_t)(s * 256) + lane_off + (uint32_t)(ch0 * 16);
+        const uint32_t tD = tS + 128u;
+        const int hc0 = hh * nqh;  // the half's first column within the chunk
+        auto release = [&]() {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(cDFREE);
-        }
-        // possible cancellation (||A||^2 >= 0.6 ||v||^2) or masked keys: careful
-        const bool cb = masked || nAmax[ch0 + cc] >= 0.6f * nv;
-        if (__any_sync(0xffffffffu, cb)) {
-          float t16[16];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) upk2(r2[cc][k], t16[2 * k], t16[2 * k + 1]);
-          acc += pairB_careful(d, t16, (ch0 + cc) * 16, qrows, nv, arows, vrow);
-        } else {
-          const uint64_t nv2 = pk2(nv, nv);
+          if (lane == 0) mbar_arrive_cluster(s ? cTF1 : cTF0);
+        };
+        // score of 16 columns (chunk ch of the half) from S^T in r[0..15] and D
+        // in r[16..31]
+        auto chunk_score = [&](const uint32_t(&r)[32], int ch) -> float {
+          bool redo = masked;
           uint64_t a2 = pk2(0.f, 0.f);
+          if (!masked) {
+            float pmax = 0.f;
+            fast16(r, kf + (hc0 / 2) + ch * 8, c2, pk2(nv, nv), a2, pmax);
+            // a large p (>= 2^-4: the series above would be short) or possible
+            // cancellation (||A||^2 >= 0.6 ||v||^2): the careful path
+            redo = pmax >= 0.0625f || nAmax[hc0 / 16 + ch] >= 0.6f * nv;
+          }
+          if (__any_sync(0xffffffffu, redo)) {
+            uint32_t rc[32];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float4 kq = kf[(ch0 + cc) * 8 + k];
-            const uint64_t zt = fadd2(fadd2(pk2(f32(d[2 * k]), f32(d[2 * k + 1])), pk2(kq.z, kq.w)), nv2);
-            a2 = ffma2(r2[cc][k], zt, a2);
+            for (int q = 0; q < 32; ++q) rc[q] = r[q];
+            return careful16(rc, hc0 + ch * 16, tok, masked, L, a.w, chunk * nqc, qrows, c, nv,
+                             arows, vrow, &sing);
           }
           float x0, x1;
           upk2(a2, x0, x1);
-          acc += x0 + x1;
+          return x0 + x1;
+        };
+        if (nch == 0 || !valid_tile) {
+          // no columns, or a step past this CTA's tiles: only hand the buffer back
+          release();
+          continue;
+        }
+        uint32_t r[32];
+        tmem_ld16x2(tS, tD, r);  // chunk ch0: 16 columns of S^T and of D
+        if (nch == 1) release();
+        acc += chunk_score(r, ch0);
+        if (nch > 1) {
+          tmem_ld16x2(tS + 16u, tD + 16u, r);  // chunk ch0 + 1
+          release();
+          acc += chunk_score(r, ch0 + 1);
         }
       }
-      if (valid) plane[tok] = acc;
+      if (live && valid) plane[tok] = acc;
     }
     if (sing) atomicMax(a.status, (int)DROPKV_ERR_SINGULAR);
   }
@@ -427,7 +340,6 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     tmem_dealloc2(tbase, 512);
   }
 }
-
 }  // namespace
 
 size_t pass2_pair_smem(int nqc) {
