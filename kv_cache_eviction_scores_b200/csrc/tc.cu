@@ -9,42 +9,34 @@
 // summed over all G*w window queries of the group (the GQA sum; the epilogue
 // divides by G).  No n x w matrix is stored: two streaming passes over K/V.
 //
-// Work split.  The G*w query rows of a KV head are cut into `chunks` chunks of
-// nqc <= 128 rows; the tokens of each (b, h, chunk) into `splits` contiguous
-// tile ranges so that about one CTA runs per SM.  Tiles are 128 tokens.
+// Work split.  The tokens of each (b, h, query chunk) unit are cut into
+// `splits` contiguous ranges of 128-token tiles so that about one CTA runs per
+// SM.  Pass 1 takes chunks of <= 256 query rows (two tiles of 128); the
+// DropKV second pass (tc_pair.cu) runs on CTA pairs; the attention-only
+// second pass below takes chunks of nqc <= 128 rows.
 //
 // k_tc_pass1 (query-major, one CTA per (b, h, chunk, split)):
-//   S = Q_chunk K_tile^T      tcgen05 M=128 (queries) N=128 (tokens) K=128
-//   online softmax per query row (log2 domain; the reference max only moves up
-//   by more than 8, so exp2 stays <= 256 and O rarely rescales).  Sixteen
-//   softmax warps share every tile: each owns 32 rows x 32 tokens, posts its
-//   row maxima for the other three warps of its rows and, one tile behind,
-//   writes P = exp2(S*c - m) back over S in TMEM as two bf16 planes,
-//   P_hi = P truncated to bf16 and P_lo = bf16(P - P_hi), so P_hi + P_lo holds
-//   P to 2^-16 relative;  O += P_hi V + P_lo V   (A from TMEM, V MN-major).
-//   Three S/P buffers let S run two tiles ahead of P V.  Each CTA writes one
-//   partial (m, l, O) per row.
+//   S_t = Q_t K_tile^T for both query tiles t, tcgen05 M=128 (queries) N=128
+//   (tokens) K=128; one softmax warpgroup per query tile, one query row per
+//   thread: a max pass over the row's 128 logits, then P = exp2(S*c - m)
+//   written back over S in TMEM as two bf16 planes, P_hi = P truncated to
+//   bf16 and P_lo = bf16(P - P_hi), so P_hi + P_lo holds P to 2^-16 relative;
+//   O_t += P_hi V + P_lo V (A from TMEM, V MN-major).  The reference max only
+//   moves up by more than 8, so exp2 stays <= 256 and O rarely rescales.
+//   While one query tile's softmax runs, the other tile's MMAs keep the
+//   tensor pipe busy.  Each CTA writes one partial (m, l, O) per row.
 // k_tc_combine: merges the partials of a row into the final max M, normaliser
 //   L and output A = O / L; writes -2A as bf16 hi/lo planes (same split) plus
-//   the per-query constants (M, 1/L, L, ||A||^2) for pass 2.
-// k_tc_pass2 (token-major, one CTA per (b, h, chunk, split)):
-//   S^T = K_tile Q^T and D = V_tile (-2A_hi)^T [+ V_tile (-2A_lo)^T], tcgen05
-//   M=128 (tokens) N=nqc (queries) K=128, into two TMEM buffers; each thread
-//   owns one token and sums over its warp's 32 queries:  p = exp2(S*c - M'),
-//   M' = M + log2 L; while p < 2^-4 the series p(1 + p(1 + p(1 + p(1 + p))))
-//   gives p / (1 - p); otherwise ratio = e / (L - e) with the singular check
-//   (L - e not > 0 => rejected); s += ratio^2 * (||A||^2 + ||v_j||^2 + D);
-//   where that expansion cancels by more than 32x (A close to v_j: a dominant
-//   token) the squared distance is recomputed directly from fp32 A and v_j.
-//   A warp hands its TMEM buffer back once its last columns are in registers.
-//   The attention-only control score (section 结果与独立对照) is the same
-//   kernel instantiated with kAttn: K tiles only, S^T only, s += p.
+//   the per-query constants (M, 1/L, L, ||A||^2) for the second pass.
+// k_tc_pass2<true> (token-major, one CTA per (b, h, chunk, split)): the
+//   attention-only control score (section 结果与独立对照): S^T = K_tile Q^T,
+//   tcgen05 M=128 (tokens) N=nqc (queries) K=128, into two TMEM buffers; each
+//   thread owns one token and sums p = exp2(S*c - M') over its warp's
+//   queries, M' = M + log2 L.  K tiles only.
 //
-// Warp roles: sixteen score / softmax warps (4 per TMEM lane quarter), one
-// warp issuing TMA loads, one allocating TMEM and issuing MMAs (lane 0), and in
-// pass 1 one more warp computing ||v_j||^2.  Every wait on an mbarrier is
-// bounded (2 s of %globaltimer); on expiry the kernel records
-// DROPKV_ERR_TIMEOUT, every role leaves its loop and TMEM is freed.
+// Every wait on an mbarrier is bounded (2 s of %globaltimer); on expiry the
+// kernel records DROPKV_ERR_TIMEOUT, every role leaves its loop and TMEM is
+// freed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -59,45 +51,32 @@ namespace dropkv {
 namespace {
 
 // =========================== pass 1 =========================================
-// Writes P = exp2(S c - mu) for 32 tokens of one query row (S already in
-// registers, masked keys at -inf) as hi/lo bf16 planes over the same 32 TMEM
-// columns: tokens 16k..16k+15 keep hi in columns [16k, 16k+8) and lo in
-// [16k+8, 16k+16).  Returns the row's sum of P over the 32 tokens.
-// Warp-collective.
-__device__ __forceinline__ float p1_exp32(const uint32_t (&sr)[32], uint32_t tS, uint64_t c2,
-                                          float mu) {
-  const uint64_t nmu2 = pk2(-mu, -mu);
+// P = exp2(S c - mu) for 16 tokens of one query row (S in s16[0..15], masked
+// keys at -inf) written as 8 hi + 8 lo bf16 pair columns at TMEM column tcol
+// (the layout P V reads: hi of the 16 tokens, then lo).  No wait on the store.
+// Returns the sum of P over the 16 tokens.  Warp-collective.
+__device__ __forceinline__ float p1_exp16(const uint32_t* s16, uint32_t tcol, uint64_t c2,
+                                          uint64_t nmu2) {
   uint64_t l2 = pk2(0.f, 0.f);
-  uint32_t pw[32];  // columns: hi of tokens 0-15, lo of 0-15, hi of 16-31, lo of 16-31
+  uint32_t pw[16];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {  // 16 tokens -> 8 hi + 8 lo columns
-#pragma unroll
-    for (int u2 = 0; u2 < 8; ++u2) {
-      const int u = half * 16 + 2 * u2;
-      float d0, d1;
-      upk2(ffma2(pk2(f32(sr[u]), f32(sr[u + 1])), c2, nmu2), d0, d1);
-      const float e0 = ex2(d0), e1 = ex2(d1);
-      const uint64_t E = pk2(e0, e1);
-      l2 = fadd2(l2, E);
-      pw[half * 16 + u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
-      const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
-      const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
-      float r0, r1;
-      upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
-      pw[half * 16 + 8 + u2] = pack_bf16_rn(r0, r1);
-    }
+  for (int u2 = 0; u2 < 8; ++u2) {
+    float d0, d1;
+    upk2(ffma2(pk2(f32(s16[2 * u2]), f32(s16[2 * u2 + 1])), c2, nmu2), d0, d1);
+    const float e0 = ex2(d0), e1 = ex2(d1);
+    const uint64_t E = pk2(e0, e1);
+    l2 = fadd2(l2, E);
+    pw[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
+    const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);
+    const float nh1 = f32((u32(e1) & 0xFFFF0000u) | 0x80000000u);
+    float r0, r1;
+    upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
+    pw[8 + u2] = pack_bf16_rn(r0, r1);
   }
-  tmem_st32(tS, pw);  // one TMEM store for the warp's 32 columns
+  tmem_st16(tcol, pw);
   float la, lb;
   upk2(l2, la, lb);
   return la + lb;
-}
-
-// Causal mask of 32 tokens starting at tok0 for a query at position prow.
-__device__ __forceinline__ void p1_mask32(uint32_t (&sr)[32], int tok0, int prow) {
-#pragma unroll
-  for (int u = 0; u < 32; ++u)
-    if (tok0 + u > prow) sr[u] = 0xFF800000u;  // -inf
 }
 
 // Rare path of pass 1, out of line: the reference max of some rows moved
@@ -356,17 +335,19 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       const int tok0 = (t0 + j) * kTok;
       const bool masked = tok0 + kTok - 1 > L - a.w;  // only the last tiles hide keys past P_t
-      uint32_t sr[32];
-      float ya = -INFINITY, yb = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        tmem_ld32(tS + 32u * cc, sr);
-        if (masked) p1_mask32(sr, tok0 + 32 * cc, Prow);
+      // the row's 128 logits in one TMEM load (one round trip per tile)
+      uint32_t sr[128];
+      tmem_ld128(tS, sr);
+      if (masked) {
 #pragma unroll
-        for (int u = 0; u < 32; u += 4) {
-          ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
-          yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
-        }
+        for (int u = 0; u < 128; ++u)
+          if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
+      }
+      float ya = -INFINITY, yb = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 128; u += 4) {
+        ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
+        yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
       }
       const float mt = fmaxf(ya, yb) * c;  // c > 0: commutes with the max
       float fac = 1.f;
@@ -386,12 +367,9 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         break;
       }
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        tmem_ld32(tS + 32u * cc, sr);
-        if (masked) p1_mask32(sr, tok0 + 32 * cc, Prow);
-        l += p1_exp32(sr, tS + 32u * cc, c2, mu);
-      }
+      const uint64_t nmu2 = pk2(-mu, -mu);
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) l += p1_exp16(sr + 16 * cc, tS + 16u * cc, c2, nmu2);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
