@@ -9,8 +9,9 @@
 // Scores map to 32-bit keys whose unsigned order is the float order.  A
 // segment (b, h) of L keys is split into kC contiguous ranges, one per CTA of
 // a kC-CTA cluster; a range is cached in shared memory when it fits.
-// A range is processed in sub-ranges of 16384 keys (one when it fits the
-// shared-memory cache, which then holds it for every phase).
+// The histogram rounds take a range in sub-ranges of 16384 keys, 32
+// consecutive keys per thread (one sub-range when it fits the shared-memory
+// cache, which then holds it for every phase).
 //   rounds 0..2: every CTA histograms an 11/11/10-bit digit of its keys that
 //       match the prefix found so far and adds the histogram into rank 0's
 //       shared memory (distributed shared memory atomics; one histogram per
@@ -20,12 +21,14 @@
 //       broadcast barrier.
 //       After round 2 the prefix is the threshold key T and `rem` is how many
 //       keys equal to T are evicted (the lowest positions among them).
-//   count: every CTA stores its counts of keys < T and == T into every CTA;
-//       each CTA then sums the counts of the lower ranks (the ranges are in
-//       position order).
-//   write: per sub-range of 16384 keys, each thread takes 32 consecutive
-//       keys; two block scans give every thread its kept / evicted ranks, the
-//       positions are staged in shared memory and copied out coalesced.
+//   count: each warp walks a contiguous part of the CTA's range, 32
+//       consecutive keys at a time (lane = key), and counts the keys < T and
+//       == T with ballots; every CTA stores its totals into every CTA, which
+//       then sums the counts of the lower ranks (the ranges are in position
+//       order).
+//   write: the same walk again: the ballots give every lane its evicted rank
+//       and an == T key's rank among the == T keys, and each lane writes its
+//       position straight to its slot of the keep or evict list.
 // The phases are separated by cluster-wide mbarrier phases with bounded waits;
 // a wait that gives up records DROPKV_ERR_TIMEOUT in the status word and the
 // CTA keeps taking the remaining phase barriers (without the work).  The kernel
@@ -191,16 +194,14 @@ template <bool kCached>
 __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 1)
 k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ keep_idx,
          int32_t* __restrict__ evict_idx) {
-  extern __shared__ uint32_t smem_dyn[];     // [kSub] key cache / staging, then histogram copies
+  extern __shared__ uint32_t smem_dyn[];     // [kSub] key cache, then histogram copies
   uint32_t* cached_keys = smem_dyn;          // this CTA's range when it fits one sub-range
-  int32_t* staging = reinterpret_cast<int32_t*>(smem_dyn + (kCached ? kSub : 0));
-  uint32_t* loc = smem_dyn + 2 * kSub;       // [kCopies][kCopyStride] this CTA's histograms
+  uint32_t* loc = smem_dyn + kSub;           // [kCopies][kCopyStride] this CTA's histograms
   __shared__ uint32_t H[3][kBins];           // the cluster histogram of each round (rank 0's)
   __shared__ int32_t warp_tot[kWarps];
   __shared__ uint32_t cnt[kC][2];            // per-rank (#< T, #== T), stored by every rank
   __shared__ uint32_t ctl[2];                // this CTA's (prefix, rem) after a round
   __shared__ int32_t wsum[2][kWarps];
-  __shared__ int32_t bcast[2];
   __shared__ __align__(8) uint64_t bar;     // all-to-all phases (count, final): kC arrivals
   __shared__ __align__(8) uint64_t gbar;    // rank 0: a round's histogram adds landed (kC)
   __shared__ __align__(8) uint64_t bbar;    // every CTA: rank 0 broadcast the round's digit (1)
@@ -345,24 +346,22 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   const uint32_t T = prefix;
   const int quota = E > 0 ? (int)rem : 0;  // keys == T that are evicted
 
-  // ---- counts below / at the threshold, gathered at rank 0 -----------------
+  // ---- counts below / at the threshold, gathered at every CTA --------------
+  // Each warp takes a contiguous, 32-aligned part of the CTA's range and walks
+  // it 32 consecutive keys at a time (lane = key); ballots count the keys
+  // below / at T.  The same walk writes the lists below.
+  const int wlen = ((hi - lo + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int w_lo = min(hi, lo + wid * wlen), w_hi = min(hi, w_lo + wlen);
+  const uint32_t lanelt = (1u << lane) - 1u;
   int nlt = 0, neq = 0;
   if (ok && E > 0)
-    for (int sub0 = lo; sub0 < hi; sub0 += kSub) {
-      uint32_t k[kPer];
-      load_run(sub0, k);
-      const int j0 = sub0 + tid * kPer;
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const bool in = j0 + u < hi;
-        nlt += in && k[u] < T;
-        neq += in && k[u] == T;
-      }
+    for (int c0 = w_lo; c0 < w_hi; c0 += 32) {
+      const int j = c0 + lane;
+      const bool in = j < w_hi;
+      const uint32_t kk = in ? key_at(j) : 0xFFFFFFFFu;
+      nlt += __popc(__ballot_sync(0xffffffffu, in && kk < T));
+      neq += __popc(__ballot_sync(0xffffffffu, in && kk == T));
     }
-  for (int o = 16; o > 0; o >>= 1) {
-    nlt += __shfl_xor_sync(0xffffffffu, nlt, o);
-    neq += __shfl_xor_sync(0xffffffffu, neq, o);
-  }
   if (lane == 0) {
     wsum[0][wid] = nlt;
     wsum[1][wid] = neq;
@@ -379,76 +378,48 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
     dsm_st(dst + 4u, (uint32_t)e);
   }
   ok = cluster_phase(barA, phase, &fail, p.status, p.wait_ns) && ok;
-  if (tid == 0) {
-    int a = 0, e = 0;
-    if (ok)
-      for (uint32_t r = 0; r < rank; ++r) {  // the lower ranks hold the lower positions
-        a += (int)cnt[r][0];
-        e += (int)cnt[r][1];
-      }
-    bcast[0] = a;
-    bcast[1] = e;
-  }
-  __syncthreads();
 
   // ---- order-preserving compaction of this CTA's range ----------------------
-  // Per sub-range: thread t owns keys [sub0 + 32 t, +32).  eq ranks come from
-  // a scan of the per-thread == T counts, evicted counts from a scan of
-  // (#< T + the == T keys within the quota); the sub-range's evicted positions
-  // are staged in shared memory first, its kept positions after them, and both
-  // lists are copied out coalesced (they are contiguous in the outputs).
+  // Per warp, in position order: the keys below / at T before its part (lower
+  // ranks, then lower warps of this CTA), then per 32 keys the ballots give
+  // every lane its evicted rank (those before it) and an == T key's rank among
+  // the == T keys (evicted while below the quota); a kept key's rank is its
+  // position minus the evicted keys before it.  Lanes write their positions
+  // straight to the lists (consecutive lanes, consecutive slots).
   if (ok) {
     int32_t* kout = keep_idx + (size_t)seg * p.max_keep;
     int32_t* eout = evict_idx + (size_t)seg * p.max_evict;
-    int eq_base = bcast[1];                           // keys == T before this sub-range
-    int ev_base = bcast[0] + min(eq_base, quota);     // evicted before this sub-range
+    int lt_run = 0, eq_run = 0;
+    for (uint32_t r = 0; r < rank; ++r) {  // the lower ranks hold the lower positions
+      lt_run += (int)cnt[r][0];
+      eq_run += (int)cnt[r][1];
+    }
+    for (int i = 0; i < wid; ++i) {
+      lt_run += wsum[0][i];
+      eq_run += wsum[1][i];
+    }
+    int ev_run = lt_run + min(eq_run, quota);  // evicted before this warp's part
     const bool any = E > 0;
-    for (int sub0 = lo; sub0 < hi; sub0 += kSub) {
-      uint32_t k[kPer];
-      load_run(sub0, k);
-      const int j0 = sub0 + tid * kPer;
-      int lt = 0, eq = 0;
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const bool in = any && j0 + u < hi;
-        lt += in && k[u] < T;
-        eq += in && k[u] == T;
-      }
-      int eq_tot, ev_tot;
-      const int eq_before = eq_base + block_excl_scan(eq, eq_tot, warp_tot);
-      // evicted == T keys of this thread: those whose eq rank is below the quota
-      const int eq_ev = max(0, min(eq, quota - eq_before));
-      const int ev_before_local = block_excl_scan(lt + eq_ev, ev_tot, warp_tot);
-      const int n_sub = min(kSub, hi - sub0);
-      // stage: evicted at [0, ev_tot), kept at [ev_tot, n_sub) of the sub-range
-      __syncthreads();  // every thread has its keys in registers before the cache is reused
-      int ev_i = ev_before_local, eqr = eq_before;
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int j = j0 + u;
-        if (j >= hi) break;
-        bool ev = false;
-        if (any) {
-          if (k[u] < T) ev = true;
-          else if (k[u] == T) ev = (eqr++ < quota);
-        }
-        if (ev) staging[ev_i++] = j;
-        else staging[ev_tot + (j - sub0) - ev_i] = j;
-      }
-      __syncthreads();
-      for (int i = tid; i < n_sub; i += kThreads) {
-        if (i < ev_tot) {
-          const int r = ev_base + i;
-          // the guards only matter after a wait gave up (inconsistent counts)
-          if (r >= 0 && r < p.max_evict) eout[r] = staging[i];
+    for (int c0 = w_lo; c0 < w_hi; c0 += 32) {
+      const int j = c0 + lane;
+      const bool in = j < w_hi;
+      const uint32_t kk = in ? key_at(j) : 0xFFFFFFFFu;
+      const bool eq = any && in && kk == T;
+      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+      const bool ev = (any && in && kk < T) || (eq && eq_run + __popc(eqm & lanelt) < quota);
+      const uint32_t evm = __ballot_sync(0xffffffffu, ev);
+      const int ev_before = ev_run + __popc(evm & lanelt);
+      if (in) {
+        // the guards only matter after a wait gave up (inconsistent counts)
+        if (ev) {
+          if (ev_before >= 0 && ev_before < p.max_evict) eout[ev_before] = j;
         } else {
-          const int r = (sub0 - ev_base) + (i - ev_tot);  // kept before + local kept rank
-          if (r >= 0 && r < p.max_keep) kout[r] = staging[i];
+          const int r = j - ev_before;
+          if (r >= 0 && r < p.max_keep) kout[r] = j;
         }
       }
-      __syncthreads();
-      eq_base += eq_tot;
-      ev_base += ev_tot;
+      ev_run += __popc(evm);
+      eq_run += __popc(eqm);
     }
     // slots past this row's own counts (rows shorter than the maxima): -1
     if (rank == kC - 1) {
@@ -517,9 +488,9 @@ cudaError_t launch_impl(int B, int Hkv, int n_max, const float* scores, const in
   for (int b = 0; b < B; ++b) max_L = L[b] > max_L ? L[b] : max_L;
   const long long span = (((long long)max_L + kC - 1) / kC + 31) & ~31ll;
   p.cache = span <= kSub ? 1 : 0;
-  // [key cache when it fits][staging][histogram copies]; the histogram copies
-  // always start at 2 * kSub words
-  const size_t smem = (2 * (size_t)kSub + kCopies * (size_t)kCopyStride) * sizeof(uint32_t);
+  // [key cache when it fits][histogram copies]; the histogram copies always
+  // start at kSub words
+  const size_t smem = ((size_t)kSub + kCopies * (size_t)kCopyStride) * sizeof(uint32_t);
   auto kern = p.cache ? k_select<true> : k_select<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
