@@ -55,24 +55,16 @@ namespace {
 // keys at -inf) written as 8 hi + 8 lo bf16 pair columns at TMEM column tcol
 // (the layout P V reads: hi of the 16 tokens, then lo).  No wait on the store.
 // Returns the sum of P over the 16 tokens.  Warp-collective.
-template <int kPoly = 0>
 __device__ __forceinline__ float p1_exp16(const uint32_t* s16, uint32_t tcol, uint64_t c2,
                                           uint64_t nmu2) {
   uint64_t l2 = pk2(0.f, 0.f);
   uint32_t pw[16];
 #pragma unroll
   for (int u2 = 0; u2 < 8; ++u2) {
-    const uint64_t d = ffma2(pk2(f32(s16[2 * u2]), f32(s16[2 * u2 + 1])), c2, nmu2);
-    uint64_t E;
-    if (u2 < kPoly) {  // these token pairs on the FMA pipe, the rest on the SFU
-      E = exp2_fma2(d);
-    } else {
-      float d0, d1;
-      upk2(d, d0, d1);
-      E = pk2(ex2(d0), ex2(d1));
-    }
-    float e0, e1;
-    upk2(E, e0, e1);
+    float d0, d1;
+    upk2(ffma2(pk2(f32(s16[2 * u2]), f32(s16[2 * u2 + 1])), c2, nmu2), d0, d1);
+    const float e0 = ex2(d0), e1 = ex2(d1);
+    const uint64_t E = pk2(e0, e1);
     l2 = fadd2(l2, E);
     pw[u2] = __byte_perm(u32(e0), u32(e1), 0x7632);  // truncated bf16 pair
     const float nh0 = f32((u32(e0) & 0xFFFF0000u) | 0x80000000u);

@@ -124,34 +124,6 @@ __device__ __forceinline__ bool warp_aborted(volatile int* f) {
 __device__ __forceinline__ uint32_t kslice(int kk, uint32_t rows) {
   return (uint32_t)(kk >> 2) * rows * 8u + (uint32_t)(kk & 3) * 2u;
 }
-// 2^y for both halves of a packed pair without the SFU: y = n + f with n the
-// nearest integer (the rounding of y + 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f
-// from a degree-5 polynomial fitted to the relative error of 2^f on that
-// interval (csrc/fit_exp2_poly.py; 2.2e-7 at most in fp32 Horner arithmetic,
-// the SFU's ex2.approx is of the same order); 2^n is added to the exponent
-// field.  y < -125 (and -inf) gives 0; y must stay below 128.
-constexpr float kE2c0 = 1.0000001192092896f, kE2c1 = 0.6931469440460205f,
-                kE2c2 = 0.24022120237350464f, kE2c3 = 0.05550713464617729f,
-                kE2c4 = 0.009675540961325169f, kE2c5 = 0.001327641773968935f;
-__device__ __forceinline__ uint64_t exp2_fma2(uint64_t y) {
-  const uint64_t t = fadd2(y, pk2(12582912.f, 12582912.f));
-  const uint64_t n = fadd2(t, pk2(-12582912.f, -12582912.f));
-  const uint64_t f = ffma2(n, pk2(-1.f, -1.f), y);  // exact: y - n
-  uint64_t q = ffma2(f, pk2(kE2c5, kE2c5), pk2(kE2c4, kE2c4));
-  q = ffma2(f, q, pk2(kE2c3, kE2c3));
-  q = ffma2(f, q, pk2(kE2c2, kE2c2));
-  q = ffma2(f, q, pk2(kE2c1, kE2c1));
-  q = ffma2(f, q, pk2(kE2c0, kE2c0));
-  float y0, y1, t0, t1, q0, q1;
-  upk2(y, y0, y1);
-  upk2(t, t0, t1);
-  upk2(q, q0, q1);
-  // the low bits of t hold n: shifted into the exponent field they scale q by 2^n
-  const uint32_t r0 = y0 < -125.f ? 0u : u32(q0) + (u32(t0) << 23);
-  const uint32_t r1 = y1 < -125.f ? 0u : u32(q1) + (u32(t1) << 23);
-  return pk2(f32(r0), f32(r1));
-}
-
 // =========================== second-pass scoring ===========================
 // ||a - v||^2 taken directly (fp32 a, bf16 v, both from global memory).  Used
 // only where the expansion ||a||^2 + ||v||^2 - 2 a.v cancels by more than 32x,
@@ -180,24 +152,16 @@ __device__ __noinline__ float direct_sqdist(const float* A, const __nv_bfloat16*
 //   (relative truncation error p^5 / (1 - p) <= 1.0e-6 for p < 2^-4),
 //   s += ratio^2 (D' + ||A||^2 + ||v||^2)   with D' = -2 A.v from the MMA.
 // kf holds (-M'_t, -M'_t+1, ||A_t||^2, ||A_t+1||^2) per column pair.
-template <int kPoly = 0>
 __device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf, uint64_t c2,
                                        uint64_t nv2, uint64_t& acc2, float& pmax) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 k = kf[i];
-    const uint64_t y = ffma2(pk2(f32(r[2 * i]), f32(r[2 * i + 1])), c2, pk2(k.x, k.y));
-    uint64_t P;
-    if (i < kPoly) {  // these column pairs on the FMA pipe, the rest on the SFU
-      P = exp2_fma2(y);
-    } else {
-      float y0, y1;
-      upk2(y, y0, y1);
-      P = pk2(ex2(y0), ex2(y1));
-    }
-    float p0, p1;
-    upk2(P, p0, p1);
+    float y0, y1;
+    upk2(ffma2(pk2(f32(r[2 * i]), f32(r[2 * i + 1])), c2, pk2(k.x, k.y)), y0, y1);
+    const float p0 = ex2(y0), p1 = ex2(y1);
     pmax = fmax3(pmax, p0, p1);
+    const uint64_t P = pk2(p0, p1);
     const uint64_t one = pk2(1.f, 1.f);
     const uint64_t ratio = fmul2(P, ffma2(P, ffma2(P, ffma2(P, fadd2(P, one), one), one), one));
     const uint64_t zt = fadd2(fadd2(pk2(f32(r[16 + 2 * i]), f32(r[16 + 2 * i + 1])),

@@ -81,50 +81,3 @@ def test_dropping_the_low_part_bound():
         z = np.sum((a - v) ** 2)
         worst = max(worst, moved / z)
     assert worst <= 2.4e-4
-
-
-# ---- exp2 on the FMA pipe (exp2_fma2 in csrc/tc_common.cuh) ------------------
-
-def _exp2_coefficients():
-    import os
-    import re
-    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                            "kv_cache_eviction_scores_b200", "csrc", "tc_common.cuh")).read()
-    return [np.float32(float(re.search(rf"kE2c{i} = ([0-9.e+-]+)f", src).group(1)))
-            for i in range(6)]
-
-
-def _fma32(a, b, c):  # fp32 fused multiply-add: exact product, the sum rounded once
-    with np.errstate(invalid="ignore"):  # -inf inputs give NaN here; the kernel selects 0
-        return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(np.float32)
-
-
-def exp2_fma2_emulated(y):
-    """The kernel's steps in fp32: rounding by adding 1.5 * 2^23, the exact
-    remainder, Horner's rule, and the integer add into the exponent field."""
-    y = np.asarray(y, dtype=np.float32)
-    magic = np.float32(12582912.0)
-    t = (y + magic).astype(np.float32)
-    n = (t - magic).astype(np.float32)
-    f = _fma32(n, np.float32(-1.0), y)
-    c = _exp2_coefficients()
-    q = np.full_like(f, c[5])
-    for k in range(4, -1, -1):
-        q = _fma32(f, q, np.full_like(f, c[k]))
-    bits = (q.view(np.uint32).astype(np.uint64) + (t.view(np.uint32).astype(np.uint64) << 23)) & 0xFFFFFFFF
-    out = bits.astype(np.uint32).view(np.float32)
-    return np.where(y < -125.0, np.float32(0.0), out)
-
-
-def test_exp2_on_the_fma_pipe_meets_its_error_bound():
-    # relative error within 3e-7 over the range the kernels use (y <= 8 in
-    # pass 1, y <= 0 in the second pass), the same order as the SFU's ex2
-    y = np.concatenate([np.linspace(-125.0, 8.0, 2_000_001), np.arange(-125, 9) + 0.0,
-                        np.arange(-125, 8) + 0.5]).astype(np.float32)
-    got = exp2_fma2_emulated(y).astype(np.float64)
-    ref = np.exp2(y.astype(np.float64))
-    rel = np.abs(got - ref) / ref
-    assert rel.max() <= 3e-7, rel.max()
-    # below -125 (and -inf, a masked logit) it is exactly 0
-    tiny = exp2_fma2_emulated(np.array([-125.5, -126.0, -200.0, -1e30, -np.inf], dtype=np.float32))
-    assert np.all(tiny == 0.0)
