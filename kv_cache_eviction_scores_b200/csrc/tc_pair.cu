@@ -75,10 +75,11 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int L = a.L[b];
   const int z = b * a.Hkv + h;
   const int qrow0 = z * a.nq + chunk * nqc;           // the chunk's first query row
-  // barriers (the leader's copies gather both CTAs): BQ, FULL[r] -- arrivals
-  // of both producers; TF[2] -- the 32 score warps of the pair hand a TMEM
-  // buffer back; EMPTY[r], MD[2] -- the leader's commits, multicast to both
-  // CTAs; FIN -- the leader's MMAs are all done
+  // barriers (the leader's copies gather both CTAs): BQ -- both producers
+  // announce their query-side bytes; FULL[r] -- the leader announces both
+  // CTAs' tile bytes and both CTAs' TMA loads complete on it; TF[2] -- the 32
+  // score warps of the pair hand a TMEM buffer back; EMPTY[r], MD[2] -- the
+  // leader's commits, multicast to both CTAs; FIN -- the leader's MMAs are done
   const uint32_t BQ = smem_u32(&bars[0]);
   auto MD = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto TF = [&](int s) { return smem_u32(&bars[3 + s]); };
@@ -91,7 +92,7 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_init(MD(s), 1); mbar_init(TF(s), 2 * kSimtWarps);
     }
     for (int r = 0; r < kRingP; ++r) {
-      mbar_init(FULL(r), 2); mbar_init(EMPTY(r), 1);
+      mbar_init(FULL(r), 1); mbar_init(EMPTY(r), 1);
     }
     mbar_init(FIN, 1);
     *abort_flag = aligned ? 0 : 1;
@@ -156,21 +157,23 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tma_load_2d_pair(smem_u32(sAl) + rows * 128 + so, &tmAlo, cBQ, 64, grow);
         }
       }
-      // K_i at load 2i, V_i at 2i + 1; a step past this CTA's tiles only arrives
+      // K_i at load 2i, V_i at 2i + 1; the leader announces the bytes of both
+      // CTAs' loads of the slot (none for a step past a CTA's tiles)
       for (int i = 0; i < 2 * steps && !*abort_flag; ++i) {
         const int r = i % kRingP, ph = (i / kRingP) & 1;
         if (!mbar_wait(EMPTY(r), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
         const uint32_t cF = mapa_u32(FULL(r), 0);
         const int st = i >> 1;
+        if (leader) {
+          const int peer_n = T - steps;
+          mbar_expect_tx(FULL(r), (uint32_t)kTileBytes * ((st < my_n ? 1u : 0u) + (st < peer_n ? 1u : 0u)));
+        }
         if (st < my_n) {
-          mbar_expect_tx_cluster(cF, kTileBytes);
           const uint32_t dst = smem_u32(sRing + r * kTileBytes);
           const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
           const int row = tile_at(st) * kTok;
           tma_load_3d_pair(dst, m, cF, 0, row, z);
           tma_load_3d_pair(dst + kBox, m, cF, 64, row, z);
-        } else {
-          mbar_arrive_cluster(cF);
         }
       }
     }
@@ -189,8 +192,8 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int rk = (2 * i) % kRingP, pk = ((2 * i) / kRingP) & 1;
         const int rv = (2 * i + 1) % kRingP, pv = ((2 * i + 1) / kRingP) & 1;
         // both CTAs' K and V tiles of this step
-        if (!__all_sync(0xffffffffu, mbar_wait_cluster(FULL(rk), pk, kWaitNs)) ||
-            !__all_sync(0xffffffffu, mbar_wait_cluster(FULL(rv), pv, kWaitNs))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(FULL(rk), pk, kWaitNs)) ||
+            !__all_sync(0xffffffffu, mbar_wait(FULL(rv), pv, kWaitNs))) {
           ok = false;
           break;
         }
@@ -198,7 +201,7 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const int s = k & 1;
           // the buffer's previous item has been read by all 32 score warps
           if (k >= 2 &&
-              !__all_sync(0xffffffffu, mbar_wait_cluster(TF(s), (uint32_t)(((k >> 1) - 1) & 1),
+              !__all_sync(0xffffffffu, mbar_wait(TF(s), (uint32_t)(((k >> 1) - 1) & 1),
                                                          kWaitNs))) {
             ok = false;
             break;
@@ -273,7 +276,7 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float acc = 0.f;
       for (int hh = 0; hh < nh; ++hh, ++k) {
         const int s = k & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait_cluster(MD(s), (uint32_t)((k >> 1) & 1), kWaitNs))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(MD(s), (uint32_t)((k >> 1) & 1), kWaitNs))) {
           fail(a, abort_flag);
           live = false;
           break;
@@ -286,7 +289,7 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         auto release = [&]() {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(s ? cTF1 : cTF0);
+          if (lane == 0) mbar_arrive_remote(s ? cTF1 : cTF0);
         };
         // score of 16 columns (chunk ch of the half) from S^T in r[0..15] and D
         // in r[16..31]
