@@ -136,8 +136,8 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   auto VE = [&](int s) { return smem_u32(&bars[1 + 2 * kStK + kSt1 + s]); };
   constexpr int kB0 = 1 + 2 * kStK + 2 * kSt1;
   auto SF = [&](int t) { return smem_u32(&bars[kB0 + t]); };
-  auto PD = [&](int t) { return smem_u32(&bars[kB0 + 2 + t]); };
-  auto PF = [&](int t, int q) { return smem_u32(&bars[kB0 + 4 + t * kPQ + q]); };
+  auto PF = [&](int t) { return smem_u32(&bars[kB0 + 2 + t]); };
+  auto PD = [&](int t) { return smem_u32(&bars[kB0 + 4 + t]); };
   if (threadIdx.x == 0) {
     mbar_init(BQ, 1);
     for (int s = 0; s < kStK; ++s) {
@@ -148,8 +148,7 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       mbar_init(VE(s), 2);  // the last P V's commit + the ||v||^2 warp's reads
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(SF(t), 1); mbar_init(PD(t), 1);
-      for (int q = 0; q < kPQ; ++q) mbar_init(PF(t, q), 4);
+      mbar_init(SF(t), 1); mbar_init(PF(t), 4); mbar_init(PD(t), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -226,10 +225,9 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       __syncwarp();
       return true;
     };
-    // O_t += P_t V_i, each 32-token part of P as soon as the softmax warps have
-    // written it, so the first parts' MMAs overlap the rest of the softmax
     auto issue_PV = [&](int t, int i) {
       const int s = i % kSt1, ph = (i / kSt1) & 1;
+      if (!warp_wait(PF(t), (uint32_t)(i & 1))) { fail(a, abort_flag); return false; }
       if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
       uint8_t* vb = sV + s * kTileBytes;
       const int tile0 = (t0 + i) * kTok;
@@ -245,27 +243,22 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         fence_proxy_async_smem();
       }
       __syncwarp();
-      const uint32_t vlo = vd0.lo + (uint32_t)s * (kTileBytes >> 4);
-      const uint32_t dO = tbase + kColO1 + (uint32_t)(128 * t);
-      const uint32_t pS = tbase + (uint32_t)(128 * t);
-      for (int q = 0; q < kPQ; ++q) {
-        if (!warp_wait(PF(t, q), (uint32_t)(i & 1))) { fail(a, abort_flag); return false; }
-        tc_fence_after();
-        if (lane == 0) {
-          // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in
-          // [16kk+8, 16kk+16); V slice kk starts 16 rows (2048 bytes) further
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t vlo = vd0.lo + (uint32_t)s * (kTileBytes >> 4);
+        const uint32_t dO = tbase + kColO1 + (uint32_t)(128 * t);
+        const uint32_t pS = tbase + (uint32_t)(128 * t);
+        // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16);
+        // V slice kk starts 16 rows (2048 bytes) further
 #pragma unroll
-          for (int kk = 2 * q; kk < 2 * q + 2; ++kk) {
-            mma_ts_w(dO, pS + (uint32_t)(16 * kk), vlo + (uint32_t)kk * 128u, vd0.hi, IDP,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-            mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
-          }
-          if (q == kPQ - 1) {
-            mma_commit(PD(t));
-            if (t == nt - 1) mma_commit(VE(s));  // the last reader of this V stage
-          }
-        }
-        __syncwarp();
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts_w(dO, pS + (uint32_t)(16 * kk), vlo + (uint32_t)kk * 128u, vd0.hi, IDP,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
+        mma_commit(PD(t));
+        if (t == nt - 1) mma_commit(VE(s));  // the last reader of this V stage
       }
       __syncwarp();
       return true;
@@ -376,15 +369,11 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
       const uint64_t nmu2 = pk2(-mu, -mu);
 #pragma unroll
-      for (int q = 0; q < kPQ; ++q) {  // 32 tokens per part, handed to P V at once
-#pragma unroll
-        for (int cc = 2 * q; cc < 2 * q + 2; ++cc)
-          l += p1_exp16(sr + 16 * cc, tS + 16u * cc, c2, nmu2);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(PF(t, q));
-      }
+      for (int cc = 0; cc < 8; ++cc) l += p1_exp16(sr + 16 * cc, tS + 16u * cc, c2, nmu2);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(PF(t));
     }
     // partial row: O, the reference max, the normaliser
     if (t < nt) {
