@@ -12,24 +12,25 @@
 // The histogram rounds take a range in sub-ranges of 16384 keys, 32
 // consecutive keys per thread (one sub-range when it fits the shared-memory
 // cache, which then holds it for every phase).
-//   rounds 0..2: every CTA histograms an 11/11/10-bit digit of its keys that
-//       match the prefix found so far and adds the histogram into rank 0's
-//       shared memory (distributed shared memory atomics; one histogram per
-//       round, all zeroed at the start) and arrives on rank 0's gather
-//       barrier; rank 0 finds the digit holding the E-th smallest key,
-//       stores (prefix, rank) into every CTA and arrives on every CTA's
-//       broadcast barrier.
-//       After round 2 the prefix is the threshold key T and `rem` is how many
-//       keys equal to T are evicted (the lowest positions among them).
-//   count: each warp walks a contiguous part of the CTA's range, 32
-//       consecutive keys at a time (lane = key), and counts the keys < T and
-//       == T with ballots; every CTA stores its totals into every CTA, which
-//       then sums the counts of the lower ranks (the ranges are in position
-//       order).
-//   write: the same walk again: the ballots give every lane its evicted rank
-//       and an == T key's rank among the == T keys, and each lane writes its
-//       position straight to its slot of the keep or evict list.
-// The phases are separated by cluster-wide mbarrier phases with bounded waits;
+//   rounds 0, 1: every CTA histograms an 11-bit digit of its keys that match
+//       the prefix found so far and adds its non-zero bins into the round's
+//       histogram of every CTA of the cluster (distributed shared memory
+//       atomics; all histograms zeroed at the start); after one cluster-wide
+//       phase every CTA finds the digit holding the E-th smallest key itself,
+//       and counts its own keys below that digit.
+//   round 2: the same for the last 10 bits, except that every CTA stores its
+//       histogram into its own slot of every CTA, together with its counts
+//       below the round-0 and round-1 digits.  After the phase the prefix is
+//       the threshold key T, `rem` is how many keys equal to T are evicted
+//       (the lowest positions among them), and every CTA knows how many keys
+//       below / at T every lower rank holds, without another pass.
+//   write: each warp walks a contiguous part of the CTA's range, 32
+//       consecutive keys at a time (lane = key), counting the keys < T and
+//       == T with ballots; a block scan orders the warps; the same walk again
+//       gives every lane its evicted rank and an == T key's rank among the
+//       == T keys, and each lane writes its position straight to its slot of
+//       the keep or evict list.
+// The rounds are separated by cluster-wide mbarrier phases with bounded waits;
 // a wait that gives up records DROPKV_ERR_TIMEOUT in the status word and the
 // CTA keeps taking the remaining phase barriers (without the work).  The kernel
 // ends on the hardware cluster barrier, so no CTA leaves while another may
@@ -46,7 +47,8 @@ namespace {
 constexpr int kC = 8;                // CTAs per cluster: one cluster per segment
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;
+constexpr int kBins = 2048;          // rounds 0, 1: 11-bit digits
+constexpr int kBins2 = 1024;         // round 2: the last 10 bits
 constexpr int kPer = 32;             // consecutive keys per thread in one sub-range
 constexpr int kSub = kThreads * kPer;  // keys per sub-range (16384)
 constexpr int kCopies = 4;           // histogram copies (warp % 4), padded apart by one bank
@@ -60,8 +62,8 @@ struct SelParams {
   int32_t E[kMaxB];                  // evictions per row
   int32_t* status;                   // device status word (0 = OK), or NULL: not reported
   int32_t cache;                     // 1: every CTA's range fits one cached sub-range
-  int32_t stall_rank;                // self-test only: this rank withholds its first
-                                     // gather arrival (-1: none, the product path)
+  int32_t stall_rank;                // self-test only: this rank withholds its arrivals
+                                     // of round 0 (-1: none, the product path)
   uint64_t wait_ns;                  // limit of every bounded wait
 };
 
@@ -121,47 +123,19 @@ __device__ __forceinline__ int block_excl_scan(int v, int& total, int* warp_tot)
   return before + x - v;
 }
 
-// Thread 0 only: arrive (release, cluster scope) on the mbarrier at shared
-// address `bar` of CTA `rank`.
-__device__ __forceinline__ void arrive_at(uint32_t bar, uint32_t rank) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(bar, rank))
-               : "memory");
-}
-// Thread 0 only: bounded wait (acquire, cluster scope) for the phase of
-// parity `parity` of this CTA's mbarrier `bar`.  On expiry records the timeout.
-__device__ bool wait_at(uint32_t bar, uint32_t parity, volatile int* fail, int32_t* status,
-                        uint64_t limit_ns) {
-  const uint64_t t0 = gtimer();
-  for (;;) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if (gtimer() - t0 > limit_ns) {
-      *fail = 1;
-      if (status) atomicMax(status, (int)DROPKV_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-
 // One cluster-wide phase: after a block barrier (which orders every thread's
 // prior shared / distributed shared memory writes before thread 0), thread 0
 // fences at cluster scope and arrives on the phase barrier of every CTA of the
 // cluster, then waits (bounded, acquire at cluster scope) for all kC arrivals
 // on its own; a second block barrier releases the other threads.  Returns
-// false once any wait of this CTA has given up.
+// false once any wait of this CTA has given up.  `withhold` (self-test only)
+// skips the arrivals.
 __device__ bool cluster_phase(uint32_t bar, int& phase, volatile int* fail, int32_t* status,
-                              uint64_t limit_ns) {
+                              uint64_t limit_ns, bool withhold = false) {
   __syncthreads();
   if (threadIdx.x == 0) {
     asm volatile("fence.acq_rel.cluster;" ::: "memory");
-    for (uint32_t r = 0; r < (uint32_t)kC; ++r)
+    for (uint32_t r = 0; r < (uint32_t)kC && !withhold; ++r)
       asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mapa(bar, r))
                    : "memory");
     const uint32_t parity = (uint32_t)(phase & 1);
@@ -194,17 +168,19 @@ template <bool kCached>
 __global__ void __cluster_dims__(kC, 1, 1) __launch_bounds__(kThreads, 1)
 k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ keep_idx,
          int32_t* __restrict__ evict_idx) {
-  extern __shared__ uint32_t smem_dyn[];     // [kSub] key cache, then histogram copies
-  uint32_t* cached_keys = smem_dyn;          // this CTA's range when it fits one sub-range
-  uint32_t* loc = smem_dyn + kSub;           // [kCopies][kCopyStride] this CTA's histograms
-  __shared__ uint32_t H[3][kBins];           // the cluster histogram of each round (rank 0's)
+  extern __shared__ uint32_t smem_dyn[];     // key cache, histogram copies, round-2 slots
+  uint32_t* cached_keys = smem_dyn;          // [kSub] this CTA's range when it fits one sub-range
+  uint32_t* loc = smem_dyn + kSub;           // [kCopies][kCopyStride] this CTA's histograms;
+                                             // copy 0 then holds this CTA's round totals
+  uint32_t* H2 = loc + kCopies * kCopyStride;  // [kC][kBins2] every rank's round-2 histogram
+  __shared__ uint32_t H[2][kBins];           // the cluster histograms of rounds 0 and 1
+  __shared__ uint32_t bel[kC][2];            // per rank: its keys below the round-0 / -1 digits
+  __shared__ uint32_t below[2];              // this CTA's counts below the round-0 / -1 digits
+  __shared__ uint32_t cross[2];              // keys < T / == T held by the lower ranks
   __shared__ int32_t warp_tot[kWarps];
-  __shared__ uint32_t cnt[kC][2];            // per-rank (#< T, #== T), stored by every rank
-  __shared__ uint32_t ctl[2];                // this CTA's (prefix, rem) after a round
+  __shared__ uint32_t ctl[2];                // (prefix, rem) after a round
   __shared__ int32_t wsum[2][kWarps];
-  __shared__ __align__(8) uint64_t bar;     // all-to-all phases (count, final): kC arrivals
-  __shared__ __align__(8) uint64_t gbar;    // rank 0: a round's histogram adds landed (kC)
-  __shared__ __align__(8) uint64_t bbar;    // every CTA: rank 0 broadcast the round's digit (1)
+  __shared__ __align__(8) uint64_t bar;     // the rounds' all-to-all phases: kC arrivals
   __shared__ uint32_t fails[kC];             // per rank: 1 if a wait of that CTA gave up
   __shared__ int fail;
   pdl_wait();  // the scores may come from the previous kernel in the stream
@@ -217,30 +193,39 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   const int lo = (int)min((long long)L, (long long)rank * span_ll);
   const int hi = (int)min((long long)L, (long long)lo + span_ll);
   const float* s = scores + (size_t)seg * p.n_max;
-  const uint32_t barA = smem_addr(&bar), gbarA = smem_addr(&gbar), bbarA = smem_addr(&bbar);
+  const uint32_t barA = smem_addr(&bar);
 
   if (tid == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(barA), "r"(kC) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(gbarA), "r"(kC) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bbarA), "r"(1) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fail = 0;
     ctl[0] = 0;
     ctl[1] = (uint32_t)E;
   }
-  for (int i = tid; i < 3 * kBins; i += kThreads) (&H[0][0])[i] = 0;
-  if (tid < 2 * kC) cnt[tid >> 1][tid & 1] = 0;
+  for (int i = tid; i < 2 * kBins; i += kThreads) (&H[0][0])[i] = 0;
+  for (int i = tid; i < kC * kBins2; i += kThreads) H2[i] = 0;
+  if (tid < 2 * kC) bel[tid >> 1][tid & 1] = 0;
+  if (tid < 2) below[tid] = cross[tid] = 0;
   if (tid < kC) fails[tid] = 0;
   // cache layout: key r of the range at r ^ ((r >> 5) & 31), so that both the
   // coalesced fill (32 consecutive r per warp) and the per-thread runs (lane t
-  // reads r = 32 t + u) touch 32 distinct banks
+  // reads r = 32 t + u) touch 32 distinct banks; eight loads in flight per thread
   if (kCached)
-    for (int j = lo + tid; j < hi; j += kThreads) {
-      const int r = j - lo;
-      cached_keys[r ^ ((r >> 5) & 31)] = key_of(__ldg(s + j));
+    for (int j0 = lo + tid; j0 < hi; j0 += 8 * kThreads) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * kThreads;
+        v[u] = j < hi ? __ldg(s + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = j0 + u * kThreads - lo;
+        if (j0 + u * kThreads < hi) cached_keys[r ^ ((r >> 5) & 31)] = key_of(v[u]);
+      }
     }
   __syncthreads();
-  // every CTA's barrier and histogram are initialised before any remote access
+  // every CTA's barrier and histograms are initialised before any remote access
   // (the one hardware cluster barrier; all threads of all CTAs reach it)
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
                    "memory");
@@ -256,7 +241,6 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
 #pragma unroll
     for (int u = 0; u < kPer; ++u) k[u] = (j0 + u < hi) ? key_at(j0 + u) : 0xFFFFFFFFu;
   };
-  const uint32_t H0 = mapa(smem_addr(&H[0][0]), 0);
   int phase = 0;
   bool ok = true;
   uint32_t prefix = 0, rem = (uint32_t)E;
@@ -266,7 +250,8 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
     for (int round = 0; round < 3; ++round) {
       const int shift = (round == 0) ? 21 : (round == 1) ? 10 : 0;
       const int width = (round == 2) ? 10 : 11;
-      const uint32_t mask = (1u << width) - 1u;
+      const int nb = 1 << width;
+      const uint32_t mask = (uint32_t)nb - 1u;
       if (ok) {
         for (int i = tid; i < kCopies * kCopyStride; i += kThreads) loc[i] = 0;
         __syncthreads();
@@ -283,70 +268,92 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
               atomicAdd(&myloc[(k[u] >> shift) & mask], 1u);
         }
         __syncthreads();
-        for (int i = tid; i < kBins; i += kThreads) {
+        // this CTA's totals (kept in copy 0) go into every CTA: added into the
+        // round's cluster histogram, or (round 2) stored into this rank's slot
+        const uint32_t dst0 =
+            round < 2 ? smem_addr(&H[round][0]) : smem_addr(H2 + rank * kBins2);
+        for (int i = tid; i < nb; i += kThreads) {
           uint32_t v = 0;
 #pragma unroll
           for (int c = 0; c < kCopies; ++c) v += loc[c * kCopyStride + i];
-          if (v) dsm_add(H0 + 4u * (uint32_t)(round * kBins + i), v);
-        }
-      }
-      // gather: every CTA's adds have landed at rank 0
-      __syncthreads();
-      if (tid == 0) {
-        asm volatile("fence.acq_rel.cluster;" ::: "memory");
-        if (!(round == 0 && (int)rank == p.stall_rank)) arrive_at(gbarA, 0);
-      }
-      if (rank == 0) {
-        if (tid == 0) wait_at(gbarA, (uint32_t)(round & 1), &fail, p.status, p.wait_ns);
-        __syncthreads();
-        if (fail == 0) {
-          // the digit holding rank `rem` (1-based) of the keys with this prefix
-          constexpr int per = kBins / kThreads;  // 4 bins per thread
-          uint32_t v[per], tot = 0;
-#pragma unroll
-          for (int i = 0; i < per; ++i) {
-            v[i] = H[round][tid * per + i];
-            tot += v[i];
-          }
-          int total;
-          uint32_t before = (uint32_t)block_excl_scan((int)tot, total, warp_tot);
-          if (before < rem && rem <= before + tot) {
-            for (int i = 0; i < per; ++i) {
-              if (before + v[i] >= rem) {
-                const uint32_t digit = (uint32_t)(tid * per + i);
-                ctl[0] = (round == 0) ? digit : ((prefix << width) | digit);
-                ctl[1] = rem - before;
-                break;
-              }
-              before += v[i];
+          loc[i] = v;
+          if (v) {
+            for (uint32_t d = 0; d < (uint32_t)kC; ++d) {
+              const uint32_t ra = mapa(dst0 + 4u * (uint32_t)i, d);
+              if (round < 2) dsm_add(ra, v);
+              else dsm_st(ra, v);
             }
           }
-          __syncthreads();
-          if (tid < kC) {  // broadcast (prefix, rem) into every CTA
-            const uint32_t dst = mapa(smem_addr(ctl), (uint32_t)tid);
-            dsm_st(dst, ctl[0]);
-            dsm_st(dst + 4u, ctl[1]);
+        }
+        if (round == 2 && tid < kC) {  // and the counts below the earlier digits
+          const uint32_t ra = mapa(smem_addr(&bel[rank][0]), (uint32_t)tid);
+          dsm_st(ra, below[0]);
+          dsm_st(ra + 4u, below[1]);
+        }
+      }
+      ok = cluster_phase(barA, phase, &fail, p.status, p.wait_ns,
+                         round == 0 && (int)rank == p.stall_rank) && ok;
+      if (ok) {
+        // the digit holding rank `rem` (1-based) of the keys with this prefix,
+        // found by every CTA from the same histogram
+        const int per = nb / kThreads;  // 4 or 2 bins per thread
+        uint32_t v[kBins / kThreads], tot = 0;
+#pragma unroll
+        for (int i = 0; i < kBins / kThreads; ++i) {
+          v[i] = 0;
+          if (i < per) {
+            const int bin = tid * per + i;
+            if (round < 2) {
+              v[i] = H[round][bin];
+            } else {
+#pragma unroll
+              for (int r = 0; r < kC; ++r) v[i] += H2[r * kBins2 + bin];
+            }
+          }
+          tot += v[i];
+        }
+        int total;
+        uint32_t before = (uint32_t)block_excl_scan((int)tot, total, warp_tot);
+        if (before < rem && rem <= before + tot) {
+          for (int i = 0; i < per; ++i) {
+            if (before + v[i] >= rem) {
+              const uint32_t digit = (uint32_t)(tid * per + i);
+              ctl[0] = (round == 0) ? digit : ((prefix << width) | digit);
+              ctl[1] = rem - before;
+              break;
+            }
+            before += v[i];
           }
         }
         __syncthreads();
-        if (tid == 0) {
-          asm volatile("fence.acq_rel.cluster;" ::: "memory");
-          for (uint32_t r = 0; r < (uint32_t)kC; ++r) arrive_at(bbarA, r);
+        prefix = ctl[0];
+        rem = ctl[1];
+        const int digit = (int)(prefix & mask);
+        if (round < 2) {
+          // this CTA's keys below the digit (those with the prefix, for round 1)
+          uint32_t part = 0;
+          for (int i = tid; i < digit; i += kThreads) part += loc[i];
+          if (part) atomicAdd(&below[round], part);
+        } else {
+          // keys below / at T held by the lower ranks
+          uint32_t lt = 0;
+          for (int i = tid; i < digit; i += kThreads)
+            for (uint32_t r = 0; r < rank; ++r) lt += H2[r * kBins2 + i];
+          if (tid == 0)
+            for (uint32_t r = 0; r < rank; ++r) {
+              lt += bel[r][0] + bel[r][1];
+              atomicAdd(&cross[1], H2[r * kBins2 + digit]);
+            }
+          if (lt) atomicAdd(&cross[0], lt);
         }
+        __syncthreads();  // ctl and copy 0 are read before the next round rewrites them
       }
-      // broadcast: the round's (prefix, rem) is in this CTA's ctl
-      if (tid == 0) wait_at(bbarA, (uint32_t)(round & 1), &fail, p.status, p.wait_ns);
-      __syncthreads();
-      ok = fail == 0;
-      prefix = ctl[0];
-      rem = ctl[1];
-      __syncthreads();  // ctl is read by every thread before the next round's broadcast
     }
   }
   const uint32_t T = prefix;
   const int quota = E > 0 ? (int)rem : 0;  // keys == T that are evicted
 
-  // ---- counts below / at the threshold, gathered at every CTA --------------
+  // ---- counts below / at the threshold per warp -----------------------------
   // Each warp takes a contiguous, 32-aligned part of the CTA's range and walks
   // it 32 consecutive keys at a time (lane = key); ballots count the keys
   // below / at T.  The same walk writes the lists below.
@@ -367,21 +374,10 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
     wsum[1][wid] = neq;
   }
   __syncthreads();
-  if (tid < kC && ok) {  // this rank's counts into every CTA of the cluster
-    int a = 0, e = 0;
-    for (int i = 0; i < kWarps; ++i) {
-      a += wsum[0][i];
-      e += wsum[1][i];
-    }
-    const uint32_t dst = mapa(smem_addr(&cnt[rank][0]), (uint32_t)tid);
-    dsm_st(dst, (uint32_t)a);
-    dsm_st(dst + 4u, (uint32_t)e);
-  }
-  ok = cluster_phase(barA, phase, &fail, p.status, p.wait_ns) && ok;
 
   // ---- order-preserving compaction of this CTA's range ----------------------
   // Per warp, in position order: the keys below / at T before its part (lower
-  // ranks, then lower warps of this CTA), then per 32 keys the ballots give
+  // ranks, from the round-2 phase, then lower warps of this CTA), then per 32 keys the ballots give
   // every lane its evicted rank (those before it) and an == T key's rank among
   // the == T keys (evicted while below the quota); a kept key's rank is its
   // position minus the evicted keys before it.  Lanes write their positions
@@ -389,11 +385,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   if (ok) {
     int32_t* kout = keep_idx + (size_t)seg * p.max_keep;
     int32_t* eout = evict_idx + (size_t)seg * p.max_evict;
-    int lt_run = 0, eq_run = 0;
-    for (uint32_t r = 0; r < rank; ++r) {  // the lower ranks hold the lower positions
-      lt_run += (int)cnt[r][0];
-      eq_run += (int)cnt[r][1];
-    }
+    int lt_run = (int)cross[0], eq_run = (int)cross[1];  // the lower ranks hold the lower positions
     for (int i = 0; i < wid; ++i) {
       lt_run += wsum[0][i];
       eq_run += wsum[1][i];
@@ -488,9 +480,10 @@ cudaError_t launch_impl(int B, int Hkv, int n_max, const float* scores, const in
   for (int b = 0; b < B; ++b) max_L = L[b] > max_L ? L[b] : max_L;
   const long long span = (((long long)max_L + kC - 1) / kC + 31) & ~31ll;
   p.cache = span <= kSub ? 1 : 0;
-  // [key cache when it fits][histogram copies]; the histogram copies always
-  // start at kSub words
-  const size_t smem = ((size_t)kSub + kCopies * (size_t)kCopyStride) * sizeof(uint32_t);
+  // [key cache when it fits][histogram copies][round-2 slots]; the histogram
+  // copies always start at kSub words
+  const size_t smem =
+      ((size_t)kSub + kCopies * (size_t)kCopyStride + (size_t)kC * kBins2) * sizeof(uint32_t);
   auto kern = p.cache ? k_select<true> : k_select<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -508,8 +501,8 @@ cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const 
                      status, -1, kWaitNs, st);
 }
 
-// Self-test: CTA rank 1 of every cluster withholds its first gather arrival,
-// so rank 0's wait for it runs out after wait_ns (and later waits of the
+// Self-test: CTA rank 1 of every cluster withholds its arrivals of round 0, so
+// every CTA's wait for them runs out after wait_ns (and later waits of the
 // segment may too); the kernel then reports the timeout and fills -1.
 cudaError_t launch_select_stalled(int B, int Hkv, int n_max, const float* scores,
                                   const int32_t* L, const int32_t* keep, int32_t* keep_idx,

@@ -430,9 +430,16 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
   const int cta0 = a.cta_base1[b] + (h * a.chunks1 + chunk) * a.splits1[b];
   const int np = a.splits1[b];
   auto P = [&](int i) { return a.partial + ((size_t)(cta0 + i) * a.rows1 + rr) * kPartStride; };
-  // lanes take the partials' (max, normaliser) pairs in parallel, 32 at a
-  // time: M, then the weights 2^(m_i - M) and L = sum_i w_i l_i; the weights
-  // of the first 32 partials stay in the lanes that loaded them
+  // The first kFly partial rows of O are requested before anything else, so
+  // that they travel with the (max, normaliser) pairs: one round trip for up
+  // to kFly partials.  Lanes take the pairs in parallel, 32 at a time: M,
+  // then the weights 2^(m_i - M) and L = sum_i w_i l_i; the weights of the
+  // first 32 partials stay in the lanes that loaded them.
+  constexpr int kFly = 24;
+  float4 o[kFly];
+#pragma unroll
+  for (int k = 0; k < kFly; ++k)
+    if (k < np) o[k] = *reinterpret_cast<const float4*>(P(k) + lane * 4);
   float M = -INFINITY, m_own = -INFINITY, l_own = 0.f;
   for (int i = lane; i < np; i += 32) {
     const float2 ml = *reinterpret_cast<const float2*>(P(i) + 128);
@@ -447,13 +454,22 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
     lpart = fmaf((ml.x == -INFINITY) ? 0.f : ex2(ml.x - M), ml.y, lpart);
   }
   const float Lsum = warp_sum(lpart);
-  // O = sum_i w_i O_i, eight partial rows in flight per step
+  // O = sum_i w_i O_i: the rows in flight, then the rest eight at a time
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < np; i0 += 8) {
-    float4 o[8];
+  auto add = [&](const float4& v, float wg) {
+    acc.x = fmaf(wg, v.x, acc.x);
+    acc.y = fmaf(wg, v.y, acc.y);
+    acc.z = fmaf(wg, v.z, acc.z);
+    acc.w = fmaf(wg, v.w, acc.w);
+  };
+#pragma unroll
+  for (int k = 0; k < kFly; ++k)
+    if (k < np) add(o[k], __shfl_sync(0xffffffffu, w_own, k));
+  for (int i0 = kFly; i0 < np; i0 += 8) {
+    float4 r[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      o[k] = *reinterpret_cast<const float4*>(P(min(i0 + k, np - 1)) + lane * 4);
+      r[k] = *reinterpret_cast<const float4*>(P(min(i0 + k, np - 1)) + lane * 4);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int i = i0 + k;
@@ -463,10 +479,7 @@ __global__ void __launch_bounds__(128) k_tc_combine(const TcArgs a) {
         wg = (mi == -INFINITY) ? 0.f : ex2(mi - M);
       }
       if (i >= np) wg = 0.f;
-      acc.x = fmaf(wg, o[k].x, acc.x);
-      acc.y = fmaf(wg, o[k].y, acc.y);
-      acc.z = fmaf(wg, o[k].z, acc.z);
-      acc.w = fmaf(wg, o[k].w, acc.w);
+      add(r[k], wg);
     }
   }
   const float inv = 1.f / Lsum;
