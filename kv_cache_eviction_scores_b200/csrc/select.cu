@@ -183,7 +183,6 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   __shared__ __align__(8) uint64_t bar;     // the rounds' all-to-all phases: kC arrivals
   __shared__ uint32_t fails[kC];             // per rank: 1 if a wait of that CTA gave up
   __shared__ int fail;
-  pdl_wait();  // the scores may come from the previous kernel in the stream
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const uint32_t rank = cluster_rank();
   const int seg = blockIdx.x / kC;
@@ -207,23 +206,39 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   if (tid < 2 * kC) bel[tid >> 1][tid & 1] = 0;
   if (tid < 2) below[tid] = cross[tid] = 0;
   if (tid < kC) fails[tid] = 0;
+  // the set-up above overlaps the previous kernel's tail; the scores may come
+  // from that kernel
+  pdl_wait();
   // cache layout: key r of the range at r ^ ((r >> 5) & 31), so that both the
-  // coalesced fill (32 consecutive r per warp) and the per-thread runs (lane t
-  // reads r = 32 t + u) touch 32 distinct banks; eight loads in flight per thread
-  if (kCached)
-    for (int j0 = lo + tid; j0 < hi; j0 += 8 * kThreads) {
-      float v[8];
+  // coalesced fill (consecutive r across a warp) and the per-thread runs (lane
+  // t reads r = 32 t + u) touch 32 distinct banks.  16-byte loads, four in
+  // flight per thread, when the range starts 16-byte aligned.
+  if (kCached) {
+    const int n = hi - lo;
+    auto put = [&](int r, float v) { cached_keys[r ^ ((r >> 5) & 31)] = key_of(v); };
+    int done = 0;
+    if ((reinterpret_cast<uintptr_t>(s + lo) & 15u) == 0) {
+      const int n4 = n >> 2;
+      const float4* s4 = reinterpret_cast<const float4*>(s + lo);
+      for (int q0 = tid; q0 < n4; q0 += 4 * kThreads) {
+        float4 v[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u * kThreads;
-        v[u] = j < hi ? __ldg(s + j) : 0.f;
-      }
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + u * kThreads;
+          v[u] = q < n4 ? __ldg(s4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int r = j0 + u * kThreads - lo;
-        if (j0 + u * kThreads < hi) cached_keys[r ^ ((r >> 5) & 31)] = key_of(v[u]);
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + u * kThreads;
+          if (q < n4) {
+            put(4 * q, v[u].x); put(4 * q + 1, v[u].y); put(4 * q + 2, v[u].z); put(4 * q + 3, v[u].w);
+          }
+        }
       }
+      done = 4 * n4;
     }
+    for (int r = done + tid; r < n; r += kThreads) put(r, __ldg(s + lo + r));
+  }
   __syncthreads();
   // every CTA's barrier and histograms are initialised before any remote access
   // (the one hardware cluster barrier; all threads of all CTAs reach it)
@@ -241,6 +256,9 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
 #pragma unroll
     for (int u = 0; u < kPer; ++u) k[u] = (j0 + u < hi) ? key_at(j0 + u) : 0xFFFFFFFFu;
   };
+  // kCached: this thread's run of the range, held in registers for every round
+  uint32_t kr[kPer];
+  if constexpr (kCached) load_run(lo, kr);
   int phase = 0;
   bool ok = true;
   uint32_t prefix = 0, rem = (uint32_t)E;
@@ -258,14 +276,20 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
         // scores concentrate in few bins: four copies (by warp), one bank apart,
         // spread the colliding atomics
         uint32_t* myloc = loc + (wid & (kCopies - 1)) * kCopyStride;
-        for (int sub0 = lo; sub0 < hi; sub0 += kSub) {
-          uint32_t k[kPer];
-          load_run(sub0, k);
-          const int j0 = sub0 + tid * kPer;
+        auto hist_run = [&](const uint32_t(&k)[kPer], int j0) {
 #pragma unroll
           for (int u = 0; u < kPer; ++u)
             if (j0 + u < hi && (round == 0 || (k[u] >> (shift + width)) == prefix))
               atomicAdd(&myloc[(k[u] >> shift) & mask], 1u);
+        };
+        if constexpr (kCached) {
+          hist_run(kr, lo + tid * kPer);
+        } else {
+          for (int sub0 = lo; sub0 < hi; sub0 += kSub) {
+            uint32_t k[kPer];
+            load_run(sub0, k);
+            hist_run(k, sub0 + tid * kPer);
+          }
         }
         __syncthreads();
         // this CTA's totals (kept in copy 0) go into every CTA: added into the
@@ -354,21 +378,36 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   const int quota = E > 0 ? (int)rem : 0;  // keys == T that are evicted
 
   // ---- counts below / at the threshold per warp -----------------------------
-  // Each warp takes a contiguous, 32-aligned part of the CTA's range and walks
-  // it 32 consecutive keys at a time (lane = key); ballots count the keys
-  // below / at T.  The same walk writes the lists below.
-  const int wlen = ((hi - lo + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  // Each warp takes a contiguous, 32-aligned part of the CTA's range: with the
+  // range cached, the 1024 keys its lanes hold in registers (counted there);
+  // otherwise an equal share, walked 32 consecutive keys at a time (lane =
+  // key) with ballots.  The compaction below walks the same parts.
+  const int wlen = kCached ? kPer * 32 : ((hi - lo + kWarps * 32 - 1) / (kWarps * 32)) * 32;
   const int w_lo = min(hi, lo + wid * wlen), w_hi = min(hi, w_lo + wlen);
   const uint32_t lanelt = (1u << lane) - 1u;
   int nlt = 0, neq = 0;
-  if (ok && E > 0)
-    for (int c0 = w_lo; c0 < w_hi; c0 += 32) {
-      const int j = c0 + lane;
-      const bool in = j < w_hi;
-      const uint32_t kk = in ? key_at(j) : 0xFFFFFFFFu;
-      nlt += __popc(__ballot_sync(0xffffffffu, in && kk < T));
-      neq += __popc(__ballot_sync(0xffffffffu, in && kk == T));
+  if (ok && E > 0) {
+    if constexpr (kCached) {
+      const int j0 = lo + tid * kPer;
+      uint32_t a = 0, e = 0;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u)
+        if (j0 + u < hi) {
+          a += kr[u] < T ? 1u : 0u;
+          e += kr[u] == T ? 1u : 0u;
+        }
+      nlt = (int)__reduce_add_sync(0xffffffffu, a);
+      neq = (int)__reduce_add_sync(0xffffffffu, e);
+    } else {
+      for (int c0 = w_lo; c0 < w_hi; c0 += 32) {
+        const int j = c0 + lane;
+        const bool in = j < w_hi;
+        const uint32_t kk = in ? key_at(j) : 0xFFFFFFFFu;
+        nlt += __popc(__ballot_sync(0xffffffffu, in && kk < T));
+        neq += __popc(__ballot_sync(0xffffffffu, in && kk == T));
+      }
     }
+  }
   if (lane == 0) {
     wsum[0][wid] = nlt;
     wsum[1][wid] = neq;
@@ -392,26 +431,41 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
     }
     int ev_run = lt_run + min(eq_run, quota);  // evicted before this warp's part
     const bool any = E > 0;
-    for (int c0 = w_lo; c0 < w_hi; c0 += 32) {
-      const int j = c0 + lane;
-      const bool in = j < w_hi;
-      const uint32_t kk = in ? key_at(j) : 0xFFFFFFFFu;
-      const bool eq = any && in && kk == T;
-      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-      const bool ev = (any && in && kk < T) || (eq && eq_run + __popc(eqm & lanelt) < quota);
-      const uint32_t evm = __ballot_sync(0xffffffffu, ev);
-      const int ev_before = ev_run + __popc(evm & lanelt);
-      if (in) {
-        // the guards only matter after a wait gave up (inconsistent counts)
-        if (ev) {
-          if (ev_before >= 0 && ev_before < p.max_evict) eout[ev_before] = j;
-        } else {
-          const int r = j - ev_before;
-          if (r >= 0 && r < p.max_keep) kout[r] = j;
-        }
+    for (int c0 = w_lo; c0 < w_hi; c0 += 4 * 32) {  // four groups of 32 keys per step
+      // the four groups' keys and their below / at-T ballots first (independent),
+      // then the running ranks group by group
+      uint32_t ltm[4], eqm[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int j = c0 + 32 * g + lane;
+        const bool in = any && j < w_hi;
+        const uint32_t kk = j < w_hi ? key_at(j) : 0xFFFFFFFFu;
+        ltm[g] = __ballot_sync(0xffffffffu, in && kk < T);
+        eqm[g] = __ballot_sync(0xffffffffu, in && kk == T);
       }
-      ev_run += __popc(evm);
-      eq_run += __popc(eqm);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int j = c0 + 32 * g + lane;
+        uint32_t evm = ltm[g];
+        if (eqm[g]) {  // keys == T: evicted while their rank among them is below the quota
+          const bool e =
+              ((eqm[g] >> lane) & 1u) && eq_run + __popc(eqm[g] & lanelt) < quota;
+          evm |= __ballot_sync(0xffffffffu, e);
+        }
+        const bool ev = (evm >> lane) & 1u;
+        const int ev_before = ev_run + __popc(evm & lanelt);
+        if (j < w_hi) {
+          // the guards only matter after a wait gave up (inconsistent counts)
+          if (ev) {
+            if (ev_before >= 0 && ev_before < p.max_evict) eout[ev_before] = j;
+          } else {
+            const int r = j - ev_before;
+            if (r >= 0 && r < p.max_keep) kout[r] = j;
+          }
+        }
+        ev_run += __popc(evm);
+        eq_run += __popc(eqm[g]);
+      }
     }
     // slots past this row's own counts (rows shorter than the maxima): -1
     if (rank == kC - 1) {
