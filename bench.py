@@ -51,10 +51,13 @@ KERNELS = {
     "tensor": ["k_tc_pass1", "k_tc_combine", "k_tc_pass2_pair", "k_epilogue"],
     "tensor_attention": ["k_tc_pass1", "k_tc_combine", "k_tc_pass2", "k_epilogue"],
 }
+# the sources a kernel's code comes from (its file and the device headers it includes)
+_TC_HDRS = ("tc_common.cuh", "tc_ptx.cuh", "common.cuh")
 KERNEL_SRC = {
-    "k_simt_pass1": "simt.cu", "k_simt_pass2": "simt.cu", "k_epilogue": "epilogue.cu",
-    "k_tc_pass1": "tc.cu", "k_tc_combine": "tc.cu", "k_tc_pass2": "tc.cu",
-    "k_tc_pass2_pair": "tc_pair.cu",
+    "k_simt_pass1": ("simt.cu", "common.cuh"), "k_simt_pass2": ("simt.cu", "common.cuh"),
+    "k_epilogue": ("epilogue.cu", "common.cuh"),
+    "k_tc_pass1": ("tc.cu",) + _TC_HDRS, "k_tc_combine": ("tc.cu",) + _TC_HDRS,
+    "k_tc_pass2": ("tc.cu",) + _TC_HDRS, "k_tc_pass2_pair": ("tc_pair.cu",) + _TC_HDRS,
 }
 
 
@@ -279,13 +282,17 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ ours ----
 
-def source_hash(fname):
-    """sha256 of a kernel source's code: line comments and blank lines removed,
-    so that a comment edit does not invalidate the stored DRAM traffic."""
-    with open(os.path.join(CSRC, fname), encoding="utf-8") as f:
-        lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in f)
-        code = "\n".join(ln for ln in lines if ln.strip())
-    return hashlib.sha256(code.encode()).hexdigest()
+def source_hash(fnames):
+    """sha256 of a kernel's source files, in order: line comments and blank
+    lines removed, so that a comment edit does not invalidate the stored DRAM
+    traffic."""
+    h = hashlib.sha256()
+    for fname in fnames:
+        with open(os.path.join(CSRC, fname), encoding="utf-8") as f:
+            lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in f)
+            code = "\n".join(ln for ln in lines if ln.strip())
+        h.update(fname.encode() + b"\n" + code.encode() + b"\n")
+    return h.hexdigest()
 
 
 def traffic_for(kernel):

@@ -261,7 +261,8 @@ DROPKV_API dropkv_status dropkv_selftest_wait_timeout(int32_t* status_dev, uint6
 
 /* Self-test of the select kernel's failure path: runs the select of
  * dropkv_select on the given arguments (B <= 64) with one CTA of every
- * segment's cluster withholding its first arrival and every bounded wait
+ * segment's cluster withholding its arrivals of the first radix round (so the
+ * other CTAs' waits for them run out) and every bounded wait
  * limited to limit_ns nanoseconds (0 < limit_ns <= 1e9).  Every segment with
  * at least one eviction then ends with DROPKV_ERR_TIMEOUT in *status_dev
  * (device int32, zeroed by the call) and all its keep and evict slots set to

@@ -24,12 +24,12 @@
 //       the threshold key T, `rem` is how many keys equal to T are evicted
 //       (the lowest positions among them), and every CTA knows how many keys
 //       below / at T every lower rank holds, without another pass.
-//   write: each warp walks a contiguous part of the CTA's range, 32
-//       consecutive keys at a time (lane = key), counting the keys < T and
-//       == T with ballots; a block scan orders the warps; the same walk again
-//       gives every lane its evicted rank and an == T key's rank among the
-//       == T keys, and each lane writes its position straight to its slot of
-//       the keep or evict list.
+//   write: each warp counts the keys < T and == T of its contiguous part of
+//       the CTA's range (from the registers when the range is cached); the
+//       lower warps' counts order the warps; the warp then walks its part 32
+//       consecutive keys at a time (lane = key): ballots give every lane its
+//       evicted rank and an == T key's rank among the == T keys, and each lane
+//       writes its position straight to its slot of the keep or evict list.
 // The rounds are separated by cluster-wide mbarrier phases with bounded waits;
 // a wait that gives up records DROPKV_ERR_TIMEOUT in the status word and the
 // CTA keeps taking the remaining phase barriers (without the work).  The kernel
@@ -206,13 +206,15 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
   if (tid < 2 * kC) bel[tid >> 1][tid & 1] = 0;
   if (tid < 2) below[tid] = cross[tid] = 0;
   if (tid < kC) fails[tid] = 0;
+  for (int i = tid; i < kCopies * kCopyStride; i += kThreads) loc[i] = 0;
   // the set-up above overlaps the previous kernel's tail; the scores may come
   // from that kernel
   pdl_wait();
   // cache layout: key r of the range at r ^ ((r >> 5) & 31), so that both the
   // coalesced fill (consecutive r across a warp) and the per-thread runs (lane
-  // t reads r = 32 t + u) touch 32 distinct banks.  16-byte loads, four in
-  // flight per thread, when the range starts 16-byte aligned.
+  // t reads r = 32 t + u) touch 32 distinct banks.  16-byte loads, eight in
+  // flight per thread (a whole 16384-key range at once), when the range starts
+  // 16-byte aligned.
   if (kCached) {
     const int n = hi - lo;
     auto put = [&](int r, float v) { cached_keys[r ^ ((r >> 5) & 31)] = key_of(v); };
@@ -220,15 +222,15 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
     if ((reinterpret_cast<uintptr_t>(s + lo) & 15u) == 0) {
       const int n4 = n >> 2;
       const float4* s4 = reinterpret_cast<const float4*>(s + lo);
-      for (int q0 = tid; q0 < n4; q0 += 4 * kThreads) {
-        float4 v[4];
+      for (int q0 = tid; q0 < n4; q0 += 8 * kThreads) {
+        float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int q = q0 + u * kThreads;
           v[u] = q < n4 ? __ldg(s4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
           const int q = q0 + u * kThreads;
           if (q < n4) {
             put(4 * q, v[u].x); put(4 * q + 1, v[u].y); put(4 * q + 2, v[u].z); put(4 * q + 3, v[u].w);
@@ -271,8 +273,7 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
       const int nb = 1 << width;
       const uint32_t mask = (uint32_t)nb - 1u;
       if (ok) {
-        for (int i = tid; i < kCopies * kCopyStride; i += kThreads) loc[i] = 0;
-        __syncthreads();
+        // (the copies are zero: cleared at the start and by each round's owners)
         // scores concentrate in few bins: four copies (by warp), one bank apart,
         // spread the colliding atomics
         uint32_t* myloc = loc + (wid & (kCopies - 1)) * kCopyStride;
@@ -297,9 +298,12 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
         const uint32_t dst0 =
             round < 2 ? smem_addr(&H[round][0]) : smem_addr(H2 + rank * kBins2);
         for (int i = tid; i < nb; i += kThreads) {
-          uint32_t v = 0;
+          uint32_t v = loc[i];
 #pragma unroll
-          for (int c = 0; c < kCopies; ++c) v += loc[c * kCopyStride + i];
+          for (int c = 1; c < kCopies; ++c) {
+            v += loc[c * kCopyStride + i];
+            loc[c * kCopyStride + i] = 0;  // ready for the next round
+          }
           loc[i] = v;
           if (v) {
             for (uint32_t d = 0; d < (uint32_t)kC; ++d) {
@@ -354,9 +358,13 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
         rem = ctl[1];
         const int digit = (int)(prefix & mask);
         if (round < 2) {
-          // this CTA's keys below the digit (those with the prefix, for round 1)
+          // this CTA's keys below the digit (those with the prefix, for round
+          // 1); each thread clears the totals it owns for the next round
           uint32_t part = 0;
-          for (int i = tid; i < digit; i += kThreads) part += loc[i];
+          for (int i = tid; i < nb; i += kThreads) {
+            if (i < digit) part += loc[i];
+            loc[i] = 0;
+          }
           if (part) atomicAdd(&below[round], part);
         } else {
           // keys below / at T held by the lower ranks
@@ -431,40 +439,74 @@ k_select(SelParams p, const float* __restrict__ scores, int32_t* __restrict__ ke
     }
     int ev_run = lt_run + min(eq_run, quota);  // evicted before this warp's part
     const bool any = E > 0;
-    for (int c0 = w_lo; c0 < w_hi; c0 += 4 * 32) {  // four groups of 32 keys per step
-      // the four groups' keys and their below / at-T ballots first (independent),
-      // then the running ranks group by group
-      uint32_t ltm[4], eqm[4];
+    if constexpr (kCached) {
+      // the warp's 32 groups: every ballot first (independent), then the
+      // running ranks group by group, one predicated store per lane
+      uint32_t ltm[32], eqm[32];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int j = c0 + 32 * g + lane;
+      for (int g = 0; g < 32; ++g) {
+        const int j = w_lo + 32 * g + lane;
         const bool in = any && j < w_hi;
         const uint32_t kk = j < w_hi ? key_at(j) : 0xFFFFFFFFu;
         ltm[g] = __ballot_sync(0xffffffffu, in && kk < T);
         eqm[g] = __ballot_sync(0xffffffffu, in && kk == T);
       }
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int j = c0 + 32 * g + lane;
+      for (int g = 0; g < 32; ++g) {
+        const int j = w_lo + 32 * g + lane;
         uint32_t evm = ltm[g];
-        if (eqm[g]) {  // keys == T: evicted while their rank among them is below the quota
-          const bool e =
-              ((eqm[g] >> lane) & 1u) && eq_run + __popc(eqm[g] & lanelt) < quota;
+        if (eqm[g]) {
+          const bool e = ((eqm[g] >> lane) & 1u) && eq_run + __popc(eqm[g] & lanelt) < quota;
           evm |= __ballot_sync(0xffffffffu, e);
         }
         const bool ev = (evm >> lane) & 1u;
         const int ev_before = ev_run + __popc(evm & lanelt);
-        if (j < w_hi) {
-          // the guards only matter after a wait gave up (inconsistent counts)
-          if (ev) {
-            if (ev_before >= 0 && ev_before < p.max_evict) eout[ev_before] = j;
-          } else {
-            const int r = j - ev_before;
-            if (r >= 0 && r < p.max_keep) kout[r] = j;
-          }
-        }
+        const int r = j - ev_before;
+        int32_t* dst = ev ? eout + ev_before : kout + r;
+        // the guards only matter after a wait gave up (inconsistent counts)
+        const bool okw =
+            ev ? (ev_before >= 0 && ev_before < p.max_evict) : (r >= 0 && r < p.max_keep);
+        if (j < w_hi && okw) *dst = j;
         ev_run += __popc(evm);
         eq_run += __popc(eqm[g]);
+      }
+    } else {
+      // uncached ranges: four groups of 32 keys per step
+      for (int c0 = w_lo; c0 < w_hi; c0 += 4 * 32) {
+        // the four groups' keys and their below / at-T ballots first (independent),
+        // then the running ranks group by group
+        uint32_t ltm[4], eqm[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int j = c0 + 32 * g + lane;
+          const bool in = any && j < w_hi;
+          const uint32_t kk = j < w_hi ? key_at(j) : 0xFFFFFFFFu;
+          ltm[g] = __ballot_sync(0xffffffffu, in && kk < T);
+          eqm[g] = __ballot_sync(0xffffffffu, in && kk == T);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int j = c0 + 32 * g + lane;
+          uint32_t evm = ltm[g];
+          if (eqm[g]) {  // keys == T: evicted while their rank among them is below the quota
+            const bool e =
+                ((eqm[g] >> lane) & 1u) && eq_run + __popc(eqm[g] & lanelt) < quota;
+            evm |= __ballot_sync(0xffffffffu, e);
+          }
+          const bool ev = (evm >> lane) & 1u;
+          const int ev_before = ev_run + __popc(evm & lanelt);
+          if (j < w_hi) {
+            // the guards only matter after a wait gave up (inconsistent counts)
+            if (ev) {
+              if (ev_before >= 0 && ev_before < p.max_evict) eout[ev_before] = j;
+            } else {
+              const int r = j - ev_before;
+              if (r >= 0 && r < p.max_keep) kout[r] = j;
+            }
+          }
+          ev_run += __popc(evm);
+          eq_run += __popc(eqm[g]);
+        }
       }
     }
     // slots past this row's own counts (rows shorter than the maxima): -1
