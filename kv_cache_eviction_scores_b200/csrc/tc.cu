@@ -28,7 +28,7 @@
 // k_tc_combine: merges the partials of a row into the final max M, normaliser
 //   L and output A = O / L; writes -2A as bf16 hi/lo planes (same split) plus
 //   the per-query constants (M, 1/L, L, ||A||^2) for the second pass.
-// k_tc_pass2<true> (token-major, one CTA per (b, h, chunk, split)): the
+// k_tc_pass2 (token-major, one CTA per (b, h, chunk, split)): the
 //   attention-only control score (section 结果与独立对照): S^T = K_tile Q^T,
 //   tcgen05 M=128 (tokens) N=nqc (queries) K=128, into two TMEM buffers; each
 //   thread owns one token and sums p = exp2(S*c - M') over its warp's
@@ -540,25 +540,17 @@ __device__ __forceinline__ float attn16(const uint32_t* r, const float4* kf, uin
   return acc;
 }
 
-// kAttn = false: the DropKV perturbation score.  kAttn = true: the attention-
-// only score; the CTA then streams K alone and issues only the S^T MMA.
-template <bool kAttn>
+// The attention-only score: the CTA streams K alone through a ring of kRing2
+// 32 KB slots and issues only the S^T MMA, into one of two TMEM buffers.
 __global__ void __maxnreg__(kMaxRegs2)
-k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmAhi,
-           const __grid_constant__ CUtensorMap tmAlo, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int nqc = a.nqc;
-  // A ring of kRing2 32 KB slots takes the K and V tiles in turn (K_0, V_0,
-  // K_1, ...).  When A needs its low part, the last slot holds A_lo instead and
-  // the ring runs on the first kRing2 - 1 slots.
   uint8_t* sRing = smem;
-  uint8_t* sAl = smem + (kRing2 - 1) * kTileBytes;
   uint8_t* sQ = smem + kRing2 * kTileBytes;  // nqc rows x 2 boxes
-  uint8_t* sAh = sQ + nqc * 256;
-  float4* kf = reinterpret_cast<float4*>(sAh + nqc * 256);   // [nqc/2] fast-path constants
-  float* nAmax = reinterpret_cast<float*>(kf + nqc / 2);      // [nqc/16] max ||A||^2 per chunk
-  uint64_t* bars = reinterpret_cast<uint64_t*>(nAmax + 8);    // 5 + 2 kRing2 barriers
+  float4* kf = reinterpret_cast<float4*>(sQ + nqc * 256);     // [nqc/2] (-M'_t, -M'_t+1, -, -)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kf + nqc / 2);  // 5 + 2 kRing2 barriers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5 + 2 * kRing2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -589,74 +581,34 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     fence_mbar_init();
   }
   pdl_trigger();
-  pdl_wait();  // qstat, A and ||v||^2 come from the combine and pass 1
+  pdl_wait();  // qstat comes from the combine
   if (threadIdx.x < nqc) {
     const int i = threadIdx.x;
     const float4 q = a.qstat[qrow0 + i];  // (M, 1/L, L, ||A||^2)
-    float* kff = reinterpret_cast<float*>(kf);
-    kff[(i >> 1) * 4 + (i & 1)] = -(q.x + log2f(q.z));  // -M' folds 1/L into the exponent
-    kff[(i >> 1) * 4 + 2 + (i & 1)] = q.w;
+    reinterpret_cast<float*>(kf)[(i >> 1) * 4 + (i & 1)] = -(q.x + log2f(q.z));  // -M'
   }
-  if (threadIdx.x < 8) nAmax[threadIdx.x] = 0.f;
   if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
     tc_fence_before();
   }
   __syncthreads();
-  if (threadIdx.x < nqc)  // ||A||^2 >= 0, so the float bits order like ints
-    atomicMax(reinterpret_cast<int*>(nAmax) + threadIdx.x / 16,
-              __float_as_int(a.qstat[qrow0 + threadIdx.x].w));
-  __syncthreads();
-  // Does A need its low part on this CTA's tiles?  Dropping A_lo leaves
-  // -2A rounded to bf16 (relative error <= 2^-8 per component), which moves
-  // -2 A.v by at most 2^-7 ||A|| ||v|| and so the squared distance
-  // ||A - v||^2 >= (||v|| - ||A||)^2 by a relative 2^-7 rho / (1 - rho)^2,
-  // rho = ||A|| / ||v||.  With ||A||^2 <= kLoSkip ||v||^2 for every query of
-  // the chunk and every token of the tiles (rho <= 0.0283) that is <= 2.4e-4.
-  bool lo = false;
-  if constexpr (!kAttn) {
-    float namx = 0.f;
-    for (int i = 0; i < (nqc + 15) / 16; ++i) namx = fmaxf(namx, nAmax[i]);
-    bool need = false;
-    for (int i = threadIdx.x; i < T * a.chunks1; i += blockDim.x) {
-      const float tm = a.tmin[((size_t)z * a.ntmax + t0) * a.chunks1 + i];
-      if (!(namx <= kLoSkip * tm)) need = true;  // NaN-safe
-    }
-    lo = __syncthreads_or(need) != 0;
-  }
-  const int R = lo ? kRing2 - 1 : kRing2;  // ring slots in use
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
   if (warp == kWarpTma) {
     if (lane == 0) {
-      prefetch_tmap(&tmQ); prefetch_tmap(&tmAhi); prefetch_tmap(&tmAlo);
-      prefetch_tmap(&tmK); prefetch_tmap(&tmV);
-      mbar_expect_tx(BQ, (kAttn ? 1 : lo ? 3 : 2) * nqc * 256);
+      prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
+      mbar_expect_tx(BQ, nqc * 256);
       tma_load_2d(smem_u32(sQ), &tmQ, BQ, 0, qrow0);
       tma_load_2d(smem_u32(sQ) + nqc * 128, &tmQ, BQ, 64, qrow0);
-      if (!kAttn) {
-        tma_load_2d(smem_u32(sAh), &tmAhi, BQ, 0, qrow0);
-        tma_load_2d(smem_u32(sAh) + nqc * 128, &tmAhi, BQ, 64, qrow0);
-      }
-      if (lo) {
-        tma_load_2d(smem_u32(sAl), &tmAlo, BQ, 0, qrow0);
-        tma_load_2d(smem_u32(sAl) + nqc * 128, &tmAlo, BQ, 64, qrow0);
-      }
-      // single thread: no warp vote needed.  Perturbation: K_j at i = 2j and
-      // V_j at 2j + 1; attention-only: K_j at i = j.
-      // (slot, phase) of load i kept incrementally: R is a runtime ring size
-      const int nload = kAttn ? T : 2 * T;
-      int r = 0, ph = 0;
-      for (int i = 0; i < nload && !*abort_flag; ++i, r = (r + 1 == R) ? 0 : r + 1, ph ^= (r == 0)) {
+      for (int j = 0; j < T && !*abort_flag; ++j) {  // K_j in slot j % kRing2
+        const int r = j % kRing2, ph = (j / kRing2) & 1;
         if (!mbar_wait(EMPTY(r), ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
         mbar_expect_tx(FULL(r), kTileBytes);
         const uint32_t dst = smem_u32(sRing + r * kTileBytes);
-        const CUtensorMap* m = (!kAttn && (i & 1)) ? &tmV : &tmK;
-        const int row = (t0 + (kAttn ? i : i >> 1)) * kTok;
-        tma_load_3d(dst, m, FULL(r), 0, row, z);
-        tma_load_3d(dst + kBox, m, FULL(r), 64, row, z);
+        tma_load_3d(dst, &tmK, FULL(r), 0, (t0 + j) * kTok, z);
+        tma_load_3d(dst + kBox, &tmK, FULL(r), 64, (t0 + j) * kTok, z);
       }
     }
   } else if (warp == kWarpMma) {
@@ -664,54 +616,24 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     bool ok = warp_wait(BQ, 0);
     if (!ok) fail(a, abort_flag);
     const SDesc rd0 = sdesc_split(smem_u32(sRing), 16, 1024);  // ring slot 0
-    const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024), hd = sdesc_split(smem_u32(sAh), 16, 1024),
-                ld = sdesc_split(smem_u32(sAl), 16, 1024);
+    const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024);
     const uint32_t nq = (uint32_t)nqc;
-    // ring (slot, phase) of K_j kept incrementally (R is a runtime ring size):
-    // V_j follows K_j, K_{j+1} follows V_j (or K_j for the attention score)
-    int pos = 0, pph = 0;
     for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
-      const int rk = pos, pk = pph;
-      int rv = rk + 1, pv = pk;
-      if (rv == R) { rv = 0; pv ^= 1; }
-      if (kAttn) {
-        pos = rv; pph = pv;
-      } else {
-        pos = rv + 1; pph = pv;
-        if (pos == R) { pos = 0; pph ^= 1; }
-      }
-      const uint32_t dS = tbase + (uint32_t)(s * 256), dD = dS + 128u;
+      const int rk = j % kRing2, pk = (j / kRing2) & 1;
       if (!warp_wait(TF(s), ph ^ 1) || !warp_wait(FULL(rk), pk)) {
         fail(a, abort_flag);
         break;
       }
       tc_fence_after();
       const uint32_t klo = rd0.lo + (uint32_t)rk * (kTileBytes >> 4);
-      const uint32_t vlo = rd0.lo + (uint32_t)rv * (kTileBytes >> 4);
       if (lane == 0) {
+        const uint32_t dS = tbase + (uint32_t)(s * 256);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ss_w(dS, klo + kslice(kk, 128), rd0.hi, qd.lo + kslice(kk, nq), qd.hi, IDT,
                    kk > 0 ? 1u : 0u);
         mma_commit(EMPTY(rk));
-        if (kAttn) mma_commit(MD(s));
-      }
-      __syncwarp();
-      if (kAttn) continue;
-      if (!warp_wait(FULL(rv), pv)) { fail(a, abort_flag); break; }
-      tc_fence_after();
-      if (lane == 0) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss_w(dD, vlo + kslice(kk, 128), rd0.hi, hd.lo + kslice(kk, nq), hd.hi, IDT,
-                   kk > 0 ? 1u : 0u);
-        if (lo) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss_w(dD, vlo + kslice(kk, 128), rd0.hi, ld.lo + kslice(kk, nq), ld.hi, IDT, 1u);
-        }
-        mma_commit(EMPTY(rv));
         mma_commit(MD(s));
       }
       __syncwarp();
@@ -720,95 +642,38 @@ k_tc_pass2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     // Sixteen warps work on every tile: warp (g, quarter) owns the tokens
     // [32 quarter, +32) of the tile (its TMEM lanes) and the query columns
     // [32 g, min(nqc, 32 g + 32)), and writes its own partial-score plane.
+    // A warp with no columns still walks the tiles, hands every buffer back
+    // and writes zeros to its plane.
     const int g = warp >> 2, ql = warp & 3;
     const int row = ql * 32 + lane;  // token within the tile
     const uint32_t lane_off = (uint32_t)(ql * 32) << 16;
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
     const int ch0 = min(nqc / 16, 2 * g), ch1 = min(nqc / 16, 2 * g + 2);  // 16-column chunks
-    const float4* qrows = a.qstat + qrow0;
-    const float* arows = a.attn_f32 + (size_t)qrow0 * kHd;
+    const int nch = ch1 - ch0;  // 0, 1 or 2 (warp-uniform)
     float* plane = a.parts + (size_t)(chunk * 4 + g) * a.part_stride + (size_t)z * a.n_max;
-    const int nch = ch1 - ch0;  // this warp's 16-column chunks: 0, 1 or 2 (warp-uniform)
-    // ||v_j||^2 of the next tile is fetched one tile ahead: under the streaming
-    // traffic a global load takes of the order of a tile's work to return
-    auto nv_at = [&](int jj) -> float {
-      const int tk = (t0 + jj) * kTok + row;
-      return (!kAttn && jj < T && tk < L) ? a.nvbuf[(size_t)z * a.ntmax * kTok + tk] : 0.f;
-    };
-    float nv_next = nv_at(0);
-    int sing = 0;
-    // A warp with no columns (nch = 0) still walks the tiles: it hands every
-    // buffer back and writes zeros to its plane.
     for (int j = 0; j < T; ++j) {
       const int s = j & 1, ph = (j >> 1) & 1;
       const int tile0 = (t0 + j) * kTok;
       const int tok = tile0 + row;
-      const bool valid = tok < L;
-      const float nv = nv_next;
-      nv_next = nv_at(j + 1);
-      const __nv_bfloat16* vrow_g = a.v + ((size_t)z * a.n_max + (valid ? tok : 0)) * kHd;
       if (!warp_wait(MD(s), ph)) { fail(a, abort_flag); break; }
       if (warp_aborted(abort_flag)) break;
       tc_fence_after();
       const uint32_t tS = tbase + (uint32_t)(s * 256) + lane_off + (uint32_t)(ch0 * 16);
-      const uint32_t tD = tS + 128u;
       const bool masked = tile0 + kTok - 1 > L - a.w;
-      // The buffer goes back to the MMA warp as soon as its last columns this
-      // warp needs are in registers (before the last chunk's arithmetic), so
-      // that the MMAs of tile j + 2 overlap the rest of this tile's work.
-      auto release = [&]() {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(TF(s));
-      };
-      // score of 16 columns (chunk ch) from S^T in r[0..15] and D in r[16..31]
-      auto chunk_score = [&](const uint32_t(&r)[32], int ch) -> float {
-        bool redo = masked;
-        uint64_t a2 = pk2(0.f, 0.f);
-        if (!masked) {
-          float pmax = 0.f;
-          fast16(r, kf + ch * 8, c2, pk2(nv, nv), a2, pmax);
-          // a large p (>= 2^-4: the series above would be short) or possible
-          // cancellation (||A||^2 >= 0.6 ||v||^2): the careful path
-          redo = pmax >= 0.0625f || nAmax[ch] >= 0.6f * nv;
-        }
-        if (__any_sync(0xffffffffu, redo)) {
-          uint32_t rc[32];
-#pragma unroll
-          for (int k = 0; k < 32; ++k) rc[k] = r[k];
-          return careful16(rc, ch * 16, tok, masked, L, a.w, chunk * nqc, qrows, c, nv, arows,
-                           vrow_g, &sing);
-        }
-        float x0, x1;
-        upk2(a2, x0, x1);
-        return x0 + x1;
-      };
       float acc = 0.f;
-      if (nch == 0) {
-        release();
-      } else if (kAttn) {
-        uint32_t r[32];
-        tmem_ld32(tS, r);  // S^T of chunks ch0, ch0 + 1 (the second unused when nch = 1)
-        release();
-        acc = attn16(r, kf + ch0 * 8, c2, masked, tok, L, a.w, chunk * nqc, ch0 * 16, c);
-        if (nch > 1)
-          acc += attn16(r + 16, kf + ch0 * 8 + 8, c2, masked, tok, L, a.w, chunk * nqc,
-                        ch0 * 16 + 16, c);
-      } else {
-        uint32_t r[32];
-        tmem_ld16x2(tS, tD, r);  // chunk ch0: 16 columns of S^T and of D
-        if (nch == 1) release();
-        acc = chunk_score(r, ch0);
-        if (nch > 1) {
-          tmem_ld16x2(tS + 16u, tD + 16u, r);  // chunk ch0 + 1
-          release();
-          acc += chunk_score(r, ch0 + 1);
-        }
-      }
-      if (valid) plane[tok] = acc;
+      uint32_t r[32];
+      if (nch > 0) tmem_ld32(tS, r);  // S^T of chunks ch0, ch0 + 1 (the second unused when nch = 1)
+      // the buffer goes back as soon as the columns are in registers
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(TF(s));
+      if (nch > 0) acc = attn16(r, kf + ch0 * 8, c2, masked, tok, L, a.w, chunk * nqc, ch0 * 16, c);
+      if (nch > 1)
+        acc += attn16(r + 16, kf + ch0 * 8 + 8, c2, masked, tok, L, a.w, chunk * nqc,
+                      ch0 * 16 + 16, c);
+      if (tok < L) plane[tok] = acc;
     }
-    if (sing) atomicMax(a.status, (int)DROPKV_ERR_SINGULAR);
   }
   tc_fence_before();
   __syncthreads();
@@ -860,7 +725,7 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
 
 size_t pass1_smem() { return (2 + kStK + kSt1) * (size_t)kTileBytes + kBars1 * 8 + 8; }
 size_t pass2_smem(int nqc) {
-  return kRing2 * (size_t)kTileBytes + 2 * (size_t)nqc * 256 + (size_t)nqc / 2 * 16 + 8 * 4 +
+  return kRing2 * (size_t)kTileBytes + (size_t)nqc * 256 + (size_t)nqc / 2 * 16 +
          (5 + 2 * kRing2) * 8 + 8;
 }
 
@@ -912,7 +777,6 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
                              float* stats_out, int32_t* status, int score, int cta_budget,
                              cudaStream_t st, KernelEvents& kev, int* nparts_used) {
   const bool attn_only = score == DROPKV_SCORE_ATTENTION;
-  auto pass2 = k_tc_pass2<true>;  // the attention-only control; DropKV runs the pair kernel
   const TcPlan plan = tc_plan(s);
   TcArgs a;
   memset(&a, 0, sizeof(a));
@@ -978,8 +842,8 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   const size_t sm1 = pass1_smem(), sm2 = pass2_smem(plan.nqc);
   cudaError_t e = cudaFuncSetAttribute(k_tc_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sm1);
-  if (e == cudaSuccess && attn_only)
-    e = cudaFuncSetAttribute(pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+  if (e == cudaSuccess && attn_only)  // the attention-only control; DropKV runs the pair kernel
+    e = cudaFuncSetAttribute(k_tc_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
   if (e != cudaSuccess) return e;
   *nparts_used = 4 * (attn_only ? plan.chunks : plan.chunks2);
 
@@ -993,7 +857,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   if (e != cudaSuccess) return e;
   kev.begin(st);
   if (attn_only) {
-    e = launch_ex(pass2, dim3(ctas), dim3(kThreads2), sm2, st, true, 1, mQ2, mAh, mAl, mK, mV, a);
+    e = launch_ex(k_tc_pass2, dim3(ctas), dim3(kThreads2), sm2, st, true, 1, mQ2, mK, a);
   } else {
     e = launch_tc_pass2_pair(a, mQ2, mAh, mAl, mK, mV, pairs, st);
   }

@@ -68,7 +68,7 @@ constexpr int kMaxCtas = 160;      // split target ceiling (one CTA per SM)
 constexpr int kSt1 = 3;            // pass-1 V stages
 constexpr int kStK = 2;            // pass-1 K stages
 constexpr int kBars1 = 1 + 2 * kStK + 2 * kSt1 + 6;  // pass-1 mbarriers
-constexpr int kRing2 = 5;          // pass-2 ring of 32 KB K/V slots (the last one doubles as A_lo)
+constexpr int kRing2 = 5;          // attention-only pass 2: ring of 32 KB K slots
 constexpr float kLoSkip = 8e-4f;   // pass 2 drops A_lo when ||A||^2 <= kLoSkip ||v||^2 throughout
 
 
