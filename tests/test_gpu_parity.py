@@ -204,11 +204,25 @@ def test_nonsingular_async_status_is_ok():
 
 # ---- selection on constructed scores (ties, +inf, NaN padding) --------------
 
-@pytest.mark.parametrize("case", ["ties", "keep_all", "evict_all", "long", "huge", "nan_in_range"])
+# The launch picks the cluster size (1, 2, 4 or 8 CTAs) from the longest row
+# and, when 8-CTA clusters would need a second wave, 4-CTA clusters with
+# 32768-key ranges: the cases below reach every kind.  "ties" and the other
+# short cases: one CTA per segment; "long": 2; "mid": 4; "wide": 8 CTAs with
+# 32768-key ranges; "many_rows": 20 segments of ~100K keys on 4-CTA clusters
+# with 32768-key ranges; "huge": uncached ranges.
+@pytest.mark.parametrize("case", ["ties", "keep_all", "evict_all", "long", "mid", "wide",
+                                  "many_rows", "huge", "nan_in_range"])
 def test_select_exact_on_constructed_scores(case):
     rng = np.random.default_rng(3)
     if case == "long":
         B, Hkv, n_max, lengths = 2, 3, 20000, [20000, 13001]
+    elif case == "mid":
+        B, Hkv, n_max, lengths = 2, 2, 60000, [60000, 33001]
+    elif case == "wide":
+        B, Hkv, n_max, lengths = 1, 2, 200000, [200000]
+    elif case == "many_rows":
+        B, Hkv, n_max = 20, 1, 100000
+        lengths = [100000 - 997 * b for b in range(B)]
     elif case == "huge":
         # per-CTA ranges of 37500 keys: past the shared-memory key cache, three
         # sub-ranges per CTA read from global memory
