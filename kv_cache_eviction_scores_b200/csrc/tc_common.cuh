@@ -146,19 +146,31 @@ __device__ __noinline__ float direct_sqdist(const float* A, const __nv_bfloat16*
 }
 
 // Fast path for 16 query columns of one token (every p < 2^-4, no possible
-// cancellation, every key visible): packed fp32 pairs,
+// cancellation): packed fp32 pairs,
 //   p = 2^(x c - M'),  M' = M + log2 L,
 //   ratio = p / (1 - p) = p (1 + p (1 + p (1 + p (1 + p)))) + O(p^6)
 //   (relative truncation error p^5 / (1 - p) <= 1.0e-6 for p < 2^-4),
 //   s += ratio^2 (D' + ||A||^2 + ||v||^2)   with D' = -2 A.v from the MMA.
 // kf holds (-M'_t, -M'_t+1, ||A_t||^2, ||A_t+1||^2) per column pair.
+// kMask: the causal window mask -- column u is the window query at position
+// pbase + (m0 + u) mod w and sees the token only up to that position; a key
+// it does not see gets p = 0 (the exponent is -inf).
+template <bool kMask>
 __device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf, uint64_t c2,
-                                       uint64_t nv2, uint64_t& acc2, float& pmax) {
+                                       uint64_t nv2, uint64_t& acc2, float& pmax, int tok = 0,
+                                       int pbase = 0, int m0 = 0, int w = 1) {
+  int m = m0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float4 k = kf[i];
     float y0, y1;
     upk2(ffma2(pk2(f32(r[2 * i]), f32(r[2 * i + 1])), c2, pk2(k.x, k.y)), y0, y1);
+    if constexpr (kMask) {
+      if (tok > pbase + m) y0 = -INFINITY;
+      m = m + 1 == w ? 0 : m + 1;
+      if (tok > pbase + m) y1 = -INFINITY;
+      m = m + 1 == w ? 0 : m + 1;
+    }
     const float p0 = ex2(y0), p1 = ex2(y1);
     pmax = fmax3(pmax, p0, p1);
     const uint64_t P = pk2(p0, p1);

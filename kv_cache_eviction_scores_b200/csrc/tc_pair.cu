@@ -269,7 +269,9 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int tile0 = (valid_tile ? tile_at(i) : my0) * kTok;
       const int tok = tile0 + row;
       const bool valid = valid_tile && tok < L;
-      const bool masked = tile0 + kTok - 1 > L - a.w;  // warp-uniform
+      // only the window's last w keys can be hidden from a window query: the
+      // warp's 32 tokens need the mask when they reach past L - w (warp-uniform)
+      const bool masked = tile0 + 32 * ql + 31 > L - a.w;
       const float nv = nv_next;
       nv_next = nv_at(i + 1);
       const __nv_bfloat16* vrow = a.v + ((size_t)z * a.n_max + (valid ? tok : 0)) * kHd;
@@ -294,15 +296,21 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // score of 16 columns (chunk ch of the half) from S^T in r[0..15] and D
         // in r[16..31]
         auto chunk_score = [&](const uint32_t(&r)[32], int ch) -> float {
-          bool redo = masked;
           uint64_t a2 = pk2(0.f, 0.f);
+          float pmax = 0.f;
+          const float4* kfc = kf + (hc0 / 2) + ch * 8;
           if (!masked) {
-            float pmax = 0.f;
-            fast16(r, kf + (hc0 / 2) + ch * 8, c2, pk2(nv, nv), a2, pmax);
-            // a large p (>= 2^-4: the series above would be short) or possible
-            // cancellation (||A||^2 >= 0.6 ||v||^2): the careful path
-            redo = pmax >= 0.0625f || nAmax[hc0 / 16 + ch] >= 0.6f * nv;
+            fast16<false>(r, kfc, c2, pk2(nv, nv), a2, pmax);
+          } else {
+            // the window's causal mask: column u is the window query at
+            // position L - w + (chunk * nqc + hc0 + 16 ch + u) mod w
+            fast16<true>(r, kfc, c2, pk2(nv, nv), a2, pmax, tok, L - a.w,
+                         (chunk * nqc + hc0 + ch * 16) % a.w, a.w);
           }
+          // a large p (>= 2^-4: the series above would be short) or possible
+          // cancellation (||A||^2 >= 0.6 ||v||^2): the careful path (lanes past
+          // L write nothing and do not vote)
+          const bool redo = valid && (pmax >= 0.0625f || nAmax[hc0 / 16 + ch] >= 0.6f * nv);
           if (__any_sync(0xffffffffu, redo)) {
             uint32_t rc[32];
 #pragma unroll
