@@ -1,10 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of DropKV prefill-time eviction scoring on B200.
 
-One step = the whole scoring path on one input set: dropkv_scores (window
-attention statistics, exact single-removal perturbation scores summed over the
-window, GQA mean-merge, MaxPool1D, window protection) followed by dropkv_select
-(exact lowest-score eviction per KV head).
+One step = the whole scoring path on one input set, in one call of the public
+API, dropkv_scores_select: window attention statistics, exact single-removal
+perturbation scores summed over the window, GQA mean-merge, MaxPool1D, window
+protection (the scores are written out), then the exact lowest-score eviction
+per KV head -- the results of dropkv_scores followed by dropkv_select.
 
 Workload (N=1): the 128K-token Llama-3.1-8B-shaped case -- B=1, Hq=32, Hkv=8,
 d=128, n=131072, w=64, bf16 Gaussian Q/K/V with 4 outlier K channels x8 per KV
@@ -45,7 +46,9 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 CSRC = os.path.join(ROOT, "kv_cache_eviction_scores_b200", "csrc")
 
-# kernel order per scoring call (must match the library's launch sequence)
+# kernel order of the scoring kernels of a call (must match the library's
+# launch sequence); a step (dropkv_scores_select) runs them and then the
+# selection kernel
 KERNELS = {
     "simt": ["k_simt_pass1", "k_simt_pass2", "k_epilogue"],
     # the DropKV score's second pass runs on CTA pairs; the attention-only
@@ -426,23 +429,24 @@ def run_ours(args):
     path = {dk.PATH_SIMT: "simt", dk.PATH_TENSOR: "tensor"}[
         dk.auto_path(shape) if args.path == "auto" else {"simt": 1, "tensor": 2}[args.path]]
     ws = torch.empty(dk.scores_workspace_bytes(shape), dtype=torch.uint8, device=dev)
-    sel_ws = torch.empty(max(16, dk.select_workspace_bytes(spec.B, spec.Hkv, spec.n_max)),
-                         dtype=torch.uint8, device=dev)
     scores = torch.empty(spec.B, spec.Hkv, spec.n_max, dtype=torch.float32, device=dev)
+    keep_idx = torch.empty(spec.B, spec.Hkv, max(spec.keep), dtype=torch.int32, device=dev)
+    ev_idx = torch.empty(spec.B, spec.Hkv, max(L - kc for L, kc in zip(wl.lengths, wl.keep)),
+                         dtype=torch.int32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    names = KERNELS["tensor_attention" if path == "tensor" and args.score == "attention" else path]
+    scoring = KERNELS["tensor_attention" if path == "tensor" and args.score == "attention"
+                      else path]
+    n_launch = dk.scores_select_launches(shape, wl.lengths, path)
+    names = scoring + ["k_select"]
     nk = len(names)
 
     def step(events=None):
-        dk.dropkv_scores(q, k, v, spec.window, spec.pool, wl.lengths, path=path, out=scores,
-                         workspace=ws, status=status, score=args.score,
-                         kernel_events=events[:2 * nk] if events else None)
-        if events:
-            events[2 * nk].record()  # the select launches, on the same (current) stream
-        out = dk.dropkv_select(scores, wl.keep, wl.lengths, workspace=sel_ws)
-        if events:
-            events[2 * nk + 1].record()
-        return out
+        # scoring and eviction in one call of the public API
+        _, kk, ee = dk.dropkv_scores_select(
+            q, k, v, spec.window, spec.pool, wl.keep, wl.lengths, path=path, score=args.score,
+            out=scores, keep_idx=keep_idx, evict_idx=ev_idx, workspace=ws, status=status,
+            kernel_events=events)
+        return kk, ee
 
     K, Wm = args.steps, args.warmup
     # K and V are read twice a step; when they fit L2 it is flushed before every
@@ -451,7 +455,7 @@ def run_ours(args):
     kv_bytes = 2 * spec.Hkv * sum(wl.lengths) * spec.d * 2
     flush_buf = (torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev)
                  if kv_bytes <= 2 * l2_bytes else None)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk + 2)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(K)]
     for row in ev:
         for e in row:
             e.record()  # creates the handle
@@ -511,8 +515,6 @@ def run_ours(args):
     for j, name in enumerate(names):
         kern_us[name] = statistics.mean(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1])
                                         for i in range(K)) * 1e3
-    kern_us["select (all launches)"] = statistics.mean(
-        ev[i][2 * nk].elapsed_time(ev[i][2 * nk + 1]) for i in range(K)) * 1e3
     if int(status.item()) != dk.OK:
         raise dk.SingularError(int(status.item()), "bench inputs")
 
@@ -524,13 +526,13 @@ def run_ours(args):
     tokens = sum(wl.lengths)
     value = whole_job_value(world, tokens, ms)
     hbm_peak, tc_peak, sm_mhz, peak_src = peaks()
-    dominant = max(names, key=kern_us.get)
+    sel_names = [n for n in names if n.startswith("k_select")]
+    dominant = max((n for n in names if n not in sel_names), key=kern_us.get)
     roof = roofline(dominant, spec, kern_us[dominant], hbm_peak, tc_peak, sm_mhz, args.score)
     roof["kernel"] = dominant
     roof["peak_of"] = peak_src
     alg_bytes = kv_bytes + q.numel() * 2 + spec.B * spec.Hkv * spec.n_max * 4
-    launches = dk.scores_launches(shape, wl.lengths, path) + dk.select_launches(
-        spec.B, spec.Hkv, spec.n_max, wl.lengths)
+    launches = n_launch
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -553,8 +555,8 @@ def run_ours(args):
                 "of": peak_src,
                 "frac_nominal": alg_bytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
                 "nominal_gbs": NOMINAL_HBM_GBS},
-        "phases_us": {"scores": sum(kern_us[n] for n in names),
-                      "select": kern_us["select (all launches)"]},
+        "phases_us": {"scores": sum(kern_us[n] for n in names if n not in sel_names),
+                      "select": sum(kern_us[n] for n in sel_names)},
         "ms_per_step_with_kernel_events": ms_events,
         "plan": (tensor_plan(spec, torch.cuda.get_device_properties(dev).multi_processor_count)
                  if path == "tensor" else None),

@@ -80,7 +80,7 @@ typedef struct dropkv_shape {
   int32_t n_max;        /* padded cache length (row stride of k, v, scores)   */
   int32_t d;            /* head dimension, 1..256                             */
   int32_t window;       /* w >= 1; every length must satisfy w < L_b <= n_max */
-  int32_t pool_kernel;  /* MaxPool1D kernel size: odd, >= 1 (1 = no pooling)  */
+  int32_t pool_kernel;  /* MaxPool1D kernel size: odd, 1..1023 (1 = no pooling) */
   int32_t dtype;        /* dropkv_dtype of q, k and v                         */
 } dropkv_shape;
 
@@ -230,6 +230,31 @@ DROPKV_API dropkv_status dropkv_select_noalloc(int32_t B, int32_t Hkv, int32_t n
                                                int32_t max_keep, int32_t* evict_idx,
                                                int32_t max_evict, void* stream);
 
+/*
+ * Scoring and eviction in one call (write-up section 核心公式 and the whole of
+ * Algorithm 1): the work of dropkv_scores_ex followed by dropkv_select_ex on
+ * its scores, with the same results -- `scores` written exactly as
+ * dropkv_scores writes them, and the same keep / evict lists -- enqueued by
+ * one call (each batch slice of up to 64 rows is scored and then selected).
+ *   Arguments as dropkv_scores_ex (shape, q, k, v, lengths, scores,
+ *   workspace of dropkv_scores_workspace_bytes(shape) bytes, stream, options)
+ *   and dropkv_select (keep_counts, keep_idx, max_keep, evict_idx, max_evict).
+ *   status_dev NULL: synchronous; returns DROPKV_ERR_SINGULAR or
+ *   DROPKV_ERR_TIMEOUT when the kernels raised one.  status_dev non-NULL
+ *   (device int32, caller-owned): asynchronous; *status_dev receives the
+ *   largest code the kernels raised.  Host-side errors are returned directly
+ *   and nothing is enqueued.  On DROPKV_ERR_SINGULAR the scores and lists are
+ *   unspecified.
+ */
+DROPKV_API dropkv_status dropkv_scores_select(const dropkv_shape* shape, const void* q,
+                                              const void* k, const void* v,
+                                              const int32_t* lengths, const int32_t* keep_counts,
+                                              float* scores, int32_t* keep_idx, int32_t max_keep,
+                                              int32_t* evict_idx, int32_t max_evict,
+                                              void* workspace, size_t workspace_bytes,
+                                              void* stream, int32_t* status_dev,
+                                              const dropkv_options* options);
+
 /* Which path DROPKV_PATH_AUTO picks for this shape (DROPKV_PATH_SIMT or
  * DROPKV_PATH_TENSOR); no device needed.  Returns -1 for an invalid shape. */
 DROPKV_API int32_t dropkv_auto_path(const dropkv_shape* shape);
@@ -239,6 +264,9 @@ DROPKV_API int32_t dropkv_auto_path(const dropkv_shape* shape);
 DROPKV_API int32_t dropkv_scores_launches(const dropkv_shape* shape, const int32_t* lengths,
                                int32_t path);
 DROPKV_API int32_t dropkv_select_launches(int32_t B, int32_t Hkv, int32_t n_max, const int32_t* lengths);
+/* Kernel launches of one dropkv_scores_select call (-1 for an invalid shape). */
+DROPKV_API int32_t dropkv_scores_select_launches(const dropkv_shape* shape, const int32_t* lengths,
+                                                 int32_t path);
 
 /* Static description of a status code. */
 DROPKV_API const char* dropkv_status_string(dropkv_status status);

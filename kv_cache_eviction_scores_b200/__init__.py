@@ -114,6 +114,11 @@ def lib():
     L.dropkv_scores_launches.restype = i32
     L.dropkv_select_launches.argtypes = [i32, i32, i32, ip]
     L.dropkv_select_launches.restype = i32
+    L.dropkv_scores_select.argtypes = [sp, vp, vp, vp, ip, ip, vp, vp, i32, vp, i32, vp, sz, vp,
+                                       vp, ctypes.POINTER(Options)]
+    L.dropkv_scores_select.restype = i32
+    L.dropkv_scores_select_launches.argtypes = [sp, ip, i32]
+    L.dropkv_scores_select_launches.restype = i32
     L.dropkv_status_string.argtypes = [i32]
     L.dropkv_status_string.restype = ctypes.c_char_p
     L.dropkv_abi_version.argtypes = []
@@ -196,6 +201,11 @@ def scores_launches(shape: Shape, lengths=None, path: str = "auto") -> int:
 
 def select_launches(B: int, Hkv: int, n_max: int, lengths=None) -> int:
     return int(lib().dropkv_select_launches(B, Hkv, n_max, _i32_array(lengths)))
+
+
+def scores_select_launches(shape: Shape, lengths=None, path: str = "auto") -> int:
+    return int(lib().dropkv_scores_select_launches(ctypes.byref(shape), _i32_array(lengths),
+                                                   _PATHS[path]))
 
 
 def _check_inputs(q, k, v):
@@ -346,10 +356,64 @@ def dropkv_select(scores: torch.Tensor, keep_counts: Sequence[int],
     return keep_idx, evict_idx
 
 
+def dropkv_scores_select(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, window: int,
+                         pool_kernel: int, keep_counts: Sequence[int],
+                         lengths: Optional[Sequence[int]] = None, *, path: str = "auto",
+                         score: str = "perturbation", out: Optional[torch.Tensor] = None,
+                         keep_idx: Optional[torch.Tensor] = None,
+                         evict_idx: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None,
+                         status: Optional[torch.Tensor] = None, kernel_events=None,
+                         tc_ctas: int = 0):
+    """Scores and the keep / evict lists in one call (dropkv_scores_select):
+    (scores, keep_idx, evict_idx), the same results as dropkv_scores followed
+    by dropkv_select.  With ``status`` the call is asynchronous (the device
+    status lands there); otherwise it synchronises and raises on a
+    device-side error.  ``kernel_events`` as for dropkv_scores."""
+    if score not in _SCORES:
+        raise ValueError(f"score must be one of {sorted(_SCORES)}")
+    _check_inputs(q, k, v)
+    shape = make_shape(q, k, window, pool_kernel)
+    dev = q.device
+    B, Hkv, n_max = shape.B, shape.Hkv, shape.n_max
+    lens = list(lengths) if lengths is not None else [n_max] * B
+    keep = [int(x) for x in keep_counts]
+    if len(keep) != B or len(lens) != B:
+        raise ValueError("keep_counts and lengths need one entry per batch row")
+    max_keep = max(keep)
+    max_evict = max(L - kc for L, kc in zip(lens, keep))
+    if out is None:
+        out = torch.empty(B, Hkv, n_max, dtype=torch.float32, device=dev)
+    if keep_idx is None:
+        keep_idx = torch.empty(B, Hkv, max_keep, dtype=torch.int32, device=dev)
+    if evict_idx is None:
+        evict_idx = torch.empty(B, Hkv, max_evict, dtype=torch.int32, device=dev)
+    need = scores_workspace_bytes(shape)
+    if need == 0:
+        raise DropKVError(ERR_ARG, "dropkv_scores_workspace_bytes")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    opts = Options(_PATHS[path], _SCORES[score], None, None, None, 0, int(tc_ctas))
+    ev_arr = None
+    if kernel_events:
+        ev_arr = (ctypes.c_void_p * len(kernel_events))(*[e.cuda_event for e in kernel_events])
+        opts.events = ctypes.cast(ev_arr, ctypes.c_void_p)
+        opts.n_events = len(kernel_events)
+    if status is not None and (not status.is_cuda or status.dtype != torch.int32):
+        raise TypeError("status must be a CUDA int32 tensor")
+    st = lib().dropkv_scores_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                    _i32_array(lengths), _i32_array(keep), _ptr(out),
+                                    _ptr(keep_idx), keep_idx.shape[2], _ptr(evict_idx),
+                                    evict_idx.shape[2], _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(dev),
+                                    _ptr(status), ctypes.byref(opts))
+    _check(st, "dropkv_scores_select")
+    return out, keep_idx, evict_idx
+
+
 def evict(q, k, v, window: int, pool_kernel: int, keep_counts: Sequence[int],
           lengths: Optional[Sequence[int]] = None, *, path: str = "auto",
           score: str = "perturbation"):
     """Scores and the keep / evict lists in one call: (scores, keep_idx, evict_idx)."""
-    s = dropkv_scores(q, k, v, window, pool_kernel, lengths, path=path, score=score)
-    keep_idx, evict_idx = dropkv_select(s, keep_counts, lengths)
-    return s, keep_idx, evict_idx
+    return dropkv_scores_select(q, k, v, window, pool_kernel, keep_counts, lengths, path=path,
+                                score=score)

@@ -181,11 +181,22 @@ dropkv_status run_select(int32_t B, int32_t Hkv, int32_t n_max, const float* sco
   return DROPKV_OK;
 }
 
-// Runs the scoring pipeline; `sync` selects the synchronous contract.
+// The selection dropkv_scores_select adds to the scoring call.
+struct SelectSpec {
+  const int32_t* keep_counts;
+  int32_t* keep_idx;
+  int32_t max_keep;
+  int32_t* evict_idx;
+  int32_t max_evict;
+};
+
+// Runs the scoring pipeline, and after each batch slice's scores its
+// selection when `sel` is given; `sync` selects the synchronous contract.
 static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const void* k,
                                 const void* v, const int32_t* lengths, float* scores,
                                 void* workspace, size_t ws_bytes, void* stream,
-                                int32_t* status_dev, const dropkv_options* opt, bool sync) {
+                                int32_t* status_dev, const dropkv_options* opt, bool sync,
+                                const SelectSpec* sel = nullptr) {
   dropkv_status r = validate_shape(sp, lengths);
   if (r != DROPKV_OK) return r;
   const dropkv_shape& s = *sp;
@@ -201,6 +212,11 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
   const int path = resolve_path(s, opt ? opt->path : DROPKV_PATH_AUTO);
   if (path == -2) return DROPKV_ERR_ARG;
   if (path == -1) return DROPKV_ERR_UNSUPPORTED;
+  if (sel) {
+    r = check_select_args(s.B, s.Hkv, s.n_max, scores, lengths, sel->keep_counts, sel->keep_idx,
+                          sel->max_keep, sel->evict_idx, sel->max_evict);
+    if (r != DROPKV_OK) return r;
+  }
   const size_t need = dropkv_scores_workspace_bytes(sp);
   if (!workspace || ws_bytes < need || !aligned16(workspace)) return DROPKV_ERR_WORKSPACE;
   r = check_device();
@@ -237,6 +253,7 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
     void* attn_ws = ws + lay.attn;
     float* parts = reinterpret_cast<float*>(ws + lay.parts);
     const size_t part_stride = (size_t)Bs * s.Hkv * s.n_max;
+    int nparts = path == DROPKV_PATH_SIMT ? 1 : lay.nparts;
     cudaError_t e;
     if (path == DROPKV_PATH_SIMT) {
       kev.begin(st);
@@ -248,20 +265,22 @@ static dropkv_status run_scores(const dropkv_shape* sp, const void* q, const voi
                               st);
         kev.end(st);
       }
-      if (e == cudaSuccess) {
-        kev.begin(st);
-        e = launch_epilogue(s, lens, parts, 1, part_stride, sc, st);
-        kev.end(st);
-      }
     } else {
-      int nparts = lay.nparts;
       e = launch_tc_scores(s, qs, ks, vs, lens, lay, ws, attn_user, stats_user, status_word, score,
                            tc_ctas, st, kev, &nparts);
-      if (e == cudaSuccess) {
-        kev.begin(st);
-        e = launch_epilogue(s, lens, parts, nparts, part_stride, sc, st);
-        kev.end(st);
-      }
+    }
+    if (e == cudaSuccess) {
+      kev.begin(st);
+      e = launch_epilogue(s, lens, parts, nparts, part_stride, sc, st);
+      kev.end(st);
+    }
+    if (e == cudaSuccess && sel) {  // the selection of this slice's rows
+      const size_t seg0 = (size_t)b0 * s.Hkv;
+      kev.begin(st);
+      e = launch_select(Bs, s.Hkv, s.n_max, sc, lens.L, sel->keep_counts + b0,
+                        sel->keep_idx + seg0 * sel->max_keep, sel->max_keep,
+                        sel->evict_idx + seg0 * sel->max_evict, sel->max_evict, status_word, st);
+      kev.end(st);
     }
     if (e != cudaSuccess) return e == cudaErrorNotSupported ? DROPKV_ERR_UNSUPPORTED : cuda_fail(e);
   }
@@ -309,6 +328,18 @@ dropkv_status dropkv_scores_ex(const dropkv_shape* shape, const void* q, const v
                                int32_t* status_dev, const dropkv_options* options) {
   return run_scores(shape, q, k, v, lengths, scores, workspace, workspace_bytes, stream,
                     status_dev, options, status_dev == nullptr);
+}
+
+dropkv_status dropkv_scores_select(const dropkv_shape* shape, const void* q, const void* k,
+                                   const void* v, const int32_t* lengths,
+                                   const int32_t* keep_counts, float* scores, int32_t* keep_idx,
+                                   int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
+                                   void* workspace, size_t workspace_bytes, void* stream,
+                                   int32_t* status_dev, const dropkv_options* options) {
+  if (!shape) return DROPKV_ERR_ARG;
+  const SelectSpec sel = {keep_counts, keep_idx, max_keep, evict_idx, max_evict};
+  return run_scores(shape, q, k, v, lengths, scores, workspace, workspace_bytes, stream,
+                    status_dev, options, status_dev == nullptr, &sel);
 }
 
 size_t dropkv_select_workspace_bytes(int32_t B, int32_t Hkv, int32_t n_max) {
@@ -376,6 +407,13 @@ int32_t dropkv_scores_launches(const dropkv_shape* shape, const int32_t* lengths
   const int slices = (shape->B + kMaxB - 1) / kMaxB;
   const int per = (p == DROPKV_PATH_SIMT) ? 3 : tc_launch_count() + 1;
   return slices * per;
+}
+
+int32_t dropkv_scores_select_launches(const dropkv_shape* shape, const int32_t* lengths,
+                                      int32_t path) {
+  const int32_t n = dropkv_scores_launches(shape, lengths, path);
+  if (n < 0) return -1;
+  return n + ((shape->B + kMaxB - 1) / kMaxB) * select_launch_count();
 }
 
 int32_t dropkv_select_launches(int32_t B, int32_t Hkv, int32_t n_max, const int32_t* lengths) {

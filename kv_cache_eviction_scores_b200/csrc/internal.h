@@ -141,8 +141,9 @@ cudaError_t launch_select(int B, int Hkv, int n_max, const float* scores, const 
                           cudaStream_t st);
 
 // The same launch for the select self-test: CTA rank 1 of every segment's
-// cluster withholds its first arrival and every bounded wait gives up after
-// wait_ns, so the segments with evictions end in DROPKV_ERR_TIMEOUT.
+// cluster withholds its arrivals of the first round and every bounded wait
+// gives up after wait_ns, so the segments with evictions end in
+// DROPKV_ERR_TIMEOUT.
 cudaError_t launch_select_stalled(int B, int Hkv, int n_max, const float* scores,
                                   const int32_t* L, const int32_t* keep, int32_t* keep_idx,
                                   int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
