@@ -24,7 +24,10 @@
 //   O_t += P_hi V + P_lo V (A from TMEM, V MN-major).  The reference max only
 //   moves up by more than 8, so exp2 stays <= 256 and O rarely rescales.
 //   While one query tile's softmax runs, the other tile's MMAs keep the
-//   tensor pipe busy.  Each CTA writes one partial (m, l, O) per row.
+//   tensor pipe busy.  A chunk of at most 128 rows is one query tile: then the
+//   two warpgroups take alternate token tiles, each with its own S/P buffer
+//   and O, and are folded together at the end.  Each CTA writes one partial
+//   (m, l, O) per row.
 // k_tc_combine: merges the partials of a row into the final max M, normaliser
 //   L and output A = O / L; writes -2A as bf16 hi/lo planes (same split) plus
 //   the per-query constants (M, 1/L, L, ||A||^2) for the second pass.
@@ -99,12 +102,21 @@ __device__ __noinline__ bool p1_rescale_o(uint32_t tO, float fac, uint32_t pd_ba
   return true;
 }
 
-// One CTA per (b, h, query chunk, token split).  The chunk's rows (<= 256)
-// are two query tiles of 128 rows; a K/V tile in shared memory serves both.
-// Tensor-pipe order per tile j: P V of tile 0, S of tile 0 for j + 1, P V of
-// tile 1, S of tile 1 for j + 1 -- each query tile's S overwrites its own P,
-// so it waits for that P V; the other tile's work keeps the pipe busy while
-// one tile's softmax runs.
+// One CTA per (b, h, query chunk, token split), two softmax warpgroups, each
+// with its own S/P buffer and O accumulator in TMEM (warpgroup u: S/P at
+// columns 128 u, O at 256 + 128 u) and its own running max and normaliser.
+//  * kAlt = false (chunks of more than 128 rows): the chunk's rows (<= 256)
+//    are two query tiles of 128 rows and warpgroup u owns tile u; a K/V tile
+//    in shared memory serves both.  Tensor-pipe order per tile j: P V of tile
+//    0, S of tile 0 for j + 1, P V of tile 1, S of tile 1 for j + 1.
+//  * kAlt = true (chunks of at most 128 rows, one query tile): the warpgroups
+//    take the token tiles in turn (warpgroup u the tiles j = u mod 2), so the
+//    second warpgroup does not idle.  Tensor-pipe order: S(0), S(1), then per
+//    tile j: P V(j), S(j + 2).  At the end warpgroup 0 folds warpgroup 1's
+//    (max, normaliser, O) into its own and writes the row's one partial.
+// A warpgroup's next S overwrites its P, so it waits for the P V that reads
+// it; the other warpgroup's work keeps the tensor pipe busy meanwhile.
+template <bool kAlt>
 __global__ void __launch_bounds__(kThreads1, 1)
 k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
@@ -115,6 +127,7 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kSt1 * kTileBytes);  // kBars1 barriers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kBars1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* xml = reinterpret_cast<float2*>(tmem_slot + 2);  // [128] kAlt: warpgroup 1's (m, l)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1 KB alignment
     if (threadIdx.x == 0) atomicMax(a.status, (int)DROPKV_ERR_CUDA);
@@ -126,9 +139,9 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int T = t1 - t0;
   const int L = a.L[b];
   const int R = min(a.rows1, a.nq - chunk * a.rows1);  // this chunk's query rows
-  const int nt = R > 128 ? 2 : 1;                       // query tiles
+  const int nt = kAlt ? 1 : (R > 128 ? 2 : 1);          // query tiles
   // barriers: Q; K full/empty (kStK stages); V full/empty (kSt1 stages); per
-  // query tile: S ready, P written, P V done
+  // softmax warpgroup: S ready, P written, P V done
   const uint32_t BQ = smem_u32(&bars[0]);
   auto KF = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto KE = [&](int s) { return smem_u32(&bars[1 + kStK + s]); };
@@ -204,36 +217,40 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024);
     const SDesc kd0 = sdesc_split(smem_u32(sK), 16, 1024);
     const SDesc vd0 = sdesc_split(smem_u32(sV), kBox, 1024);
-    // S_t(i) = Q_t K_i^T into tile t's S/P columns, which hold P_t(i - 1)
-    // until P V_t(i - 1) has read it
-    auto issue_S = [&](int t, int i) {
-      const int s = i % kStK, ph = (i / kStK) & 1;
+    // S = Q_q K_j^T (query tile q) into warpgroup u's S/P columns, the n-th
+    // S of that warpgroup; they hold its previous P until the P V reading it
+    // has completed.  K_j's last reader commits the stage free.
+    auto issue_S = [&](int u, int q, int j, int n) {
+      const int s = j % kStK, ph = (j / kStK) & 1;
       if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
-      if (i >= 1 && !warp_wait(PD(t), (uint32_t)((i - 1) & 1))) { fail(a, abort_flag); return false; }
+      if (n >= 1 && !warp_wait(PD(u), (uint32_t)((n - 1) & 1))) { fail(a, abort_flag); return false; }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t qlo = qd.lo + (uint32_t)t * (kTileBytes >> 4);
+        const uint32_t qlo = qd.lo + (uint32_t)q * (kTileBytes >> 4);
         const uint32_t klo = kd0.lo + (uint32_t)s * (kTileBytes >> 4);
-        const uint32_t dS = tbase + (uint32_t)(128 * t);
+        const uint32_t dS = tbase + (uint32_t)(128 * u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ss_w(dS, qlo + kslice(kk, 128), qd.hi, klo + kslice(kk, 128), kd0.hi, IDS,
                    kk > 0 ? 1u : 0u);
-        mma_commit(SF(t));
-        if (t == nt - 1) mma_commit(KE(s));  // the last reader of this K stage
+        mma_commit(SF(u));
+        if (kAlt || u == nt - 1) mma_commit(KE(s));
       }
       __syncwarp();
       return true;
     };
-    auto issue_PV = [&](int t, int i) {
-      const int s = i % kSt1, ph = (i / kSt1) & 1;
-      if (!warp_wait(PF(t), (uint32_t)(i & 1))) { fail(a, abort_flag); return false; }
+    // O_u += P V_j, the n-th P V of warpgroup u; V_j's last reader commits the
+    // stage free
+    auto issue_PV = [&](int u, int j, int n) {
+      const int s = j % kSt1, ph = (j / kSt1) & 1;
+      if (!warp_wait(PF(u), (uint32_t)(n & 1))) { fail(a, abort_flag); return false; }
       if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
       uint8_t* vb = sV + s * kTileBytes;
-      const int tile0 = (t0 + i) * kTok;
-      if (t == 0 && tile0 + kTok > L) {
-        // rows at or beyond L hold no data (possibly NaN): zero them so that the
-        // P = 0 weights of those rows contribute exactly 0 to O
+      const int tile0 = (t0 + j) * kTok;
+      if ((kAlt || u == 0) && tile0 + kTok > L) {
+        // rows at or beyond L hold no data (possibly NaN): zero them (once per
+        // V tile, before its first P V) so that the P = 0 weights of those
+        // rows contribute exactly 0 to O
         const int r0 = L - tile0;
         for (int idx = r0 * 8 + lane; idx < kTok * 8; idx += 32) {
           const int r = idx >> 3, c16 = idx & 7;
@@ -246,29 +263,37 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tc_fence_after();
       if (lane == 0) {
         const uint32_t vlo = vd0.lo + (uint32_t)s * (kTileBytes >> 4);
-        const uint32_t dO = tbase + kColO1 + (uint32_t)(128 * t);
-        const uint32_t pS = tbase + (uint32_t)(128 * t);
+        const uint32_t dO = tbase + kColO1 + (uint32_t)(128 * u);
+        const uint32_t pS = tbase + (uint32_t)(128 * u);
         // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16);
         // V slice kk starts 16 rows (2048 bytes) further
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts_w(dO, pS + (uint32_t)(16 * kk), vlo + (uint32_t)kk * 128u, vd0.hi, IDP,
-                   (i > 0 || kk > 0) ? 1u : 0u);
+                   (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
-        mma_commit(PD(t));
-        if (t == nt - 1) mma_commit(VE(s));  // the last reader of this V stage
+        mma_commit(PD(u));
+        if (kAlt || u == nt - 1) mma_commit(VE(s));
       }
       __syncwarp();
       return true;
     };
-    for (int t = 0; t < nt && t < 2 && ok && T > 0; ++t) ok = issue_S(t, 0);
-    for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j)
-      for (int t = 0; t < nt && ok; ++t) {
-        ok = issue_PV(t, j);
-        if (ok && j + 1 < T) ok = issue_S(t, j + 1);
+    if (kAlt) {
+      for (int j = 0; j < 2 && j < T && ok; ++j) ok = issue_S(j, 0, j, 0);
+      for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
+        ok = issue_PV(j & 1, j, j >> 1);
+        if (ok && j + 2 < T) ok = issue_S(j & 1, 0, j + 2, (j >> 1) + 1);
       }
+    } else {
+      for (int t = 0; t < nt && ok && T > 0; ++t) ok = issue_S(t, t, 0, 0);
+      for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j)
+        for (int t = 0; t < nt && ok; ++t) {
+          ok = issue_PV(t, j, j);
+          if (ok && j + 1 < T) ok = issue_S(t, t, j + 1, j + 1);
+        }
+    }
   } else if (warp == kW1Nv) {
     // ---------------- ||v_j||^2 ----------------
     // This CTA's share of every V tile's rows (the query chunks of a KV head
@@ -312,25 +337,31 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     }
   } else if (warp < kSmWarps1) {
     // ---------------- softmax warps ----------------
-    // Warpgroup t owns query tile t; thread = one query row (its TMEM lane),
-    // all 128 tokens of a tile: a max pass over S, then P = 2^(S c - m)
-    // written back over S as hi/lo planes.  The reference max moves only when
-    // a tile exceeds it by more than 8 (so 2^(.) <= 256); then l and the row
-    // of O are rescaled, after the P V that last accumulated into O.
-    const int t = warp >> 2, ql = warp & 3;
-    const int row = ql * 32 + lane;       // row within the query tile
-    const int crow = 128 * t + row;       // row within the chunk
+    // Warpgroup u: query tile u and every token tile (kAlt = false), or the
+    // query tile and the token tiles j = u, u + 2, ... (kAlt = true).  Thread
+    // = one query row (its TMEM lane), all 128 tokens of a tile: a max pass
+    // over S, then P = 2^(S c - m) written back over S as hi/lo planes.  The
+    // reference max moves only when a tile exceeds it by more than 8 (so
+    // 2^(.) <= 256); then l and the row of the warpgroup's O are rescaled,
+    // after the P V that last accumulated into it.
+    const int u = warp >> 2, ql = warp & 3;
+    const int row = ql * 32 + lane;                // row within the query tile
+    const int crow = kAlt ? row : 128 * u + row;   // row within the chunk
     const bool valid_row = crow < R;
     const int Prow = L - a.w + (chunk * a.rows1 + crow) % a.w;
     const uint32_t lane_off = (uint32_t)(ql * 32) << 16;
-    const uint32_t tS = tbase + (uint32_t)(128 * t) + lane_off;
-    const uint32_t tO = tbase + kColO1 + (uint32_t)(128 * t) + lane_off;
+    const uint32_t tS = tbase + (uint32_t)(128 * u) + lane_off;
+    const uint32_t tO = tbase + kColO1 + (uint32_t)(128 * u) + lane_off;
     const float c = a.c_log2;
     const uint64_t c2 = pk2(c, c);
     float m_ref = -INFINITY, l = 0.f;
-    bool live = t < nt;  // a second warpgroup without a second tile only idles
-    for (int j = 0; j < T && live; ++j) {
-      if (!warp_wait(SF(t), (uint32_t)(j & 1))) { fail(a, abort_flag); live = false; break; }
+    // this warpgroup's tiles (a second warpgroup without a second query tile
+    // has none when kAlt is false)
+    const int nmine = kAlt ? (T > u ? (T - u + 1) / 2 : 0) : (u < nt ? T : 0);
+    bool live = true;
+    for (int n = 0; n < nmine && live; ++n) {
+      const int j = kAlt ? u + 2 * n : n;
+      if (!warp_wait(SF(u), (uint32_t)(n & 1))) { fail(a, abort_flag); live = false; break; }
       if (warp_aborted(abort_flag)) { live = false; break; }
       tc_fence_after();
       const int tok0 = (t0 + j) * kTok;
@@ -340,28 +371,29 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tmem_ld128(tS, sr);
       if (masked) {
 #pragma unroll
-        for (int u = 0; u < 128; ++u)
-          if (tok0 + u > Prow) sr[u] = 0xFF800000u;  // -inf
+        for (int x = 0; x < 128; ++x)
+          if (tok0 + x > Prow) sr[x] = 0xFF800000u;  // -inf
       }
       float ya = -INFINITY, yb = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 128; u += 4) {
-        ya = fmax3(ya, f32(sr[u]), f32(sr[u + 1]));
-        yb = fmax3(yb, f32(sr[u + 2]), f32(sr[u + 3]));
+      for (int x = 0; x < 128; x += 4) {
+        ya = fmax3(ya, f32(sr[x]), f32(sr[x + 1]));
+        yb = fmax3(yb, f32(sr[x + 2]), f32(sr[x + 3]));
       }
       const float mt = fmaxf(ya, yb) * c;  // c > 0: commutes with the max
       float fac = 1.f;
       bool resc = false;
       if (mt > m_ref + 8.f) {
         if (m_ref != -INFINITY) fac = ex2(m_ref - mt);
-        resc = m_ref != -INFINITY && j > 0;
+        resc = m_ref != -INFINITY && n > 0;
         m_ref = mt;
         l *= fac;
       }
       // warp-uniform: every lane votes, and all or none call the rescale; O
-      // holds P V up to tile j - 1, which has landed once PD completes its phase
+      // holds the warpgroup's P V up to its previous tile, which has landed
+      // once PD completes that phase
       if (__any_sync(0xffffffffu, resc) &&
-          !p1_rescale_o(tO, fac, PD(t), (uint32_t)((j - 1) & 1))) {
+          !p1_rescale_o(tO, fac, PD(u), (uint32_t)((n - 1) & 1))) {
         fail(a, abort_flag);
         live = false;
         break;
@@ -373,28 +405,63 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(PF(t));
+      if (lane == 0) mbar_arrive(PF(u));
     }
-    // partial row: O, the reference max, the normaliser
-    if (t < nt) {
-      bool have = live && T > 0 && !warp_aborted(abort_flag);
-      if (have) {
-        if (!warp_wait(PD(t), (uint32_t)((T - 1) & 1))) {
-          fail(a, abort_flag);
-          have = false;
-        }
-        tc_fence_after();
+    // the warpgroup's O is complete once its last P V has landed
+    bool have = live && nmine > 0 && !warp_aborted(abort_flag);
+    bool own = false;  // O read from this warpgroup's accumulator
+    if (have) {
+      if (!warp_wait(PD(u), (uint32_t)((nmine - 1) & 1))) {
+        fail(a, abort_flag);
+        have = false;
       }
+      tc_fence_after();
+    }
+    own = have;
+    // kAlt: warpgroup 1 hands (m, l) over through shared memory; warpgroup 0
+    // reads its O straight from TMEM (same lanes) and folds it in
+    float w0 = 1.f, w1 = 0.f;
+    bool have1 = false;
+    if (kAlt) {
+      if (u == 1) xml[row] = make_float2(have ? m_ref : -INFINITY, have ? l : 0.f);
+      tc_fence_before();
+      named_barrier_sync(1, kSmWarps1 * 32);  // both softmax warpgroups, unconditionally
+      tc_fence_after();
+      if (u == 0) {
+        const float2 ml1 = xml[row];
+        have1 = ml1.x != -INFINITY;
+        const float m0 = have ? m_ref : -INFINITY;
+        const float M = fmaxf(m0, ml1.x);
+        w0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
+        w1 = have1 ? ex2(ml1.x - M) : 0.f;
+        l = (have ? w0 * l : 0.f) + (have1 ? w1 * ml1.y : 0.f);
+        m_ref = M;
+        have = have || have1;
+      }
+    }
+    // the row's partial: O, the reference max, the normaliser
+    if (u < nt) {
       float* out = a.partial + ((size_t)blockIdx.x * a.rows1 + crow) * kPartStride;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
-        if (have) tmem_ld32(tO + 32u * cc, o);
+        if (own) {
+          tmem_ld32(tO + 32u * cc, o);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = 0u;
+        }
+        if (kAlt && have1) {
+          uint32_t o1[32];
+          tmem_ld32(tO + 128u + 32u * cc, o1);  // warpgroup 1's O
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = u32(fmaf(w1, f32(o1[x]), w0 * f32(o[x])));
+        }
         if (valid_row) {
 #pragma unroll
-          for (int u = 0; u < 32; u += 4)
-            *reinterpret_cast<float4*>(out + 32 * cc + u) =
-                have ? make_float4(f32(o[u]), f32(o[u + 1]), f32(o[u + 2]), f32(o[u + 3]))
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(out + 32 * cc + x) =
+                have ? make_float4(f32(o[x]), f32(o[x + 1]), f32(o[x + 2]), f32(o[x + 3]))
                      : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
@@ -723,7 +790,7 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t heads, uint64_t n_max) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t pass1_smem() { return (2 + kStK + kSt1) * (size_t)kTileBytes + kBars1 * 8 + 8; }
+size_t pass1_smem() { return (2 + kStK + kSt1) * (size_t)kTileBytes + kBars1 * 8 + 8 + 128 * 8; }
 size_t pass2_smem(int nqc) {
   return kRing2 * (size_t)kTileBytes + (size_t)nqc * 256 + (size_t)nqc / 2 * 16 +
          (5 + 2 * kRing2) * 8 + 8;
@@ -840,7 +907,10 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
     return cudaErrorNotSupported;
 
   const size_t sm1 = pass1_smem(), sm2 = pass2_smem(plan.nqc);
-  cudaError_t e = cudaFuncSetAttribute(k_tc_pass1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // one query tile per chunk: the two softmax warpgroups alternate token tiles
+  const bool alt1 = plan.rows1 <= 128;
+  auto* pass1 = alt1 ? k_tc_pass1<true> : k_tc_pass1<false>;
+  cudaError_t e = cudaFuncSetAttribute(pass1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sm1);
   if (e == cudaSuccess && attn_only)  // the attention-only control; DropKV runs the pair kernel
     e = cudaFuncSetAttribute(k_tc_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
@@ -848,7 +918,7 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   *nparts_used = 4 * (attn_only ? plan.chunks : plan.chunks2);
 
   kev.begin(st);
-  k_tc_pass1<<<ctas1, kThreads1, sm1, st>>>(mQ1, mK, mV, a);
+  pass1<<<ctas1, kThreads1, sm1, st>>>(mQ1, mK, mV, a);
   kev.end(st);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kev.begin(st);
