@@ -55,11 +55,10 @@ namespace {
 
 // =========================== pass 1 =========================================
 // P = exp2(S c - mu) for 16 tokens of one query row (S in s16[0..15], masked
-// keys at -inf) written as 8 hi + 8 lo bf16 pair columns at TMEM column tcol
-// (the layout P V reads: hi of the 16 tokens, then lo).  No wait on the store.
-// Returns the sum of P over the 16 tokens.  Warp-collective.
-__device__ __forceinline__ float p1_exp16(const uint32_t* s16, uint32_t tcol, uint64_t c2,
-                                          uint64_t nmu2) {
+// keys at -inf), written back over s16 as 8 hi + 8 lo bf16 pair words (the
+// column layout P V reads: hi of the 16 tokens, then lo).  Returns the sum of
+// P over the 16 tokens.
+__device__ __forceinline__ float p1_exp16(uint32_t* s16, uint64_t c2, uint64_t nmu2) {
   uint64_t l2 = pk2(0.f, 0.f);
   uint32_t pw[16];
 #pragma unroll
@@ -76,7 +75,8 @@ __device__ __forceinline__ float p1_exp16(const uint32_t* s16, uint32_t tcol, ui
     upk2(fadd2(E, pk2(nh0, nh1)), r0, r1);  // exact remainders e - hi
     pw[8 + u2] = pack_bf16_rn(r0, r1);
   }
-  tmem_st16(tcol, pw);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) s16[k] = pw[k];
   float la, lb;
   upk2(l2, la, lb);
   return la + lb;
@@ -176,166 +176,180 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const uint32_t tbase = *tmem_slot;
   const int z = b * a.Hkv + h;
   const int qrow0 = (b * a.Hkv + h) * a.nq + chunk * a.rows1;
+  // Two query tiles: the producer warpgroup (TMA, MMA and ||v||^2 warps)
+  // hands registers to the softmax warpgroups, whose rows of 128 logits
+  // otherwise spill.  The shares add up to the launch's 384 x 168.
+  constexpr uint32_t kRegsSm = 224, kRegsPr = 56;
+  static_assert(kThreads1 == 384 && kSmWarps1 == 8 &&
+                    2 * 128 * kRegsSm + 128 * kRegsPr == kThreads1 * 168,
+                "register split of pass 1");
 
-  if (warp == kW1Tma || warp == kW1TmaV) {
-    // ---------------- TMA producers ----------------
-    // warp kW1Tma: the query tiles, then K_0, K_1, ... (K_{i+2} once both
-    // query tiles' S have read K_i); warp kW1TmaV: V_0, V_1, ... (kSt1 ahead).
-    if (lane == 0) {
-      const bool kq = warp == kW1Tma;
-      if (kq) {
-        prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
-        mbar_expect_tx(BQ, (uint32_t)nt * 2u * 128u * (uint32_t)a.qbox_rows);
-        for (int t = 0; t < nt; ++t) {  // rows past the tensor read as zeros
-          tma_load_2d(smem_u32(sQ) + t * kTileBytes, &tmQ, BQ, 0, qrow0 + 128 * t);
-          tma_load_2d(smem_u32(sQ) + t * kTileBytes + kBox, &tmQ, BQ, 64, qrow0 + 128 * t);
+  if (warp >= kSmWarps1) {
+    if constexpr (!kAlt) setmaxnreg_dec<kRegsPr>();
+    if (warp == kW1Tma || warp == kW1TmaV) {
+      // ---------------- TMA producers ----------------
+      // warp kW1Tma: the query tiles, then K_0, K_1, ... (K_{i+2} once both
+      // query tiles' S have read K_i); warp kW1TmaV: V_0, V_1, ... (kSt1 ahead).
+      if (lane == 0) {
+        const bool kq = warp == kW1Tma;
+        if (kq) {
+          prefetch_tmap(&tmQ); prefetch_tmap(&tmK);
+          mbar_expect_tx(BQ, (uint32_t)nt * 2u * 128u * (uint32_t)a.qbox_rows);
+          for (int t = 0; t < nt; ++t) {  // rows past the tensor read as zeros
+            tma_load_2d(smem_u32(sQ) + t * kTileBytes, &tmQ, BQ, 0, qrow0 + 128 * t);
+            tma_load_2d(smem_u32(sQ) + t * kTileBytes + kBox, &tmQ, BQ, 64, qrow0 + 128 * t);
+          }
+        } else {
+          prefetch_tmap(&tmV);
+        }
+        uint8_t* buf = kq ? sK : sV;
+        const int nst = kq ? kStK : kSt1;
+        const CUtensorMap* m = kq ? &tmK : &tmV;
+        for (int i = 0; i < T && !*abort_flag; ++i) {
+          const int st = i % nst, ph = (i / nst) & 1;
+          const uint32_t full = kq ? KF(st) : VF(st), empty = kq ? KE(st) : VE(st);
+          if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
+          mbar_expect_tx(full, kTileBytes);
+          const uint32_t dst = smem_u32(buf + st * kTileBytes);
+          tma_load_3d(dst, m, full, 0, (t0 + i) * kTok, z);
+          tma_load_3d(dst + kBox, m, full, 64, (t0 + i) * kTok, z);
+        }
+      }
+    } else if (warp == kW1Mma) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T
+      constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);    // O += P V (V MN-major)
+      bool ok = warp_wait(BQ, 0);
+      if (!ok) fail(a, abort_flag);
+      // operand descriptors of stage 0; a stage, tile or K slice only moves the
+      // start address, i.e. adds to the low word
+      const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024);
+      const SDesc kd0 = sdesc_split(smem_u32(sK), 16, 1024);
+      const SDesc vd0 = sdesc_split(smem_u32(sV), kBox, 1024);
+      // S = Q_q K_j^T (query tile q) into warpgroup u's S/P columns, the n-th
+      // S of that warpgroup; they hold its previous P until the P V reading it
+      // has completed.  K_j's last reader commits the stage free.
+      auto issue_S = [&](int u, int q, int j, int n) {
+        const int s = j % kStK, ph = (j / kStK) & 1;
+        if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
+        if (n >= 1 && !warp_wait(PD(u), (uint32_t)((n - 1) & 1))) {
+          fail(a, abort_flag);
+          return false;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t qlo = qd.lo + (uint32_t)q * (kTileBytes >> 4);
+          const uint32_t klo = kd0.lo + (uint32_t)s * (kTileBytes >> 4);
+          const uint32_t dS = tbase + (uint32_t)(128 * u);
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss_w(dS, qlo + kslice(kk, 128), qd.hi, klo + kslice(kk, 128), kd0.hi, IDS,
+                     kk > 0 ? 1u : 0u);
+          mma_commit(SF(u));
+          if (kAlt || u == nt - 1) mma_commit(KE(s));
+        }
+        __syncwarp();
+        return true;
+      };
+      // O_u += P V_j, the n-th P V of warpgroup u; V_j's last reader commits the
+      // stage free
+      auto issue_PV = [&](int u, int j, int n) {
+        const int s = j % kSt1, ph = (j / kSt1) & 1;
+        if (!warp_wait(PF(u), (uint32_t)(n & 1))) { fail(a, abort_flag); return false; }
+        if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
+        uint8_t* vb = sV + s * kTileBytes;
+        const int tile0 = (t0 + j) * kTok;
+        if ((kAlt || u == 0) && tile0 + kTok > L) {
+          // rows at or beyond L hold no data (possibly NaN): zero them (once per
+          // V tile, before its first P V) so that the P = 0 weights of those
+          // rows contribute exactly 0 to O
+          const int r0 = L - tile0;
+          for (int idx = r0 * 8 + lane; idx < kTok * 8; idx += 32) {
+            const int r = idx >> 3, c16 = idx & 7;
+            *reinterpret_cast<uint4*>(vb + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(vb + kBox + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t vlo = vd0.lo + (uint32_t)s * (kTileBytes >> 4);
+          const uint32_t dO = tbase + kColO1 + (uint32_t)(128 * u);
+          const uint32_t pS = tbase + (uint32_t)(128 * u);
+          // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16);
+          // V slice kk starts 16 rows (2048 bytes) further
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts_w(dO, pS + (uint32_t)(16 * kk), vlo + (uint32_t)kk * 128u, vd0.hi, IDP,
+                     (n > 0 || kk > 0) ? 1u : 0u);
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
+          mma_commit(PD(u));
+          if (kAlt || u == nt - 1) mma_commit(VE(s));
+        }
+        __syncwarp();
+        return true;
+      };
+      if (kAlt) {
+        for (int j = 0; j < 2 && j < T && ok; ++j) ok = issue_S(j, 0, j, 0);
+        for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
+          ok = issue_PV(j & 1, j, j >> 1);
+          if (ok && j + 2 < T) ok = issue_S(j & 1, 0, j + 2, (j >> 1) + 1);
         }
       } else {
-        prefetch_tmap(&tmV);
-      }
-      uint8_t* buf = kq ? sK : sV;
-      const int nst = kq ? kStK : kSt1;
-      const CUtensorMap* m = kq ? &tmK : &tmV;
-      for (int i = 0; i < T && !*abort_flag; ++i) {
-        const int st = i % nst, ph = (i / nst) & 1;
-        const uint32_t full = kq ? KF(st) : VF(st), empty = kq ? KE(st) : VE(st);
-        if (!mbar_wait(empty, ph ^ 1, kWaitNs)) { fail(a, abort_flag); break; }
-        mbar_expect_tx(full, kTileBytes);
-        const uint32_t dst = smem_u32(buf + st * kTileBytes);
-        tma_load_3d(dst, m, full, 0, (t0 + i) * kTok, z);
-        tma_load_3d(dst + kBox, m, full, 64, (t0 + i) * kTok, z);
-      }
-    }
-  } else if (warp == kW1Mma) {
-    // ---------------- MMA issuer ----------------
-    constexpr uint32_t IDS = idesc_bf16(128, 128, false, false);   // S = Q K^T
-    constexpr uint32_t IDP = idesc_bf16(128, 128, false, true);    // O += P V (V MN-major)
-    bool ok = warp_wait(BQ, 0);
-    if (!ok) fail(a, abort_flag);
-    // operand descriptors of stage 0; a stage, tile or K slice only moves the
-    // start address, i.e. adds to the low word
-    const SDesc qd = sdesc_split(smem_u32(sQ), 16, 1024);
-    const SDesc kd0 = sdesc_split(smem_u32(sK), 16, 1024);
-    const SDesc vd0 = sdesc_split(smem_u32(sV), kBox, 1024);
-    // S = Q_q K_j^T (query tile q) into warpgroup u's S/P columns, the n-th
-    // S of that warpgroup; they hold its previous P until the P V reading it
-    // has completed.  K_j's last reader commits the stage free.
-    auto issue_S = [&](int u, int q, int j, int n) {
-      const int s = j % kStK, ph = (j / kStK) & 1;
-      if (!warp_wait(KF(s), ph)) { fail(a, abort_flag); return false; }
-      if (n >= 1 && !warp_wait(PD(u), (uint32_t)((n - 1) & 1))) { fail(a, abort_flag); return false; }
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t qlo = qd.lo + (uint32_t)q * (kTileBytes >> 4);
-        const uint32_t klo = kd0.lo + (uint32_t)s * (kTileBytes >> 4);
-        const uint32_t dS = tbase + (uint32_t)(128 * u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss_w(dS, qlo + kslice(kk, 128), qd.hi, klo + kslice(kk, 128), kd0.hi, IDS,
-                   kk > 0 ? 1u : 0u);
-        mma_commit(SF(u));
-        if (kAlt || u == nt - 1) mma_commit(KE(s));
-      }
-      __syncwarp();
-      return true;
-    };
-    // O_u += P V_j, the n-th P V of warpgroup u; V_j's last reader commits the
-    // stage free
-    auto issue_PV = [&](int u, int j, int n) {
-      const int s = j % kSt1, ph = (j / kSt1) & 1;
-      if (!warp_wait(PF(u), (uint32_t)(n & 1))) { fail(a, abort_flag); return false; }
-      if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); return false; }
-      uint8_t* vb = sV + s * kTileBytes;
-      const int tile0 = (t0 + j) * kTok;
-      if ((kAlt || u == 0) && tile0 + kTok > L) {
-        // rows at or beyond L hold no data (possibly NaN): zero them (once per
-        // V tile, before its first P V) so that the P = 0 weights of those
-        // rows contribute exactly 0 to O
-        const int r0 = L - tile0;
-        for (int idx = r0 * 8 + lane; idx < kTok * 8; idx += 32) {
-          const int r = idx >> 3, c16 = idx & 7;
-          *reinterpret_cast<uint4*>(vb + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(vb + kBox + r * 128 + c16 * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-      }
-      __syncwarp();
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t vlo = vd0.lo + (uint32_t)s * (kTileBytes >> 4);
-        const uint32_t dO = tbase + kColO1 + (uint32_t)(128 * u);
-        const uint32_t pS = tbase + (uint32_t)(128 * u);
-        // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16);
-        // V slice kk starts 16 rows (2048 bytes) further
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts_w(dO, pS + (uint32_t)(16 * kk), vlo + (uint32_t)kk * 128u, vd0.hi, IDP,
-                   (n > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
-        mma_commit(PD(u));
-        if (kAlt || u == nt - 1) mma_commit(VE(s));
-      }
-      __syncwarp();
-      return true;
-    };
-    if (kAlt) {
-      for (int j = 0; j < 2 && j < T && ok; ++j) ok = issue_S(j, 0, j, 0);
-      for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j) {
-        ok = issue_PV(j & 1, j, j >> 1);
-        if (ok && j + 2 < T) ok = issue_S(j & 1, 0, j + 2, (j >> 1) + 1);
-      }
-    } else {
-      for (int t = 0; t < nt && ok && T > 0; ++t) ok = issue_S(t, t, 0, 0);
-      for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j)
-        for (int t = 0; t < nt && ok; ++t) {
-          ok = issue_PV(t, j, j);
-          if (ok && j + 1 < T) ok = issue_S(t, t, j + 1, j + 1);
-        }
-    }
-  } else if (warp == kW1Nv) {
-    // ---------------- ||v_j||^2 ----------------
-    // This CTA's share of every V tile's rows (the query chunks of a KV head
-    // cover the same tokens and split the rows), 4 rows per lane; the order of
-    // the squares is free, so the 128-byte swizzle only picks a bank-conflict-
-    // free order.  Arrives on the V stage's empty barrier when done, and
-    // records the share's minimum for pass 2.
-    for (int j = 0; j < T; ++j) {
-      const int s = j % kSt1, ph = (j / kSt1) & 1;
-      if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); break; }
-      if (warp_aborted(abort_flag)) break;
-      const uint8_t* vb = sV + s * kTileBytes;
-      const int tile0 = (t0 + j) * kTok;
-      float vmin = INFINITY;
-      for (int rr = 0; rr < 4; ++rr) {
-        const int row = rr * 32 + lane;
-        if ((row * a.chunks1) / 128 != chunk || tile0 + row >= L) continue;
-        uint64_t acc2 = pk2(0.f, 0.f);
-#pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 q4 =
-                *reinterpret_cast<const uint4*>(vb + bx * kBox + row * 128 + ((q ^ (row & 7)) * 16));
-            const uint32_t wv[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t pr = pk2(f32(wv[k] << 16), f32(wv[k] & 0xFFFF0000u));
-              acc2 = ffma2(pr, pr, acc2);
-            }
+        for (int t = 0; t < nt && ok && T > 0; ++t) ok = issue_S(t, t, 0, 0);
+        for (int j = 0; j < T && ok && !warp_aborted(abort_flag); ++j)
+          for (int t = 0; t < nt && ok; ++t) {
+            ok = issue_PV(t, j, j);
+            if (ok && j + 1 < T) ok = issue_S(t, t, j + 1, j + 1);
           }
-        float na, nb;
-        upk2(acc2, na, nb);
-        a.nvbuf[(size_t)z * a.ntmax * kTok + tile0 + row] = na + nb;
-        vmin = fminf(vmin, na + nb);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(VE(s));
-      vmin = warp_min(vmin);  // pass 2 decides from it whether A needs its low part
-      if (lane == 0) a.tmin[((size_t)z * a.ntmax + t0 + j) * a.chunks1 + chunk] = vmin;
+    } else if (warp == kW1Nv) {
+      // ---------------- ||v_j||^2 ----------------
+      // This CTA's share of every V tile's rows (the query chunks of a KV head
+      // cover the same tokens and split the rows), 4 rows per lane; the order of
+      // the squares is free, so the 128-byte swizzle only picks a bank-conflict-
+      // free order.  Arrives on the V stage's empty barrier when done, and
+      // records the share's minimum for pass 2.
+      for (int j = 0; j < T; ++j) {
+        const int s = j % kSt1, ph = (j / kSt1) & 1;
+        if (!warp_wait(VF(s), ph)) { fail(a, abort_flag); break; }
+        if (warp_aborted(abort_flag)) break;
+        const uint8_t* vb = sV + s * kTileBytes;
+        const int tile0 = (t0 + j) * kTok;
+        float vmin = INFINITY;
+        for (int rr = 0; rr < 4; ++rr) {
+          const int row = rr * 32 + lane;
+          if ((row * a.chunks1) / 128 != chunk || tile0 + row >= L) continue;
+          uint64_t acc2 = pk2(0.f, 0.f);
+  #pragma unroll
+          for (int bx = 0; bx < 2; ++bx)
+  #pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint4 q4 = *reinterpret_cast<const uint4*>(vb + bx * kBox + row * 128 +
+                                                               ((q ^ (row & 7)) * 16));
+              const uint32_t wv[4] = {q4.x, q4.y, q4.z, q4.w};
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t pr = pk2(f32(wv[k] << 16), f32(wv[k] & 0xFFFF0000u));
+                acc2 = ffma2(pr, pr, acc2);
+              }
+            }
+          float na, nb;
+          upk2(acc2, na, nb);
+          a.nvbuf[(size_t)z * a.ntmax * kTok + tile0 + row] = na + nb;
+          vmin = fminf(vmin, na + nb);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(VE(s));
+        vmin = warp_min(vmin);  // pass 2 decides from it whether A needs its low part
+        if (lane == 0) a.tmin[((size_t)z * a.ntmax + t0 + j) * a.chunks1 + chunk] = vmin;
+      }
     }
-  } else if (warp < kSmWarps1) {
+  } else {
+    if constexpr (!kAlt) setmaxnreg_inc<kRegsSm>();
     // ---------------- softmax warps ----------------
     // Warpgroup u: query tile u and every token tile (kAlt = false), or the
     // query tile and the token tiles j = u, u + 2, ... (kAlt = true).  Thread
@@ -401,7 +415,8 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
       const uint64_t nmu2 = pk2(-mu, -mu);
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) l += p1_exp16(sr + 16 * cc, tS + 16u * cc, c2, nmu2);
+      for (int cc = 0; cc < 8; ++cc) l += p1_exp16(sr + 16 * cc, c2, nmu2);
+      tmem_st128(tS, sr);  // the whole row of P in one store
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

@@ -191,6 +191,26 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
 #undef DKV_O16
 }
 // 16 consecutive 32-bit columns stored for every lane (no wait).
+// 128 consecutive 32-bit columns stored for every lane (no wait).
+__device__ __forceinline__ void tmem_st128(uint32_t taddr, const uint32_t (&r)[128]) {
+#define DKV_I16(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \
+    "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7]), "r"(r[i + 8]), "r"(r[i + 9]), "r"(r[i + 10]), \
+    "r"(r[i + 11]), "r"(r[i + 12]), "r"(r[i + 13]), "r"(r[i + 14]), "r"(r[i + 15])
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x128.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, "
+      "%33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, "
+      "%49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, "
+      "%65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, "
+      "%81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, "
+      "%97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, "
+      "%113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127, %128};"
+      ::"r"(taddr), DKV_I16(0), DKV_I16(16), DKV_I16(32), DKV_I16(48), DKV_I16(64), DKV_I16(80),
+      DKV_I16(96), DKV_I16(112)
+      : "memory");
+#undef DKV_I16
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -331,6 +351,18 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
+}
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute the same instruction): raise or lower this warpgroup's per-thread
+// register count.  The raises of a CTA wait until the lowerings have freed
+// the registers they take.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 // Named barrier `id` (1..15) over `count` threads (whole warps).
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
