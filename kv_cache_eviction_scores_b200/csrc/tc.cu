@@ -241,7 +241,7 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const uint32_t qlo = qd.lo + (uint32_t)q * (kTileBytes >> 4);
           const uint32_t klo = kd0.lo + (uint32_t)s * (kTileBytes >> 4);
           const uint32_t dS = tbase + (uint32_t)(128 * u);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss_w(dS, qlo + kslice(kk, 128), qd.hi, klo + kslice(kk, 128), kd0.hi, IDS,
                      kk > 0 ? 1u : 0u);
@@ -279,11 +279,11 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const uint32_t pS = tbase + (uint32_t)(128 * u);
           // tokens 16kk..16kk+15: P_hi in columns [16kk, 16kk+8), P_lo in [16kk+8, 16kk+16);
           // V slice kk starts 16 rows (2048 bytes) further
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts_w(dO, pS + (uint32_t)(16 * kk), vlo + (uint32_t)kk * 128u, vd0.hi, IDP,
                      (n > 0 || kk > 0) ? 1u : 0u);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts_w(dO, pS + (uint32_t)(16 * kk + 8), vlo + (uint32_t)kk * 128u, vd0.hi, IDP, 1u);
           mma_commit(PD(u));
@@ -324,14 +324,14 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
           const int row = rr * 32 + lane;
           if ((row * a.chunks1) / 128 != chunk || tile0 + row >= L) continue;
           uint64_t acc2 = pk2(0.f, 0.f);
-  #pragma unroll
+#pragma unroll
           for (int bx = 0; bx < 2; ++bx)
-  #pragma unroll
+#pragma unroll
             for (int q = 0; q < 8; ++q) {
               const uint4 q4 = *reinterpret_cast<const uint4*>(vb + bx * kBox + row * 128 +
                                                                ((q ^ (row & 7)) * 16));
               const uint32_t wv[4] = {q4.x, q4.y, q4.z, q4.w};
-  #pragma unroll
+#pragma unroll
               for (int k = 0; k < 4; ++k) {
                 const uint64_t pr = pk2(f32(wv[k] << 16), f32(wv[k] & 0xFFFF0000u));
                 acc2 = ffma2(pr, pr, acc2);

@@ -55,7 +55,7 @@ constexpr int kTileBytes = 2 * kBox;
 constexpr int kSimtWarps = 16;     // pass-2 score warps: 4 per TMEM lane quarter
 constexpr int kWarpTma = kSimtWarps, kWarpMma = kSimtWarps + 1;
 constexpr int kThreads2 = (kSimtWarps + 2) * 32;  // pass 2: + TMA warp, MMA warp
-constexpr int kMaxRegs2 = 96;      // pass 2: 18 warps, 5 on a sub-partition (16K registers)
+constexpr int kMaxRegs2 = 96;      // second passes at launch: 5 warps on a sub-partition (16K registers)
 // pass 1: two softmax warpgroups (one per 128-row query tile, one row per
 // thread), TMA warps for Q/K and for V, an MMA warp and a ||v||^2 warp
 constexpr int kSmWarps1 = 8;
