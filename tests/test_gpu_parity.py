@@ -207,17 +207,20 @@ def test_nonsingular_async_status_is_ok():
 # The launch picks the cluster size (1, 2, 4 or 8 CTAs) from the longest row
 # and, when 8-CTA clusters would need a second wave, 4-CTA clusters with
 # 32768-key ranges: the cases below reach every kind.  "ties" and the other
-# short cases: one CTA per segment; "long": 2; "mid": 4; "wide": 8 CTAs with
-# 32768-key ranges; "many_rows": 20 segments of ~100K keys on 4-CTA clusters
-# with 32768-key ranges; "huge": uncached ranges.
-@pytest.mark.parametrize("case", ["ties", "keep_all", "evict_all", "long", "mid", "wide",
-                                  "many_rows", "huge", "nan_in_range"])
+# short cases: one CTA per segment; "long": 2; "mid": 4; "eight": 8 CTAs with
+# ragged rows; "wide": 8 CTAs with 32768-key ranges; "many_rows": 20 segments
+# of ~100K keys on 4-CTA clusters with 32768-key ranges; "huge": uncached
+# ranges.
+@pytest.mark.parametrize("case", ["ties", "keep_all", "evict_all", "long", "mid", "eight",
+                                  "wide", "many_rows", "huge", "nan_in_range"])
 def test_select_exact_on_constructed_scores(case):
     rng = np.random.default_rng(3)
     if case == "long":
         B, Hkv, n_max, lengths = 2, 3, 20000, [20000, 13001]
     elif case == "mid":
         B, Hkv, n_max, lengths = 2, 2, 60000, [60000, 33001]
+    elif case == "eight":
+        B, Hkv, n_max, lengths = 2, 2, 120000, [120000, 70001]
     elif case == "wide":
         B, Hkv, n_max, lengths = 1, 2, 200000, [200000]
     elif case == "many_rows":
