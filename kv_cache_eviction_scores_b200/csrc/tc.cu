@@ -178,10 +178,10 @@ k_tc_pass1(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
   const int qrow0 = (b * a.Hkv + h) * a.nq + chunk * a.rows1;
   // Two query tiles: the producer warpgroup (TMA, MMA and ||v||^2 warps)
   // hands registers to the softmax warpgroups, whose rows of 128 logits
-  // otherwise spill.  The shares add up to the launch's 384 x 168.
+  // otherwise spill.  The shares add up to the launch's 384 x kRegs1.
   constexpr uint32_t kRegsSm = 224, kRegsPr = 56;
   static_assert(kThreads1 == 384 && kSmWarps1 == 8 &&
-                    2 * 128 * kRegsSm + 128 * kRegsPr == kThreads1 * 168,
+                    2 * 128 * kRegsSm + 128 * kRegsPr == kThreads1 * kRegs1,
                 "register split of pass 1");
 
   if (warp >= kSmWarps1) {
@@ -927,6 +927,13 @@ cudaError_t launch_tc_scores(const dropkv_shape& s, const void* q, const void* k
   auto* pass1 = alt1 ? k_tc_pass1<true> : k_tc_pass1<false>;
   cudaError_t e = cudaFuncSetAttribute(pass1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sm1);
+  if (e == cudaSuccess && !alt1) {
+    // the register split of the two-query-tile schedule assumes the launch's
+    // kRegs1 registers a thread; any other count would leave its raise waiting
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, pass1);
+    if (e == cudaSuccess && fa.numRegs != kRegs1) return cudaErrorInvalidConfiguration;
+  }
   if (e == cudaSuccess && attn_only)  // the attention-only control; DropKV runs the pair kernel
     e = cudaFuncSetAttribute(k_tc_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
   if (e != cudaSuccess) return e;

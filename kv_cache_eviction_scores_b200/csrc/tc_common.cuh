@@ -61,6 +61,7 @@ constexpr int kMaxRegs2 = 96;      // second passes at launch: 5 warps on a sub-
 constexpr int kSmWarps1 = 8;
 constexpr int kW1Tma = 8, kW1Mma = 9, kW1Nv = 10, kW1TmaV = 11;
 constexpr int kThreads1 = 12 * 32;
+constexpr int kRegs1 = 168;        // pass 1's registers a thread at launch (65536 / 384, rounded down to 8)
 constexpr uint32_t kColO1 = 256;   // pass-1 TMEM: S/P of tile t at 128 t, O of tile t at 256 + 128 t
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kPartStride = kTcPartStride;  // floats per partial row: O[128], m, l, pad

@@ -384,6 +384,12 @@ cudaError_t launch_tc_pass2_pair(const TcArgs& a, const CUtensorMap& mQ, const C
   cudaError_t e = cudaFuncSetAttribute(k_tc_pass2_pair,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // the register split assumes the launch's kMaxRegs2 registers a thread; any
+  // other count would leave the score warps' raise waiting
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, k_tc_pass2_pair);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kMaxRegs2) return cudaErrorInvalidConfiguration;
   return launch_ex(k_tc_pass2_pair, dim3(2 * pairs), dim3(kThreadsP), smem, st, true, 2, mQ, mAh,
                    mAl, mK, mV, a);
 }
