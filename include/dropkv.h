@@ -175,11 +175,14 @@ DROPKV_API size_t dropkv_select_workspace_bytes(int32_t B, int32_t Hkv, int32_t 
  *   evict_idx    device int32 [B, Hkv, max_evict]: evicted positions ascending,
  *                then -1;  max_evict >= every lengths[b] - keep_counts[b].
  *                (keep_idx / evict_idx may be NULL when max_keep / max_evict is 0.)
- * Asynchronous on `stream`; integer results are exact.  The kernels' waits on
- * one another are bounded; if one gives up, that (b, h)'s keep and evict
- * slots are all filled with -1.  Only dropkv_select_ex reports the timeout
- * itself (DROPKV_ERR_TIMEOUT); this entry point enqueues nothing but the
- * selection kernel and leaves the workspace untouched.
+ * Asynchronous on `stream`; integer results are exact.  The CTAs of a
+ * (b, h)'s cluster meet at hardware cluster barriers that every thread
+ * reaches unconditionally, so the kernel has no wait that can give up; the
+ * failure path (a wait that gives up, its (b, h)'s keep and evict slots all
+ * -1, DROPKV_ERR_TIMEOUT) belongs to the bounded build that
+ * dropkv_selftest_select_timeout runs.  Only dropkv_select_ex reports the
+ * device status itself; this entry point enqueues nothing but the selection
+ * kernel and leaves the workspace untouched.
  */
 DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* scores,
                             const int32_t* lengths, const int32_t* keep_counts,
@@ -188,11 +191,11 @@ DROPKV_API dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, co
                             void* stream);
 
 /* dropkv_select that reports the device-side status.  status_dev NULL: the
- * call synchronises `stream` and returns DROPKV_ERR_TIMEOUT if a bounded wait
- * of the kernels gave up, else DROPKV_OK.  status_dev non-NULL (device int32,
- * 4-byte aligned, caller-owned): asynchronous; the call zeroes *status_dev on
- * the stream and the kernels raise it to DROPKV_ERR_TIMEOUT on a timeout.
- * Host-side errors are returned directly and nothing is enqueued. */
+ * call synchronises `stream` and returns the kernels' status (DROPKV_OK, or
+ * DROPKV_ERR_TIMEOUT from a build with bounded waits).  status_dev non-NULL
+ * (device int32, 4-byte aligned, caller-owned): asynchronous; the call zeroes
+ * *status_dev on the stream and the kernels raise it on an error.  Host-side
+ * errors are returned directly and nothing is enqueued. */
 DROPKV_API dropkv_status dropkv_select_ex(int32_t B, int32_t Hkv, int32_t n_max,
                                           const float* scores, const int32_t* lengths,
                                           const int32_t* keep_counts, int32_t* keep_idx,
@@ -288,10 +291,12 @@ DROPKV_API dropkv_status dropkv_selftest_wait_timeout(int32_t* status_dev, uint6
                                                       void* stream);
 
 /* Self-test of the select kernel's failure path: runs the select of
- * dropkv_select on the given arguments (B <= 64) with one CTA of every
- * segment's cluster withholding its arrivals of the first radix round (so the
- * other CTAs' waits for them run out) and every bounded wait
- * limited to limit_ns nanoseconds (0 < limit_ns <= 1e9).  Every segment with
+ * dropkv_select on the given arguments (B <= 64) in its bounded build (the
+ * radix rounds separated by mbarrier phases with bounded waits instead of
+ * hardware cluster barriers) with one CTA of every segment's cluster
+ * withholding its arrivals of the first radix round (so the other CTAs'
+ * waits for them run out) and every bounded wait limited to limit_ns
+ * nanoseconds (0 < limit_ns <= 1e9).  Every segment with
  * at least one eviction then ends with DROPKV_ERR_TIMEOUT in *status_dev
  * (device int32, zeroed by the call) and all its keep and evict slots set to
  * -1.  Asynchronous on `stream`; no fault or trap is involved and the context
