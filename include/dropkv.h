@@ -222,10 +222,9 @@ DROPKV_API dropkv_status dropkv_select_ex(int32_t B, int32_t Hkv, int32_t n_max,
  *   call enqueues one memset of the array's 4-byte status word on `stream`
  *   before its kernels.  Calls whose work overlaps on the GPU, e.g. on
  *   two streams at once, race and must be serialised by the caller.
- *   A device-side timeout of the kernels' bounded waits is not reported by
- *   this entry point (its status word sits in the shared array); the lists of
- *   the affected (b, h) are then filled with -1.  Use dropkv_select_ex where a
- *   timeout must be detected.
+ *   The kernel's device status is not reported by this entry point (its
+ *   status word sits in the shared array); use dropkv_select_ex where it
+ *   must be read.
  */
 DROPKV_API dropkv_status dropkv_select_noalloc(int32_t B, int32_t Hkv, int32_t n_max,
                                                const float* scores, const int32_t* lengths,
