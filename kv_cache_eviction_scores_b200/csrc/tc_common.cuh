@@ -146,11 +146,20 @@ __device__ __noinline__ float direct_sqdist(const float* A, const __nv_bfloat16*
   return s;
 }
 
+// The ratio p / (1 - p) on the fast path's interval 0 <= p < 2^-4 is p t(p),
+// t the quadratic closest to 1 / (1 - p) in relative error there (minimax):
+// t(p) (1 - p) - 1 is the cubic of least maximum on [0, 2^-4] that takes -1
+// at p = 1, i.e. -T3(32 p - 1) / T3(31) (Chebyshev's extremal property of
+// T3 outside [-1, 1]), so |p t(p) / (p / (1 - p)) - 1| <= 1 / T3(31) =
+// 1 / 119071 = 8.4e-6.  t(p) = (1 - T3(32 p - 1) / T3(31)) / (1 - p) is a
+// quadratic (the numerator vanishes at p = 1); kT0, kT1, kT2 are the fp32
+// roundings of its coefficients.
+constexpr float kT0 = 1.00000834f, kT1 = 0.997589648f, kT2 = 1.10078859f;
+
 // Fast path for 16 query columns of one token (every p < 2^-4, no possible
 // cancellation): packed fp32 pairs,
 //   p = 2^(x c - M'),  M' = M + log2 L,
-//   ratio = p / (1 - p) = p (1 + p (1 + p (1 + p (1 + p)))) + O(p^6)
-//   (relative truncation error p^5 / (1 - p) <= 1.0e-6 for p < 2^-4),
+//   ratio = p / (1 - p) = p t(p) to 8.4e-6 relative (t above),
 //   s += ratio^2 (D' + ||A||^2 + ||v||^2)   with D' = -2 A.v from the MMA.
 // kf holds (-M'_t, -M'_t+1, ||A_t||^2, ||A_t+1||^2) per column pair.
 // kMask: the causal window mask -- column u is the window query at position
@@ -175,8 +184,8 @@ __device__ __forceinline__ void fast16(const uint32_t (&r)[32], const float4* kf
     const float p0 = ex2(y0), p1 = ex2(y1);
     pmax = fmax3(pmax, p0, p1);
     const uint64_t P = pk2(p0, p1);
-    const uint64_t one = pk2(1.f, 1.f);
-    const uint64_t ratio = fmul2(P, ffma2(P, ffma2(P, ffma2(P, fadd2(P, one), one), one), one));
+    const uint64_t ratio =
+        fmul2(P, ffma2(P, ffma2(P, pk2(kT2, kT2), pk2(kT1, kT1)), pk2(kT0, kT0)));
     const uint64_t zt = fadd2(fadd2(pk2(f32(r[16 + 2 * i]), f32(r[16 + 2 * i + 1])),
                                     pk2(k.z, k.w)), nv2);
     acc2 = ffma2(fmul2(ratio, ratio), zt, acc2);

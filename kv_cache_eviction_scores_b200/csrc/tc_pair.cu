@@ -326,7 +326,7 @@ k_tc_pass2_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             fast16<true>(r, kfc, c2, pk2(nv, nv), a2, pmax, tok, L - a.w,
                          (chunk * nqc + hc0 + ch * 16) % a.w, a.w);
           }
-          // a large p (>= 2^-4: the series above would be short) or possible
+          // a large p (>= 2^-4: outside the fast ratio's interval) or possible
           // cancellation (||A||^2 >= 0.6 ||v||^2): the careful path (lanes past
           // L write nothing and do not vote)
           const bool redo = valid && (pmax >= 0.0625f || nAmax[hc0 / 16 + ch] >= 0.6f * nv);

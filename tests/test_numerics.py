@@ -1,8 +1,11 @@
 """Error bounds the tensor-core path relies on, checked by emulating its
 bf16 / fp32 operations in numpy (CPU only).
 
-* Pass 2's fast path replaces p / (1 - p) by p (1 + p (1 + p (1 + p (1 + p))))
-  for p < 2^-4: relative truncation error p^5 <= 2^-20 < 1.0e-6.
+* Pass 2's fast path replaces p / (1 - p) by p t(p) for p < 2^-4, t the
+  minimax quadratic of 1 / (1 - p) in relative error on [0, 2^-4]: relative
+  error <= 1 / T3(31) = 8.4e-6 (ratio^2: 1.7e-5).  The kernel's three
+  coefficients are read from its source and rebuilt here from numpy's
+  Chebyshev polynomials.
 * Pass 1 stores P in [0, 256] as P_hi = P truncated to bf16 plus
   P_lo = bf16_rn(P - P_hi): P to 2^-16 relative.
 * The combine stores -2A as bf16_rn hi + bf16_rn lo: to 2^-16 relative per
@@ -11,7 +14,12 @@ bf16 / fp32 operations in numpy (CPU only).
   distance then moves by at most 2^-7 rho / (1 - rho)^2 <= 2.4e-4 relative.
 """
 
+import os
+import re
+
 import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def bf16_trunc(x):
@@ -35,14 +43,40 @@ def test_bf16_rounding_emulation():
     assert bf16_trunc(np.float32(1.0 + 3 * 2.0 ** -8)) == np.float32(1.0 + 2.0 ** -7)
 
 
-def test_fast_path_series_truncation():
-    p = np.linspace(1e-9, 2.0 ** -4, 200001)
-    series = p * (1 + p * (1 + p * (1 + p * (1 + p))))
+def _kernel_ratio_coefficients():
+    src = open(os.path.join(ROOT, "kv_cache_eviction_scores_b200", "csrc", "tc_common.cuh")).read()
+    m = re.search(r"constexpr float kT0 = ([0-9.]+)f, kT1 = ([0-9.]+)f, kT2 = ([0-9.]+)f;", src)
+    assert m, "the fast ratio's coefficients are not in tc_common.cuh"
+    return np.array([np.float32(float(x)) for x in m.groups()], np.float32)
+
+
+def test_fast_path_ratio_coefficients_are_the_chebyshev_construction():
+    # t(p) (1 - p) = 1 - T3(32 p - 1) / T3(31): numpy's T3 on the domain
+    # [0, 2^-4] is T3(32 p - 1), and p = 1 maps to 31
+    T3 = np.polynomial.Chebyshev.basis(3, domain=[0.0, 2.0 ** -4])
+    assert T3(1.0) == 119071.0
+    num = (1 - T3 / T3(1.0)).convert(kind=np.polynomial.Polynomial)
+    t, rem = divmod(num, np.polynomial.Polynomial([1.0, -1.0]))
+    assert t.degree() == 2 and np.abs(rem.coef).max() < 1e-9
+    assert np.array_equal(t.coef.astype(np.float32), _kernel_ratio_coefficients())
+
+
+def test_fast_path_ratio_error():
+    c = _kernel_ratio_coefficients().astype(np.float64)
+    p = np.linspace(1e-9, 2.0 ** -4, 400001)
+    ratio = p * (c[0] + p * (c[1] + p * c[2]))
     exact = p / (1 - p)
-    rel = np.abs(series - exact) / exact
-    assert rel.max() <= 1.0e-6
-    m = p >= 1e-2  # the error is exactly p^5 (below, fp64 rounding dominates)
-    assert np.allclose(rel[m], p[m] ** 5, rtol=1e-5)
+    rel = np.abs(ratio - exact) / exact
+    assert rel.max() <= 8.5e-6
+    # equioscillation: at the four extrema of T3(32 p - 1) on [0, 2^-4] the
+    # error alternates in sign at (within the coefficients' fp32 rounding)
+    # the bound 1 / 119071
+    pk = (1 + np.cos(np.arange(4) * np.pi / 3)) / 32
+    e = (c[0] + pk * (c[1] + pk * c[2])) * (1 - pk) - 1
+    assert np.all(np.sign(e[:-1]) != np.sign(e[1:]))
+    assert np.allclose(np.abs(e), 1 / 119071, rtol=0.02)
+    # the Taylor quadratic, p (1 + p + p^2), is off by p^3 relative: 2.4e-4 at 2^-4
+    assert rel.max() < 0.1 * (2.0 ** -4) ** 3
 
 
 def test_probability_hi_lo_split():
