@@ -300,13 +300,16 @@ def source_hash(fnames):
     return h.hexdigest()
 
 
-def traffic_for(kernel):
-    """ncu DRAM bytes per launch of `kernel`, if captured on the current source."""
+def traffic_for(kernel, spec):
+    """ncu DRAM bytes per launch of `kernel`, if captured on the current source
+    and on this workload (the stored figure is for one workload's launch)."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
         e = d[kernel]
         if e.get("csrc_sha256") != source_hash(KERNEL_SRC[kernel]):
+            return None
+        if e.get("workload") != workload_desc(spec):
             return None
         return float(e["bytes_per_launch"])
     except Exception:
@@ -324,7 +327,7 @@ def roofline(kernel, spec, us, hbm_peak, tc_peak, sm_mhz, score="perturbation"):
         peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12  # FP32 lanes x FMA x clock, TFLOP/s
         ach = flops / (us * 1e-6) / 1e12
         return {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": traffic_for(kernel),
+                "frac": ach / peak, "traffic": traffic_for(kernel, spec),
                 "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x max SM clock",
                 "work": f"{flops:.4g} flop (4*d per visible element)"}
     if kernel == "k_tc_pass2" and score == "attention":
@@ -349,7 +352,7 @@ def roofline(kernel, spec, us, hbm_peak, tc_peak, sm_mhz, score="perturbation"):
         flops = 2 * 2 * d * elems
         tach = flops / (us * 1e-6) / 1e12
         return {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-                "frac": ach / hbm_peak, "traffic": traffic_for(kernel),
+                "frac": ach / hbm_peak, "traffic": traffic_for(kernel, spec),
                 "work": f"{nbytes} B (one read of the valid K and V rows)",
                 "tensor": {"achieved": tach, "peak": tc_peak, "unit": "TFLOP/s",
                            "frac": tach / tc_peak,
@@ -358,7 +361,7 @@ def roofline(kernel, spec, us, hbm_peak, tc_peak, sm_mhz, score="perturbation"):
     nbytes = valid * 4 * 2
     ach = nbytes / (us * 1e-6) / 1e9
     return {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-            "frac": ach / hbm_peak, "traffic": traffic_for(kernel),
+            "frac": ach / hbm_peak, "traffic": traffic_for(kernel, spec),
             "work": f"{nbytes} B"}
 
 
