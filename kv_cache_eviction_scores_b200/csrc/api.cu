@@ -309,6 +309,7 @@ size_t dropkv_scores_workspace_bytes(const dropkv_shape* shape) {
 dropkv_status dropkv_scores(const dropkv_shape* shape, const void* q, const void* k,
                             const void* v, const int32_t* lengths, float* scores,
                             void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange range("dropkv_scores");
   return run_scores(shape, q, k, v, lengths, scores, workspace, workspace_bytes, stream, nullptr,
                     nullptr, true);
 }
@@ -317,6 +318,7 @@ dropkv_status dropkv_scores_async(const dropkv_shape* shape, const void* q, cons
                                   const void* v, const int32_t* lengths, float* scores,
                                   void* workspace, size_t workspace_bytes, void* stream,
                                   int32_t* status_dev) {
+  NvtxRange range("dropkv_scores_async");
   if (!status_dev) return DROPKV_ERR_ARG;
   return run_scores(shape, q, k, v, lengths, scores, workspace, workspace_bytes, stream,
                     status_dev, nullptr, false);
@@ -326,6 +328,7 @@ dropkv_status dropkv_scores_ex(const dropkv_shape* shape, const void* q, const v
                                const void* v, const int32_t* lengths, float* scores,
                                void* workspace, size_t workspace_bytes, void* stream,
                                int32_t* status_dev, const dropkv_options* options) {
+  NvtxRange range("dropkv_scores_ex");
   return run_scores(shape, q, k, v, lengths, scores, workspace, workspace_bytes, stream,
                     status_dev, options, status_dev == nullptr);
 }
@@ -336,6 +339,7 @@ dropkv_status dropkv_scores_select(const dropkv_shape* shape, const void* q, con
                                    int32_t max_keep, int32_t* evict_idx, int32_t max_evict,
                                    void* workspace, size_t workspace_bytes, void* stream,
                                    int32_t* status_dev, const dropkv_options* options) {
+  NvtxRange range("dropkv_scores_select");
   if (!shape) return DROPKV_ERR_ARG;
   const SelectSpec sel = {keep_counts, keep_idx, max_keep, evict_idx, max_evict};
   return run_scores(shape, q, k, v, lengths, scores, workspace, workspace_bytes, stream,
@@ -381,6 +385,7 @@ dropkv_status dropkv_select(int32_t B, int32_t Hkv, int32_t n_max, const float* 
                             int32_t* keep_idx, int32_t max_keep, int32_t* evict_idx,
                             int32_t max_evict, void* workspace, size_t workspace_bytes,
                             void* stream) {
+  NvtxRange range("dropkv_select");
   return select_entry(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx, max_keep, evict_idx,
                       max_evict, workspace, workspace_bytes, stream, nullptr, false);
 }
@@ -390,6 +395,7 @@ dropkv_status dropkv_select_ex(int32_t B, int32_t Hkv, int32_t n_max, const floa
                                int32_t* keep_idx, int32_t max_keep, int32_t* evict_idx,
                                int32_t max_evict, void* workspace, size_t workspace_bytes,
                                void* stream, int32_t* status_dev) {
+  NvtxRange range("dropkv_select_ex");
   return select_entry(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx, max_keep, evict_idx,
                       max_evict, workspace, workspace_bytes, stream, status_dev,
                       status_dev == nullptr);

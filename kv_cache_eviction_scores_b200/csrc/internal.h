@@ -2,12 +2,24 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stddef.h>
 #include <stdint.h>
 
 #include "dropkv.h"
 
 namespace dropkv {
+
+// An NVTX range named after a C entry point, held over its argument checks
+// and launches, so that a timeline tool (or ncu's --nvtx-include filter) can
+// attribute the kernels to the call.  NVTX is header-only: with no tool
+// attached a push / pop pair is a call through a no-op function pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Batch rows handled per launch; larger batches are processed in slices.
 constexpr int kMaxB = 64;

@@ -64,6 +64,7 @@ extern "C" dropkv_status dropkv_select_noalloc(int32_t B, int32_t Hkv, int32_t n
                                                const int32_t* keep_counts, int32_t* keep_idx,
                                                int32_t max_keep, int32_t* evict_idx,
                                                int32_t max_evict, void* stream) {
+  NvtxRange range("dropkv_select_noalloc");
   dropkv_status r = check_select_args(B, Hkv, n_max, scores, lengths, keep_counts, keep_idx,
                                       max_keep, evict_idx, max_evict);
   if (r != DROPKV_OK) return r;
