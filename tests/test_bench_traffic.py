@@ -1,6 +1,9 @@
-"""The bench's stored ncu DRAM traffic is reported only where it applies: on the
-kernel sources it was captured on (comment edits aside) and on the workload
-whose launch it measured.  Host logic only (no GPU)."""
+"""The bench's roofline bookkeeping, host logic only (no GPU): the stored ncu
+DRAM traffic is reported only where it applies (the kernel sources it was
+captured on, comment edits aside, and the workload whose launch it measured),
+and the algorithmic bytes and flops of a pass follow their definitions (one
+read of K and V; 4 d flop per visible (token, query) pair, counted here by
+brute force)."""
 
 import json
 import os
@@ -53,3 +56,27 @@ def test_stored_traffic_names_its_workload():
         assert kernel in bench.KERNEL_SRC
         assert e["workload"] == bench.workload_desc(W.config_spec(3))
         assert e["bytes_per_launch"] == e["dram_read"] + e["dram_write"]
+
+
+def test_visible_elements_by_brute_force():
+    # window query i (0-based) sits at position L - w + i and sees tokens 0 .. L - w + i
+    spec = W.Spec("tiny", B=2, Hq=4, Hkv=2, d=8, lengths=[9, 13], window=3, pool=1,
+                  keep=[2, 3], dtype="f32")
+    brute = 0
+    for L in spec.lengths:
+        for i in range(spec.window):
+            brute += sum(1 for j in range(L) if j <= L - spec.window + i)
+    assert bench.visible_elements(spec) == brute * spec.Hq
+
+
+def test_roofline_of_a_tensor_pass():
+    spec = W.config_spec(3)
+    us = 200.0
+    r = bench.roofline("k_tc_pass2_pair", spec, us, 6650.0, 1590.0, 1965.0)
+    nbytes = sum(spec.lengths) * spec.Hkv * spec.d * 2 * 2  # one read of K and V, bf16
+    assert nbytes == 536870912
+    assert abs(r["achieved"] - nbytes / (us * 1e-6) / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6650.0) < 1e-12
+    flops = 4 * spec.d * bench.visible_elements(spec)
+    assert abs(r["tensor"]["achieved"] - flops / (us * 1e-6) / 1e12) < 1e-9
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
